@@ -1,0 +1,353 @@
+"""Pins for the oracle's codec: octahedral map, indexing, joint rounding,
+packing, codec quality against the pages' printed numbers, logits, attention
+and the QJL sketch."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, baselines, codec, tables
+from rotation_preconditioned_quantization_b200 import inputs
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _unit(seed, n):
+    v = inputs.normal(seed, (n, 3), np.float64)
+    return v / np.linalg.norm(v, axis=1, keepdims=True)
+
+
+# ---------------------------------------------------------------- octahedral
+def test_octahedral_round_trip():
+    n = _unit(1, 1_000_000)
+    xi, eta = codec.oct_forward(n)
+    assert np.all(np.abs(xi) <= 1) and np.all(np.abs(eta) <= 1)
+    back = codec.oct_inverse(xi, eta)
+    assert np.max(np.abs(back - n)) < 1e-12
+    # upper hemisphere <-> inside the diamond
+    inside = np.abs(xi) + np.abs(eta) <= 1 + 1e-15
+    assert np.array_equal(inside, n[:, 2] >= 0) or np.mean(inside != (n[:, 2] >= 0)) < 1e-5
+
+
+def test_octahedral_special_points():
+    pts = np.array([[0, 0, 1], [0, 0, -1], [1, 0, 0], [-1, 0, 0], [0, 1, 0], [0, -1, 0],
+                    [1, 1, -1e-300], [0.0, 0.0, 0.0]], float)
+    xi, eta = codec.oct_forward(pts)
+    want = np.array([[0, 0], [1, 1], [1, 0], [-1, 0], [0, 1], [0, -1], [0, 0], [0, 0]], float)
+    got = np.stack([xi, eta], axis=1)
+    assert np.allclose(got[:6], want[:6], atol=0)
+    # a point just below the equator on the x=y diagonal folds to the square's centre
+    assert np.allclose(got[6], [0.5 * 0 + 0.0, 0.0], atol=1e-12) or np.allclose(got[6], [0.5, 0.5], atol=1e-12)
+    assert np.array_equal(got[7], [0.0, 0.0])
+    # corners of the square are the south pole, centre the north pole
+    assert np.allclose(codec.oct_inverse(np.array([1.0, -1, 1, -1]), np.array([1.0, 1, -1, -1])),
+                       np.tile([0, 0, -1.0], (4, 1)), atol=1e-15)
+    assert np.allclose(codec.oct_inverse(0.0, 0.0), [0, 0, 1.0])
+
+
+def test_octahedral_by_hand():
+    # n = (1, 2, 2)/3 : l1 = 5/3 -> p = (0.2, 0.4, 0.4), upper: (0.2, 0.4)
+    xi, eta = codec.oct_forward(np.array([1.0, 2.0, 2.0]) / 3)
+    assert abs(xi - 0.2) < 1e-15 and abs(eta - 0.4) < 1e-15
+    # n = (1, -2, -2)/3 : p = (0.2, -0.4, -0.4), lower: ((1-0.4)*1, (1-0.2)*(-1)) = (0.6, -0.8)
+    xi, eta = codec.oct_forward(np.array([1.0, -2.0, -2.0]) / 3)
+    assert abs(xi - 0.6) < 1e-15 and abs(eta + 0.8) < 1e-15
+    # inverse of (0.6, -0.8): r = -0.4 -> v = ((1-0.8), -(1-0.6), -0.4) = (0.2, -0.4, -0.4)
+    v = codec.oct_inverse(0.6, -0.8)
+    assert np.allclose(v, np.array([1.0, -2.0, -2.0]) / 3, atol=1e-15)
+
+
+# ---------------------------------------------------------------- indexing
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_scalar_index_is_nearest_centroid(b):
+    c, t = tables.direction_codebook(b)
+    x = inputs.rng(b).uniform(-1, 1, 100000)
+    idx = codec.scalar_index(x, t)
+    brute = np.argmin(np.abs(x[:, None] - c[None, :]), axis=1)
+    assert np.array_equal(idx, brute)
+    # a value exactly on a threshold goes to the upper cell
+    assert np.array_equal(codec.scalar_index(t, t), np.arange(1, len(c)))
+
+
+def _rot_triplets(seed, n, d=128):
+    k = inputs.gaussian_keys(seed, 1, n, d)[0].astype(np.float64)
+    s = tables.rotation_signs(seed, d, 1)[0]
+    u = k / np.linalg.norm(k, axis=1, keepdims=True)
+    return codec.triplets(codec.rotate(u, s))[:, : d // 3].reshape(-1, 3)
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_joint_rounding_equals_exhaustive(b):
+    """[EXPL] "joint rounding": the 3x3 search matched exhaustive search on 10 000 triplets."""
+    g = _gold("synthetic_quality.json")["joint_3x3_equals_exhaustive"]
+    d = 128
+    dc, dt, rc, rt = tables.codebooks(d, b)
+    t = _rot_triplets(40 + b, 240)[: g["triplets"]]
+    t = np.concatenate([t, _rot_triplets(90 + b, 240)])[: g["triplets"]]
+    assert len(t) == g["triplets"]
+    xi, eta = codec.oct_forward(t)
+    _, _, _, ej = codec.joint_round(t, codec.scalar_index(xi, dt), codec.scalar_index(eta, dt), dc, rc, rt)
+    _, _, _, ee = codec.exhaustive_round(t, dc, rc)
+    assert np.max(ej - ee) < 1e-15
+
+
+def test_joint_rounding_tiny_brute_force():
+    """Hand-checkable case: 2 direction levels... via a full enumeration on random triplets."""
+    dc = np.array([-0.5, 0.5])
+    rc = np.array([0.1, 0.3])
+    rt = np.array([0.2])
+    t = inputs.normal(5, (500, 3), np.float64) * 0.2
+    xi, eta = codec.oct_forward(t)
+    ix, iy, ir, e = codec.joint_round(t, codec.scalar_index(xi, [0.0]), codec.scalar_index(eta, [0.0]), dc, rc, rt)
+    bx, by, br, be = codec.exhaustive_round(t, dc, rc)
+    assert np.max(np.abs(e - be)) < 1e-15
+    # the error formula is ||t - rho_hat n_hat||^2
+    nh = codec.oct_inverse(dc[ix], dc[iy])
+    assert np.max(np.abs(np.sum((t - rc[ir][:, None] * nh) ** 2, axis=1) - e)) < 1e-15
+
+
+def test_joint_rho_is_nearest_to_projection():
+    """For a fixed direction the best rho level is the one nearest s = n_hat . t."""
+    d, b = 128, 3
+    dc, dt, rc, rt = tables.codebooks(d, b)
+    t = _rot_triplets(3, 50)
+    xi, eta = codec.oct_forward(t)
+    ix, iy = codec.scalar_index(xi, dt), codec.scalar_index(eta, dt)
+    nh = codec.oct_inverse(dc[ix], dc[iy])
+    errs = np.stack([np.sum((t - r * nh) ** 2, axis=1) for r in rc], axis=1)
+    s = np.sum(nh * t, axis=1)
+    assert np.array_equal(np.argmin(errs, axis=1), np.argmin(np.abs(s[:, None] - rc[None, :]), axis=1))
+
+
+# ---------------------------------------------------------------- packing
+def test_pack_by_hand():
+    # b=2: c = 7 bits; triplet codes 93 (xi 5, eta 3, rho 1) and 71 (xi 7, eta 0, rho 1)
+    lay = codec.Layout(6, 2)
+    w = codec.pack(np.array([[5, 7]]), np.array([[3, 0]]), np.array([[1, 1]]), lay)
+    assert lay.words == 1 and int(w[0, 0]) == 93 + (71 << 7)
+    # b=4: c = 13 bits; the third code crosses into word 1
+    lay = codec.Layout(9, 4)
+    code = [0x1ABC, 0x0F0F, 0x1FFF]
+    ix = np.array([[v & 31 for v in code]])
+    iy = np.array([[(v >> 5) & 31 for v in code]])
+    ir = np.array([[(v >> 10) & 7 for v in code]])
+    w = codec.pack(ix, iy, ir, lay)
+    assert lay.words == 2
+    assert int(w[0, 0]) == (0x1ABC | (0x0F0F << 13) | ((0x1FFF & 63) << 26))
+    assert int(w[0, 1]) == 0x1FFF >> 6
+
+
+@pytest.mark.parametrize("d,b", [(64, 2), (128, 3), (128, 4), (256, 2), (256, 4)])
+def test_pack_round_trip_and_sizes(d, b):
+    lay = codec.Layout(d, b)
+    assert lay.code_bits == 3 * b + 1
+    assert lay.words == math.ceil(lay.T * (3 * b + 1) / 32)
+    ix = inputs.random_codes(1, (7, lay.T), lay.n_dir)
+    iy = inputs.random_codes(2, (7, lay.T), lay.n_dir)
+    ir = inputs.random_codes(3, (7, lay.T), lay.n_rho)
+    w = codec.pack(ix, iy, ir, lay)
+    # bit-by-bit reference of the stream
+    for r in range(7):
+        stream = 0
+        for i in range(lay.T):
+            stream |= (int(ix[r, i]) | int(iy[r, i]) << lay.b_dir | int(ir[r, i]) << 2 * lay.b_dir) << (i * lay.code_bits)
+        assert [int(x) for x in w[r]] == [(stream >> (32 * j)) & 0xFFFFFFFF for j in range(lay.words)]
+    a, bb, c = codec.unpack(w, lay)
+    assert np.array_equal(a, ix) and np.array_equal(bb, iy) and np.array_equal(c, ir)
+
+
+# ---------------------------------------------------------------- quality
+def _mse(d, b, mode, reps=4, n=1024, dir_bits=None, rho_bits=None):
+    if dir_bits is None:
+        dc, dt, rc, rt = tables.codebooks(d, b)
+    else:
+        # the sweep's MSE (second order in centroid errors) needs codebooks to ~1e-7, not to the 1e-13 of the shipped tables
+        dc, dt = tables.direction_codebook_levels(1 << dir_bits, 1e-7)
+        rc, rt = tables.rho_codebook_levels(d, 1 << rho_bits, 1e-7)
+    lay = codec.Layout(d, b)
+    out = []
+    for rep in range(reps):
+        k = inputs.gaussian_keys(1000 + rep, 1, n, d)[0].astype(np.float64)
+        s = tables.rotation_signs(rep, d, 1)[0]
+        u = k / np.linalg.norm(k, axis=1, keepdims=True)
+        t = codec.triplets(codec.rotate(u, s))
+        xi, eta = codec.oct_forward(t)
+        ix, iy = codec.scalar_index(xi, dt), codec.scalar_index(eta, dt)
+        if mode == codec.SCALAR:
+            ir = codec.scalar_index(np.linalg.norm(t, axis=-1), rt)
+        else:
+            ix, iy, ir, _ = codec.joint_round(t, ix, iy, dc, rc, rt)
+        nh = codec.oct_inverse(dc[ix], dc[iy])
+        ur = (rc[ir][..., None] * nh).reshape(n, -1)[:, :d]
+        uh = ur @ codec.rotation_matrix(s)
+        out.append(np.mean(np.sum((u - uh) ** 2, axis=1)))
+    return float(np.mean(out))
+
+
+@pytest.mark.parametrize("b", [2, 4])
+def test_mse_matches_printed_values(b):
+    g = _gold("synthetic_quality.json")["mse"]
+    printed = g[f"octopus_b{b}"]
+    scalar = _mse(128, b, codec.SCALAR)
+    joint = _mse(128, b, codec.JOINT)
+    assert abs(scalar - printed) < 0.03 * printed
+    assert abs(joint - printed) < 0.10 * printed
+    assert joint < scalar
+
+
+def test_per_coordinate_baseline_matches_printed_value():
+    g = _gold("synthetic_quality.json")["mse"]
+    k = inputs.gaussian_keys(1000, 1, 1024, 128)[0].astype(np.float64)
+    u = k / np.linalg.norm(k, axis=1, keepdims=True)
+    m = baselines.per_coordinate_mse(u, tables.rotation_signs(0, 128, 1)[0], 4)
+    assert abs(m - g["turboquant_mse_b4"]) < 0.03 * g["turboquant_mse_b4"]
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_octopus_beats_per_coordinate_lloyd_max(b):
+    k = inputs.gaussian_keys(1000, 1, 1024, 128)[0].astype(np.float64)
+    u = k / np.linalg.norm(k, axis=1, keepdims=True)
+    base = baselines.per_coordinate_mse(u, tables.rotation_signs(0, 128, 1)[0], b)
+    assert _mse(128, b, codec.JOINT, reps=1) < base
+
+
+@pytest.mark.parametrize("b", [3, 4])
+def test_bit_allocation_sweep(b):
+    """[EXPL] "non-uniform bit allocation": delta=+1 is best; +2 is 44-73% worse than 0; -1 >200% worse."""
+    g = _gold("synthetic_quality.json")["delta_sweep"]
+    m = {dl: _mse(128, b, codec.JOINT, reps=1, dir_bits=b + dl, rho_bits=b - dl) for dl in (-1, 0, 1, 2)}
+    assert min(m, key=m.get) == g["best_delta"]
+    gain = 100 * (1 - m[1] / m[0])
+    lo, hi = g["gain_delta_plus1_vs_0_percent"]
+    assert lo - 10 <= gain <= hi + 10
+    assert 100 * (m[-1] / m[0] - 1) > g["loss_delta_minus1_vs_0_percent_min"]
+    lo, hi = g["loss_delta_plus2_vs_0_percent"]
+    assert lo - 10 <= 100 * (m[2] / m[0] - 1) <= hi + 10
+
+
+def test_zero_key():
+    d, b = 128, 3
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    e = codec.encode(np.zeros((2, d)), tables.rotation_signs(0, d, 1)[0], tb, lay)
+    assert np.array_equal(e.gamma, [0.0, 0.0])
+    L = lay.n_dir
+    assert np.all(e.i_xi == L // 2) and np.all(e.i_eta == L // 2) and np.all(e.i_rho == 0)
+
+
+def test_encode_matches_stepwise_definition():
+    d, b = 128, 3
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    s = tables.rotation_signs(2, d, 1)[0]
+    k = inputs.llm_keys(4, 1, 300, d)[0].astype(np.float64)
+    e = codec.encode(k, s, tb, lay, codec.SCALAR)
+    # independent restatement with explicit loops on a few keys
+    H = np.array([[(-1) ** bin(i & j).count("1") for j in range(d)] for i in range(d)], float)
+    for r in range(0, 300, 37):
+        g = math.sqrt(sum(x * x for x in k[r]))
+        assert abs(g - e.gamma[r]) < 1e-12 * g
+        ur = H @ (s * k[r] / g) / math.sqrt(d)
+        ur = list(ur) + [0.0] * (3 * lay.T - d)
+        for i in range(lay.T):
+            t = ur[3 * i: 3 * i + 3]
+            l1 = sum(abs(x) for x in t)
+            p = [x / l1 for x in t]
+            if p[2] >= 0:
+                xi, eta = p[0], p[1]
+            else:
+                xi = (1 - abs(p[1])) * (1 if p[0] >= 0 else -1)
+                eta = (1 - abs(p[0])) * (1 if p[1] >= 0 else -1)
+            assert e.i_xi[r, i] == int(np.argmin(np.abs(tb[0] - xi)))
+            assert e.i_eta[r, i] == int(np.argmin(np.abs(tb[0] - eta)))
+            rho = math.sqrt(sum(x * x for x in t))
+            assert e.i_rho[r, i] == int(np.argmin(np.abs(tb[2] - rho)))
+
+
+# ---------------------------------------------------------------- logits / attention
+def test_logits_materialised_equals_rotated_query_route():
+    d, b = 128, 3
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    s = tables.rotation_signs(9, d, 1)[0]
+    k = inputs.llm_keys(1, 1, 500, d)[0]
+    q = inputs.normal(2, (4, d), np.float64)
+    e = codec.encode(k, s, tb, lay)
+    lg = attention.logits(q, e.gamma, e.i_xi, e.i_eta, e.i_rho, s, tb, lay)
+    ur = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, lay)
+    lg2 = (codec.rotate(q, s) @ ur.T) * e.gamma[None, :]
+    assert np.max(np.abs(lg - lg2)) < 1e-12 * np.max(np.abs(lg))
+
+
+def test_attention_identity_codec_equals_sdpa():
+    G, N, d = 4, 300, 64
+    q = inputs.normal(1, (G, d), np.float64)
+    K = inputs.normal(2, (N, d), np.float64)
+    V = inputs.to_bf16(inputs.normal(3, (N, d))).astype(np.float64)
+    out = attention.softmax_attention(q @ K.T, V, 1.0 / math.sqrt(d))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0].numpy()
+    assert np.max(np.abs(out - ref)) < 1e-13
+
+
+def test_attention_of_decoded_keys_equals_sdpa_on_materialised_keys():
+    d, b = 64, 2
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    s = tables.rotation_signs(1, d, 1)[0]
+    k = inputs.gaussian_keys(5, 1, 200, d)[0]
+    V = inputs.to_bf16(inputs.normal(6, (200, d))).astype(np.float64)
+    q = inputs.normal(7, (8, d), np.float64)
+    e = codec.encode(k, s, tb, lay)
+    out, _ = attention.decode_attention(q, e.gamma, e.i_xi, e.i_eta, e.i_rho, V, s, tb, lay)
+    kh = codec.decode_keys(e.gamma, e.i_xi, e.i_eta, e.i_rho, s, tb, lay)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(kh)[None], torch.from_numpy(V)[None])[0].numpy()
+    assert np.max(np.abs(out - ref)) < 1e-13
+
+
+# ---------------------------------------------------------------- QJL
+def test_qjl_estimator_is_unbiased_over_seeds():
+    """[EXPL] "optional residual correction": the sketch makes the inner-product estimate unbiased."""
+    d, b = 64, 2
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    s = tables.rotation_signs(0, d, 1)[0]
+    k = inputs.gaussian_keys(8, 1, 4, d)[0].astype(np.float64)
+    q = inputs.normal(9, (1, d), np.float64)
+    e = codec.encode(k, s, tb, lay)
+    ur_hat = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, lay)
+    q_rot = codec.rotate(q, s)
+    exact = (q @ k.T)[0]
+    base = e.gamma * (q_rot @ ur_hat.T)[0]
+    ests = []
+    for seed in range(2000):
+        S = tables.qjl_matrix(10_000 + seed, d, 1)[0]
+        bits, nu, _ = codec.qjl_encode(e.u_rot, ur_hat, S)
+        ests.append(base + e.gamma * codec.qjl_correction(q_rot, bits, nu, S)[0])
+    ests = np.array(ests)
+    mean = ests.mean(axis=0)
+    se = ests.std(axis=0) / math.sqrt(len(ests))
+    assert np.all(np.abs(mean - exact) < 4 * se + 1e-12)
+    # the base estimate is biased by more than the corrected one's noise for some key
+    assert np.max(np.abs(base - exact)) > np.max(4 * se)
+    # error shrinks like 1/sqrt(seeds)
+    half = np.abs(ests[:500].mean(axis=0) - exact)
+    assert np.all(half < 4 * ests.std(axis=0) / math.sqrt(500) + 1e-12)
+
+
+def test_qjl_pack_round_trip():
+    bits = inputs.random_codes(4, (5, 128), 2)
+    w = codec.qjl_pack(bits)
+    assert w.shape == (5, 4)
+    assert np.array_equal(codec.qjl_unpack(w, 128), bits)
+    assert int(w[0, 0]) == sum(int(bits[0, j]) << j for j in range(32))
