@@ -1,0 +1,380 @@
+"""Benchmark of the OCTOPUS codec on B200: encode + fused decode attention.
+
+Workload (one GPU): LLM-shaped decode - batch 1, 32 query heads over 8 KV
+heads (GQA 4), head_dim 128, context 32768, bf16 keys (N(0,1), four outlier
+channels x10, per-token lognormal(0, 0.5) scale), bf16 V and q ~ N(0,1),
+b = 3, joint rounding. One step = encode the prefill cache (8 x 32768 keys)
++ one fused decode-attention step (32 query heads over the whole cache).
+
+Timing: CUDA events on the launching stream around each kernel; the step
+loop is bracketed by a barrier and a device synchronize; the max over ranks
+is reported. L2 (126 MB): inputs rotate over 3 independent copies of the
+workload (~150 MB each) and each step decodes the cache that the previous
+step encoded, so no decode input was touched within the last ~150 MB of
+traffic. Primary metric: decode-attention achieved HBM GB/s over the
+algorithmic bytes (packed codes + gamma + bf16 V + q + out); encode is
+reported in Mkeys/s.
+
+``--impl reference`` times the CPU oracle (the plain float64 restatement of
+the method) on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+# workload
+B, HQ, HKV, D, N, BITS = 1, 32, 8, 128, 32768, 3
+SEED = 0
+WORKLOAD = "llm-decode: B=1, Hq=32, Hkv=8 (GQA 4), d=128, ctx=32768, bf16 K/V/q, b=3 joint"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j.get("hbm_gbs", 6650.0)), "measured"
+    return 6650.0, "fallback"
+
+
+def _bytes_decode(words):
+    units = B * HKV * N
+    per_unit = 4 * words + 4 + 2 * D            # packed words + gamma + bf16 V row
+    return units * per_unit + B * HQ * D * 2 + B * HQ * D * 4   # + q (bf16) + out (fp32)
+
+
+def _bytes_encode(words):
+    return B * HKV * N * (2 * D + 4 * words + 4)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist_init():
+    import torch
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_baseline(kv_heads: int = 1, tokens: int = N):
+    """Time the CPU oracle on a bounded sample: oracle encode + decode attention of
+    ``kv_heads`` KV heads (4 query heads each) over ``tokens`` tokens."""
+    from oracle import attention, codec, tables
+    from rotation_preconditioned_quantization_b200 import inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    tb = tables.as_f32(*tables.codebooks(D, BITS))
+    lay = codec.Layout(D, BITS)
+    signs = tables.rotation_signs(SEED, D, HKV)
+    keys = inputs.to_bf16(inputs.llm_keys(SEED + 1, kv_heads, tokens, D))
+    V = inputs.to_bf16(inputs.normal(SEED + 3, (kv_heads, tokens, D)))
+    q = inputs.to_bf16(inputs.normal(SEED + 2, (kv_heads, HQ // HKV, D)))
+    t0 = time.perf_counter()
+    encs = [codec.encode(keys[h].astype(np.float64), signs[h], tb, lay) for h in range(kv_heads)]
+    t1 = time.perf_counter()
+    for h in range(kv_heads):
+        e = encs[h]
+        attention.decode_attention(q[h].astype(np.float64), e.gamma, e.i_xi, e.i_eta, e.i_rho,
+                                   V[h].astype(np.float64), signs[h], tb, lay)
+    t2 = time.perf_counter()
+    per_unit = 4 * lay.words + 4 + 2 * D
+    dec_bytes = kv_heads * tokens * per_unit + kv_heads * (HQ // HKV) * D * 6
+    return {
+        "value": dec_bytes / (t2 - t1) / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+        "sample": f"{kv_heads} KV head(s) x {tokens} tokens (of {HKV} x {N}); oracle float64 numpy",
+        "encode_mkeys_per_s": kv_heads * tokens / (t1 - t0) / 1e6,
+        "encode_s": t1 - t0, "decode_s": t2 - t1,
+    }
+
+
+def run_reference(args):
+    ws, rank, _ = _dist_init()
+    if rank != 0:
+        return 0
+    tokens = 4096
+    steps = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(1, tokens)
+        if i >= args.warmup:
+            steps.append(r)
+    dec_s = float(np.mean([s["decode_s"] for s in steps]))
+    enc_s = float(np.mean([s["encode_s"] for s in steps]))
+    val = float(np.mean([s["value"] for s in steps]))
+    line = {
+        "impl": "reference", "metric": "decode-attention HBM GB/s (encode Mkeys/s alongside)", "value": val,
+        "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * (dec_s + enc_s), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": f"1 KV head x {tokens} tokens per step"},
+        "encode_mkeys_per_s": float(np.mean([s["encode_mkeys_per_s"] for s in steps])),
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": steps[0]["cores"], "kind": "oracle",
+                         "sample": steps[0]["sample"]},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_gpu(args):
+    import torch
+    from rotation_preconditioned_quantization_b200 import api, inputs
+
+    ws, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lay = api.Layout(D, BITS)
+    tabs = api.DeviceTables.build(lay, SEED, HKV, device=dev)
+    n_copies = 3
+
+    # inputs: distinct per copy and per rank
+    def make(copy):
+        s = SEED + 1000 * rank + 10 * copy
+        keys = torch.from_numpy(inputs.llm_keys(s + 1, B * HKV, N, D)).to(torch.bfloat16)
+        V = torch.from_numpy(inputs.normal(s + 3, (B * HKV, N, D))).to(torch.bfloat16)
+        q = torch.from_numpy(inputs.normal(s + 2, (B, HQ, 1, D))).to(torch.bfloat16)
+        return keys, V, q
+
+    host = [make(c) for c in range(n_copies)]
+    devc = []
+    for keys, V, q in host:
+        devc.append(dict(keys=keys.to(dev), V=V.to(dev), q=q.to(dev), cache=api.Cache.empty(lay, B * HKV, N, dev),
+                         out=torch.empty((B, HQ, 1, D), dtype=torch.float32, device=dev)))
+    wsp = api.Workspace(api.decode_attn_workspace_bytes(lay, B, HQ, HKV, 1, N), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        c_enc = devc[i % n_copies]
+        c_dec = devc[(i - 1) % n_copies]
+        if ev is not None:
+            ev[0].record(stream)
+        api.encode(lay, tabs, c_enc["keys"], c_enc["cache"], 0)
+        if ev is not None:
+            ev[1].record(stream)
+        api.decode_attn(lay, tabs, c_dec["q"], c_dec["cache"], c_dec["V"], HKV, kv_len=N, out=c_dec["out"],
+                        workspace=wsp)
+        if ev is not None:
+            ev[2].record(stream)
+
+    # prime: every copy's cache encoded once, then warm-up steps
+    for c in range(n_copies):
+        api.encode(lay, tabs, devc[c]["keys"], devc[c]["cache"], 0)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    _barrier(ws)
+    total_ms = t_start.elapsed_time(t_end)
+    enc_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    launches = 2 * args.steps
+
+    total_ms_max = _max_over_ranks(total_ms, ws)
+    dec_sum_max = _max_over_ranks(float(np.sum(dec_ms)), ws)
+    enc_sum_max = _max_over_ranks(float(np.sum(enc_ms)), ws)
+    dbytes = _bytes_decode(lay.words)
+    ebytes = _bytes_encode(lay.words)
+    value = ws * dbytes * args.steps / (dec_sum_max * 1e-3) / 1e9
+    enc_mkeys = ws * B * HKV * N * args.steps / (enc_sum_max * 1e-3) / 1e6
+
+    # end to end through the public API from pinned host buffers
+    hk, hV, hq = (t.pin_memory() for t in host[0])
+    hout = torch.empty((B, HQ, 1, D), dtype=torch.float32).pin_memory()
+    e2e_cache = api.Cache.empty(lay, B * HKV, N, dev)
+    dk = torch.empty_like(hk, device=dev)
+    dV = torch.empty_like(hV, device=dev)
+    dq = torch.empty_like(hq, device=dev)
+    dout = torch.empty((B, HQ, 1, D), dtype=torch.float32, device=dev)
+
+    def e2e_step():
+        dk.copy_(hk, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        dq.copy_(hq, non_blocking=True)
+        api.encode(lay, tabs, dk, e2e_cache, 0)
+        api.decode_attn(lay, tabs, dq, e2e_cache, dV, HKV, kv_len=N, out=dout, workspace=wsp)
+        hout.copy_(dout, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    _barrier(ws)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), ws)
+    h2d = hk.numel() * 2 + hV.numel() * 2 + hq.numel() * 2
+    d2h = hout.numel() * 4
+    e2e_val = ws * dbytes * args.steps / (e2e_ms * 1e-3) / 1e9
+
+    peak, peak_kind = _peaks()
+    dec_avg_s = float(np.mean(dec_ms)) * 1e-3
+    achieved = dbytes / dec_avg_s / 1e9
+    traffic = _ncu_traffic()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "decode-attention HBM GB/s (encode Mkeys/s alongside)",
+        "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "per_rank": "independent batch per GPU (no collective)",
+                   "l2": "3 rotating input copies (~150 MB each > 126 MB L2); decode reads the cache encoded one step earlier"},
+        "encode_mkeys_per_s": enc_mkeys,
+        "encode_ms": float(np.mean(enc_ms)), "decode_ms": float(np.mean(dec_ms)),
+        "decode_bytes_per_step": dbytes, "encode_bytes_per_step": ebytes,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": "octo_decode_attn",
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6650 GB/s"},
+        "encode_roofline": {"bound": "hbm", "achieved": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9, "peak": peak,
+                            "unit": "GB/s", "frac": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9 / peak},
+        "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and ws == 1:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(1, N).items() if k not in ("encode_s", "decode_s")}
+    print(json.dumps(line))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def _ncu_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it matches the current kernel."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return j.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="octopus", choices=["octopus", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,83 @@
+// Device helpers shared by the encode and decode kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/octopus.h"
+
+namespace octo {
+
+constexpr int kWarp = 32;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Walsh-Hadamard butterflies (Sylvester order) on a vector of D values held
+// E = D/32 per lane, lane l owning coordinates [l*E, l*E + E). Unnormalised.
+// The explainer ("engineering implementation") describes the encoder's WHT as
+// an in-place Kronecker-factored butterfly: here the E-point factor runs in
+// registers and the 32-point factor across lanes with shuffles.
+template <int E>
+__device__ __forceinline__ void fwht_warp(float (&v)[E], int lane) {
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if ((e & h) == 0) {
+        const float a = v[e], b = v[e + h];
+        v[e] = a + b;
+        v[e + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
+      v[e] = upper ? (o - v[e]) : (v[e] + o);
+    }
+  }
+}
+
+// Inverse octahedral map of (a, b) = (xi, eta), normalised (explainer,
+// "octahedral folding": r = 1 - |xi| - |eta|; unfold when r < 0; normalise).
+__device__ __forceinline__ float3 oct_inverse(float a, float b) {
+  const float r = 1.0f - fabsf(a) - fabsf(b);
+  float x = a, y = b;
+  if (r < 0.0f) {
+    x = copysignf(1.0f - fabsf(b), a);
+    y = copysignf(1.0f - fabsf(a), b);
+    // sgn(0) = +1 (copysignf keeps +0's positive sign; -0 cannot reach here
+    // from a centroid table)
+  }
+  const float inv = 1.0f / sqrtf(x * x + y * y + r * r);
+  return make_float3(x * inv, y * inv, r * inv);
+}
+
+// Number of entries of the increasing array t[0..n) that are <= x.
+__device__ __forceinline__ int count_le(const float* t, int n, float x) {
+  int lo = 0, hi = n;  // answer in [lo, hi]
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (t[mid] <= x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+}  // namespace octo

@@ -1,0 +1,347 @@
+// OCTOPUS key encoder for sm_100a.
+//
+// Per key (explainer, "triplet decomposition"): gamma = ||k|| (fp32),
+// u = k / gamma; rotate u by the sign-flipped Walsh-Hadamard transform
+// (section "rotation"); cut the rotated direction into triplets, zero-padded
+// at the end; per triplet take rho = ||t|| and the octahedral coordinates
+// (xi, eta) of its direction (section "octahedral folding"); index xi and eta
+// with the (b+1)-bit codebook and rho with the (b-1)-bit codebook, then (by
+// default) refine by the 3x3 joint search of section "joint rounding"; pack
+// the (3b+1)-bit codes into the key's bit stream. With OCTOPUS-QJL (section
+// "optional residual correction") also store sign(S e) and ||e|| for the
+// rotated residual e = u_rot - u_rot_hat.
+//
+// Kernel structure: a persistent grid walks tiles of KT consecutive tokens
+// of one head. Phase 1: one warp per key - coalesced vector loads, norm by
+// warp reduction, sign flip, WHT butterflies in registers + shuffles; the
+// rotated direction goes to shared memory. Phase 2: one thread per triplet
+// over the whole tile (balanced whatever T is) - octahedral map, indexing,
+// joint search against a shared-memory table of decoded unit directions.
+// Phase 3: one thread per (key, word) assembles the packed words and stores
+// them token-contiguously (coalesced). Phase 4 (QJL): one lane per key, one
+// warp per 32 sketch rows.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "octo_common.cuh"
+
+namespace octo {
+
+struct EncodeArgs {
+  const void* keys;
+  int key_bf16;
+  int64_t n_heads, n_tokens, head_stride, token_stride, cache_cap, token_offset;
+  uint32_t* packed;
+  float* gamma;
+  uint32_t* qjl_bits;
+  float* qjl_norm;
+  const float* dir_c;
+  const float* dir_t;
+  const float* rho_c;
+  const float* rho_t;
+  const float* signs;
+  const float* qjl_S;
+  int64_t table_heads;
+  int joint;
+  int64_t n_tiles, tiles_per_head;
+};
+
+template <int D, int B>
+struct EncCfg {
+  static constexpr int T = (D + 2) / 3;
+  static constexpr int BD = B + 1, BR = B - 1;
+  static constexpr int C = 2 * BD + BR;
+  static constexpr int W = (T * C + 31) / 32;
+  static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
+  static constexpr int E = D / 32;                 // coordinates per lane in phase 1
+  static constexpr int KT = 8192 / D;              // keys per tile
+  static constexpr int US = ((3 * T) % 2 == 0) ? 3 * T + 1 : 3 * T;  // odd row stride (floats)
+  static constexpr int THREADS = 256;
+};
+
+template <int D, int B, bool QJL>
+__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+  using Cfg = EncCfg<D, B>;
+  constexpr int T = Cfg::T, KT = Cfg::KT, US = Cfg::US, E = Cfg::E, W = Cfg::W, C = Cfg::C;
+  constexpr int NDIR = Cfg::NDIR, NRHO = Cfg::NRHO;
+
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float4* nhat = reinterpret_cast<float4*>(smem_raw);                 // [NDIR*NDIR]
+  float* U = reinterpret_cast<float*>(nhat + NDIR * NDIR);            // [KT][US]
+  uint16_t* codes = reinterpret_cast<uint16_t*>(U + KT * US);         // [KT][T]
+  __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[8], s_rho_t[8];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NWARP = Cfg::THREADS / 32;
+
+  if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
+  if (tid < NDIR - 1) s_dir_t[tid] = a.dir_t[tid];
+  if (tid < NRHO) s_rho_c[tid] = a.rho_c[tid];
+  if (tid < NRHO - 1) s_rho_t[tid] = a.rho_t[tid];
+  __syncthreads();
+  for (int e = tid; e < NDIR * NDIR; e += Cfg::THREADS) {
+    const float3 n = oct_inverse(s_dir_c[e / NDIR], s_dir_c[e % NDIR]);
+    nhat[e] = make_float4(n.x, n.y, n.z, 0.0f);
+  }
+  // (the first __syncthreads of the tile loop orders these writes)
+
+  const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+
+  for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
+    const int64_t h = tile / a.tiles_per_head;
+    const int64_t n0 = (tile % a.tiles_per_head) * KT;
+    const int nk = static_cast<int>(a.n_tokens - n0 < KT ? a.n_tokens - n0 : KT);
+    const float* sg = a.signs + (h % a.table_heads) * D;
+    __syncthreads();  // previous tile's shared buffers are free
+
+    // ---------------- phase 1: warp per key
+    float sgn[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) sgn[e] = __ldg(sg + lane * E + e);
+    for (int k = warp; k < nk; k += NWARP) {
+      const int64_t base = h * a.head_stride + (n0 + k) * a.token_stride + lane * E;
+      float v[E];
+      if (a.key_bf16) {
+        const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(a.keys) + base;
+        if constexpr (E == 2) {
+          const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p));
+          v[0] = bf16_lo(w); v[1] = bf16_hi(w);
+        } else if constexpr (E == 4) {
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
+          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+        } else {
+          const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+          v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+        }
+      } else {
+        const float* p = static_cast<const float*>(a.keys) + base;
+        if constexpr (E == 2) {
+          const float2 w = __ldg(reinterpret_cast<const float2*>(p));
+          v[0] = w.x; v[1] = w.y;
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; e += 4) {
+            const float4 w = __ldg(reinterpret_cast<const float4*>(p + e));
+            v[e] = w.x; v[e + 1] = w.y; v[e + 2] = w.z; v[e + 3] = w.w;
+          }
+        }
+      }
+      float ss = 0.0f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
+      ss = warp_sum(ss);
+      const float g = sqrtf(ss);
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = (g > 0.0f ? v[e] / g : 0.0f) * sgn[e];
+      fwht_warp<E>(v, lane);
+      float* row = U + k * US;
+#pragma unroll
+      for (int e = 0; e < E; ++e) row[lane * E + e] = v[e] * inv_sqrt_d;
+      if (lane < 3 * T - D) row[D + lane] = 0.0f;
+      if (lane == 0) a.gamma[h * a.cache_cap + a.token_offset + n0 + k] = g;
+    }
+    __syncthreads();
+
+    // ---------------- phase 2: thread per triplet
+    for (int j = tid; j < nk * T; j += Cfg::THREADS) {
+      const int k = j / T, i = j - k * T;
+      float* tp = U + k * US + 3 * i;
+      const float x = tp[0], y = tp[1], z = tp[2];
+      const float rho = sqrtf(x * x + y * y + z * z);
+      const float l1 = fabsf(x) + fabsf(y) + fabsf(z);
+      float px = 0.0f, py = 0.0f, pz = 1.0f;
+      if (l1 > 0.0f) { px = x / l1; py = y / l1; pz = z / l1; }
+      float xi = px, eta = py;
+      if (!(pz >= 0.0f)) {
+        xi = (1.0f - fabsf(py)) * (px >= 0.0f ? 1.0f : -1.0f);
+        eta = (1.0f - fabsf(px)) * (py >= 0.0f ? 1.0f : -1.0f);
+      }
+      int ix = count_le(s_dir_t, NDIR - 1, xi);
+      int iy = count_le(s_dir_t, NDIR - 1, eta);
+      int ir;
+      float4 nb;
+      if (!a.joint) {
+        ir = count_le(s_rho_t, NRHO - 1, rho);
+        nb = nhat[ix * NDIR + iy];
+      } else {
+        // centre first, then (dx, dy) row-major; replace only on strictly smaller error
+        nb = nhat[ix * NDIR + iy];
+        float s = nb.x * x + nb.y * y + nb.z * z;
+        ir = count_le(s_rho_t, NRHO - 1, s);
+        float rh = s_rho_c[ir];
+        float best = rh * (rh - 2.0f * s);
+        const int cx = ix, cy = iy;
+#pragma unroll
+        for (int dx = -1; dx <= 1; ++dx) {
+#pragma unroll
+          for (int dy = -1; dy <= 1; ++dy) {
+            if (dx == 0 && dy == 0) continue;
+            const int ux = cx + dx, uy = cy + dy;
+            if (ux < 0 || ux >= NDIR || uy < 0 || uy >= NDIR) continue;
+            const float4 n = nhat[ux * NDIR + uy];
+            const float sc = n.x * x + n.y * y + n.z * z;
+            const int rc = count_le(s_rho_t, NRHO - 1, sc);
+            const float rr = s_rho_c[rc];
+            const float err = rr * (rr - 2.0f * sc);
+            if (err < best) { best = err; ix = ux; iy = uy; ir = rc; nb = n; }
+          }
+        }
+      }
+      codes[k * T + i] = static_cast<uint16_t>(ix | (iy << Cfg::BD) | (ir << (2 * Cfg::BD)));
+      if constexpr (QJL) {
+        // residual e = t - rho_hat n_hat, in place (the pad coordinate is dropped later)
+        const float rh = s_rho_c[ir];
+        tp[0] = x - rh * nb.x;
+        tp[1] = y - rh * nb.y;
+        tp[2] = z - rh * nb.z;
+      }
+    }
+    __syncthreads();
+
+    // ---------------- phase 3: thread per (key, word), token-contiguous stores
+    for (int j = tid; j < nk * W; j += Cfg::THREADS) {
+      const int w = j / nk, k = j - w * nk;
+      const int first = (32 * w) / C;
+      const int last = min(T - 1, (32 * w + 31) / C);
+      uint32_t word = 0;
+      for (int i = first; i <= last; ++i) {
+        const uint32_t code = codes[k * T + i];
+        const int sh = i * C - 32 * w;
+        word |= sh >= 0 ? (code << sh) : (code >> (-sh));
+      }
+      a.packed[(h * W + w) * a.cache_cap + a.token_offset + n0 + k] = word;
+    }
+
+    if constexpr (QJL) {
+      // ---------------- phase 4: sketch bits = [ (S e)_r >= 0 ], nu = ||e||
+      constexpr int QW = D / 32;                  // sketch words per key
+      constexpr int KG = (KT + 31) / 32;          // 32-key groups
+      const float* S = a.qjl_S + (h % a.table_heads) * D * D;
+      for (int item = warp; item < QW * KG; item += NWARP) {
+        const int qw = item % QW, kg = item / QW;
+        const int k = kg * 32 + lane;
+        if (k < nk) {
+          const float* e = U + k * US;
+          uint32_t bits = 0;
+          for (int r = 0; r < 32; ++r) {
+            const float4* srow = reinterpret_cast<const float4*>(S + (qw * 32 + r) * D);
+            float acc = 0.0f;
+#pragma unroll 8
+            for (int m4 = 0; m4 < D / 4; ++m4) {
+              const float4 sv = __ldg(srow + m4);
+              acc = fmaf(sv.x, e[4 * m4], acc);
+              acc = fmaf(sv.y, e[4 * m4 + 1], acc);
+              acc = fmaf(sv.z, e[4 * m4 + 2], acc);
+              acc = fmaf(sv.w, e[4 * m4 + 3], acc);
+            }
+            bits |= (acc >= 0.0f ? 1u : 0u) << r;
+          }
+          a.qjl_bits[(h * QW + qw) * a.cache_cap + a.token_offset + n0 + k] = bits;
+          if (qw == 0) {
+            float ss = 0.0f;
+            for (int m = 0; m < D; ++m) ss = fmaf(e[m], e[m], ss);
+            a.qjl_norm[h * a.cache_cap + a.token_offset + n0 + k] = sqrtf(ss);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int D, int B, bool QJL>
+static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
+  using Cfg = EncCfg<D, B>;
+  EncodeArgs a = a0;
+  a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
+  a.n_tiles = a.tiles_per_head * a.n_heads;
+  const size_t smem = sizeof(float4) * Cfg::NDIR * Cfg::NDIR + sizeof(float) * Cfg::KT * Cfg::US +
+                      sizeof(uint16_t) * Cfg::KT * Cfg::T;
+  auto kern = encode_kernel<D, B, QJL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, smem);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t grid = std::min<int64_t>(a.n_tiles, static_cast<int64_t>(sms) * per_sm);
+  kern<<<static_cast<unsigned>(grid), Cfg::THREADS, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, int B>
+static cudaError_t dispatch_qjl(const EncodeArgs& a, bool qjl, cudaStream_t st) {
+  return qjl ? launch_encode<D, B, true>(a, st) : launch_encode<D, B, false>(a, st);
+}
+
+template <int D>
+static cudaError_t dispatch_b(const EncodeArgs& a, int b, bool qjl, cudaStream_t st) {
+  switch (b) {
+    case 2: return dispatch_qjl<D, 2>(a, qjl, st);
+    case 3: return dispatch_qjl<D, 3>(a, qjl, st);
+    default: return dispatch_qjl<D, 4>(a, qjl, st);
+  }
+}
+
+}  // namespace octo
+
+extern "C" int octo_encode(const octo_layout* L, const octo_tables* tab, const void* keys, int key_dtype,
+                           int64_t n_heads, int64_t n_tokens, int64_t head_stride, int64_t token_stride,
+                           int64_t cache_cap, int64_t token_offset, uint32_t* packed, float* gamma,
+                           uint32_t* qjl_bits, float* qjl_norm, octo_stream_t stream) {
+  using namespace octo;
+  if (!L || !tab) return OCTO_EINVAL;
+  if (L->d != 64 && L->d != 128 && L->d != 256) return OCTO_EUNSUPPORTED;
+  if (L->b < 2 || L->b > 4) return OCTO_EUNSUPPORTED;
+  octo_layout chk;
+  if (octo_layout_init(&chk, L->d, L->b, L->qjl, L->rounding) != OCTO_OK) return OCTO_EINVAL;
+  if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits) return OCTO_EINVAL;
+  if (key_dtype != OCTO_F32 && key_dtype != OCTO_BF16) return OCTO_EINVAL;
+  if (n_heads < 0 || n_tokens < 0 || token_offset < 0 || cache_cap < 0) return OCTO_EINVAL;
+  if (token_offset + n_tokens > cache_cap) return OCTO_EINVAL;
+  if (n_heads == 0 || n_tokens == 0) return OCTO_OK;
+  if (!keys || !packed || !gamma || !tab->dir_c || !tab->dir_t || !tab->rho_c || !tab->signs ||
+      tab->n_heads < 1)
+    return OCTO_EINVAL;
+  if (L->n_rho > 1 && !tab->rho_t) return OCTO_EINVAL;
+  if (L->qjl && (!qjl_bits || !qjl_norm || !tab->qjl_S)) return OCTO_EINVAL;
+  if (head_stride < 0 || token_stride < 0) return OCTO_EINVAL;
+  const int esz = key_dtype == OCTO_F32 ? 4 : 2;
+  // each lane loads D/32 contiguous elements with one vector load
+  const int64_t vec = std::min<int64_t>(16, static_cast<int64_t>(L->d / 32) * esz);
+  if (reinterpret_cast<uintptr_t>(keys) % vec != 0 || (head_stride * esz) % vec != 0 ||
+      (token_stride * esz) % vec != 0)
+    return OCTO_EINVAL;
+  EncodeArgs a{};
+  a.keys = keys;
+  a.key_bf16 = key_dtype == OCTO_BF16;
+  a.n_heads = n_heads;
+  a.n_tokens = n_tokens;
+  a.head_stride = head_stride;
+  a.token_stride = token_stride;
+  a.cache_cap = cache_cap;
+  a.token_offset = token_offset;
+  a.packed = packed;
+  a.gamma = gamma;
+  a.qjl_bits = qjl_bits;
+  a.qjl_norm = qjl_norm;
+  a.dir_c = tab->dir_c;
+  a.dir_t = tab->dir_t;
+  a.rho_c = tab->rho_c;
+  a.rho_t = tab->rho_t;
+  a.signs = tab->signs;
+  a.qjl_S = tab->qjl_S;
+  a.table_heads = tab->n_heads;
+  a.joint = L->rounding == OCTO_ROUND_JOINT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  switch (L->d) {
+    case 64: e = dispatch_b<64>(a, L->b, L->qjl != 0, st); break;
+    case 128: e = dispatch_b<128>(a, L->b, L->qjl != 0, st); break;
+    default: e = dispatch_b<256>(a, L->b, L->qjl != 0, st); break;
+  }
+  return e == cudaSuccess ? OCTO_OK : OCTO_ECUDA;
+}

@@ -1,0 +1,131 @@
+"""CPU tests of the C ABI: the library loads, exports every declared symbol,
+its host table builders agree with the oracle, and argument validation
+returns a status before anything is launched."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tables
+from rotation_preconditioned_quantization_b200 import _lib, api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "octopus.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(octo_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.lib()
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib.exported_symbols())
+    assert L.octo_abi_version() == 100
+
+
+@pytest.mark.parametrize("d,b", [(64, 2), (64, 4), (128, 3), (128, 4), (256, 2), (256, 4)])
+def test_layout_init(d, b):
+    lay = api.Layout(d, b, qjl=True)
+    T = -(-d // 3)
+    assert (lay.T, lay.b_dir, lay.b_rho, lay.code_bits) == (T, b + 1, b - 1, 3 * b + 1)
+    assert lay.words == -(-T * (3 * b + 1) // 32)
+    assert (lay.n_dir, lay.n_rho, lay.qjl_words) == (2 ** (b + 1), 2 ** (b - 1), d // 32)
+
+
+def test_layout_words_of_the_workloads():
+    # 43 triplets x 10 bits = 14 words (d=128, b=3); 22 x 7 = 5 (d=64, b=2); 43 x 13 = 18 (d=128, b=4)
+    assert api.Layout(128, 3).words == 14
+    assert api.Layout(64, 2).words == 5
+    assert api.Layout(128, 4).words == 18
+
+
+def test_layout_rejects_unsupported():
+    L = _lib.OctoLayout()
+    f = _lib.lib().octo_layout_init
+    assert f(ctypes.byref(L), 96, 3, 0, 1) == _lib.OCTO_EUNSUPPORTED
+    assert f(ctypes.byref(L), 128, 5, 0, 1) == _lib.OCTO_EUNSUPPORTED
+    assert f(ctypes.byref(L), 128, 1, 0, 1) == _lib.OCTO_EUNSUPPORTED
+    assert f(ctypes.byref(L), 128, 3, 2, 1) == _lib.OCTO_EINVAL
+    assert f(ctypes.byref(L), 128, 3, 0, 7) == _lib.OCTO_EINVAL
+    assert f(None, 128, 3, 0, 1) == _lib.OCTO_EINVAL
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_host_codebooks_match_oracle(d, b):
+    lay = api.Layout(d, b)
+    dc, dt, rc, rt = api.codebook_build(lay)
+    odc, odt, orc, ort = tables.codebooks(d, b)
+    # independent constructions (closed-form marginal + own quadrature vs nested quadrature)
+    assert np.max(np.abs(dc - odc)) < 1e-7 and np.max(np.abs(rc - orc)) < 1e-7
+    assert np.max(np.abs(dt - odt)) < 1e-7
+    if len(ort):
+        assert np.max(np.abs(rt - ort)) < 1e-7
+    # and after rounding to float32 they are the same tables
+    f = lambda x: np.asarray(x, dtype=np.float32)
+    assert np.array_equal(dc, f(odc)) and np.array_equal(rc, f(orc)) and np.array_equal(dt, f(odt))
+
+
+def test_host_signs_and_qjl_match_oracle():
+    s = api.rotation_build(7, 128, 3)
+    assert np.array_equal(s, tables.rotation_signs(7, 128, 3).astype(np.float32))
+    S = api.qjl_build(3, 64, 2)
+    oS = tables.qjl_matrix(3, 64, 2).astype(np.float32)
+    # libm vs numpy transcendental functions may differ in the last bit of the double
+    ulp = np.spacing(np.abs(oS))
+    assert np.all(np.abs(S - oS) <= ulp)
+    assert np.mean(S == oS) > 0.999
+
+
+def test_encode_and_decode_validate_before_launch():
+    L = api.Layout(128, 3)
+    lib = _lib.lib()
+    T = _lib.OctoTables()
+    null = None
+    # NULL tables / keys
+    assert lib.octo_encode(L.ref, None, null, 0, 1, 1, 128, 128, 4, 0, null, null, null, null, null) == _lib.OCTO_EINVAL
+    assert lib.octo_encode(L.ref, ctypes.byref(T), null, 0, 1, 1, 128, 128, 4, 0, null, null, null, null, null) == _lib.OCTO_EINVAL
+    # range checks: offset + n > cap, negative sizes, bad dtype
+    assert lib.octo_encode(L.ref, ctypes.byref(T), 16, 0, 1, 5, 128, 128, 4, 0, 16, 16, null, null, null) == _lib.OCTO_EINVAL
+    assert lib.octo_encode(L.ref, ctypes.byref(T), 16, 0, -1, 1, 128, 128, 4, 0, 16, 16, null, null, null) == _lib.OCTO_EINVAL
+    assert lib.octo_encode(L.ref, ctypes.byref(T), 16, 9, 1, 1, 128, 128, 4, 0, 16, 16, null, null, null) == _lib.OCTO_EINVAL
+    # zero tokens is a no-op
+    assert lib.octo_encode(L.ref, ctypes.byref(T), null, 0, 1, 0, 128, 128, 4, 0, null, null, null, null, null) == _lib.OCTO_OK
+    # decode: kv_len > cap, Hq % Hkv, both outputs NULL, too many query rows
+    args = lambda **k: dict(dict(q=16, qd=0, B=1, Hq=4, Hkv=1, Lq=1, kv=8, cap=8, V=16, out=16, lg=null), **k)
+
+    def dec(a):
+        return lib.octo_decode_attn(L.ref, ctypes.byref(T), a["q"], a["qd"], a["B"], a["Hq"], a["Hkv"], a["Lq"],
+                                    a["kv"], a["cap"], 16, 16, null, null, a["V"], ctypes.c_float(0.1), a["out"], a["lg"],
+                                    null, 0, null)
+    assert dec(args()) == _lib.OCTO_EINVAL                    # tables hold NULL pointers
+    Tf = _lib.OctoTables(16, 16, 16, 16, 16, None, 1)
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 9, 8, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 3, 2, 1, 8, 8, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 16, 16, null, null, null,
+                                ctypes.c_float(0.1), null, null, null, 0, null) == _lib.OCTO_EINVAL
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 16, 1, 1, 8, 8, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EUNSUPPORTED
+    # QJL layout without sketch buffers
+    Lq = api.Layout(128, 4, qjl=True)
+    assert lib.octo_decode_attn(Lq.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
+    assert lib.octo_decode_attn_workspace(L.ref, 1, 16, 1, 1, 8) == 0
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4):
+        assert _lib.status_string(s).startswith("OCTO_")
+    with pytest.raises(_lib.OctoError):
+        _lib.check(-1, "x")

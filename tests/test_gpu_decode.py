@@ -1,0 +1,181 @@
+"""GPU parity of octo_decode_attn against the oracle (called through the C ABI).
+
+The cache the GPU decodes is the ORACLE's encoding of the keys (packed by
+the oracle and copied into the word-planar layout), so encode boundary flips
+cannot leak into these checks and no oracle input comes from the GPU.
+The oracle takes the materialised route (k_hat = gamma R^T u_hat, q . k_hat);
+the kernel the rotated-query route.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, codec, tables
+from rotation_preconditioned_quantization_b200 import api, inputs
+
+from . import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_cache(keys, d, b, signs_rows, tb, qjl_S=None, cap=None):
+    """Oracle-encode keys [H][N][d]; return (encodings, device Cache)."""
+    H, N, _ = keys.shape
+    cap = N if cap is None else cap
+    olay = codec.Layout(d, b)
+    lay = api.Layout(d, b, qjl=qjl_S is not None)
+    encs, words, gam, qb, qn = [], [], [], [], []
+    for h in range(H):
+        e = codec.encode(keys[h].astype(np.float64), signs_rows[h], tb, olay)
+        encs.append(e)
+        words.append(e.words)
+        gam.append(e.gamma)
+        if qjl_S is not None:
+            uh = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, olay)
+            bits, nu, _ = codec.qjl_encode(e.u_rot, uh, qjl_S[h])
+            e.qbits, e.nu = bits, nu
+            qb.append(codec.qjl_pack(bits))
+            qn.append(nu)
+    cache = api.Cache.empty(lay, H, cap)
+    planar = parity.to_planar(np.stack(words)).view(np.int32)
+    cache.packed[:, :, :N] = torch.from_numpy(planar).cuda()
+    cache.gamma[:, :N] = torch.from_numpy(np.stack(gam).astype(np.float32)).cuda()
+    if qjl_S is not None:
+        cache.qjl_bits[:, :, :N] = torch.from_numpy(parity.to_planar(np.stack(qb)).view(np.int32)).cuda()
+        cache.qjl_norm[:, :N] = torch.from_numpy(np.stack(qn).astype(np.float32)).cuda()
+    cache.length = N
+    return encs, cache
+
+
+def _run_case(B, Hq, Hkv, Lq, d, b, N, qjl=False, q_dtype=torch.bfloat16, cap=None, seed=0, logits_only=False,
+              kv_len=None, check_logits=True):
+    tb = parity.oracle_tables(d, b)
+    H = B * Hkv
+    signs = tables.rotation_signs(seed, d, Hkv)
+    S = tables.qjl_matrix(seed + 7, d, Hkv) if qjl else None
+    keys = inputs.to_bf16(inputs.llm_keys(seed + 1, H, N, d))
+    rows = [signs[h % Hkv] for h in range(H)]
+    Srows = [S[h % Hkv] for h in range(H)] if qjl else None
+    encs, cache = _oracle_cache(keys, d, b, rows, tb, Srows, cap)
+    cap = cache.cap
+    kv = N if kv_len is None else kv_len
+    q = inputs.normal(seed + 2, (B, Hq, Lq, d))
+    if q_dtype == torch.bfloat16:
+        q = inputs.to_bf16(q)
+    Vn = inputs.to_bf16(inputs.normal(seed + 3, (H, cap, d)))
+    lay = api.Layout(d, b, qjl=qjl)
+    dev = api.DeviceTables(*tb, signs, S)
+    qt = torch.from_numpy(q).to(q_dtype).cuda()
+    Vt = None if logits_only else torch.from_numpy(Vn).to(torch.bfloat16).cuda()
+    out, lg = api.decode_attn(lay, dev, qt, cache, Vt, Hkv, kv_len=kv, logits=check_logits)
+    torch.cuda.synchronize()
+    olay = codec.Layout(d, b)
+    g = Hq // Hkv
+    if kv == 0:
+        assert torch.count_nonzero(out) == 0
+        return
+    worst_l, worst_o = 0.0, 0.0
+    for bi in range(B):
+        for hk in range(Hkv):
+            h = bi * Hkv + hk
+            e = encs[h]
+            qq = q[bi, hk * g:(hk + 1) * g].reshape(g * Lq, d).astype(np.float64)
+            sl = slice(0, kv)
+            qjl_args = (e.qbits[sl], e.nu[sl], S[hk]) if qjl else None
+            ref_o, ref_l = attention.decode_attention(qq, e.gamma[sl], e.i_xi[sl], e.i_eta[sl], e.i_rho[sl],
+                                                      Vn[h, sl].astype(np.float64), signs[hk], tb, olay, qjl=qjl_args)
+            if check_logits and kv > 0:
+                got_l = lg[bi, hk * g:(hk + 1) * g].reshape(g * Lq, kv).cpu().numpy()
+                tol = 1e-4 * e.gamma[sl][None, :] * np.linalg.norm(qq, axis=1)[:, None]
+                err = np.abs(got_l - ref_l)
+                assert np.all(err <= tol), f"logit error {np.max(err / np.maximum(tol, 1e-30))} x tol"
+                worst_l = max(worst_l, float(np.max(err / np.maximum(tol, 1e-30))))
+            if not logits_only:
+                got_o = out[bi, hk * g:(hk + 1) * g].reshape(g * Lq, d).cpu().numpy()
+                tol = 2e-3 * np.max(np.abs(ref_o), axis=1, keepdims=True)
+                err = np.abs(got_o - ref_o)
+                assert np.all(err <= tol), f"output error {np.max(err / tol)} x tol"
+                worst_o = max(worst_o, float(np.max(err / tol)))
+    print(f"\n[decode parity] B={B} Hq={Hq} Hkv={Hkv} Lq={Lq} d={d} b={b} N={N} kv={kv} qjl={qjl}: "
+          f"worst logit err {worst_l:.3g} x tol, worst output err {worst_o:.3g} x tol")
+
+
+def test_logits_single_head_4096(cuda_ok):
+    """One head, d=128, 4096 keys, b=3, one fp32 query: raw logits only."""
+    tb = parity.oracle_tables(128, 3)
+    signs = tables.rotation_signs(0, 128, 1)
+    keys = inputs.gaussian_keys(0, 1, 4096, 128)
+    encs, cache = _oracle_cache(keys, 128, 3, signs, tb)
+    q = inputs.normal(1, (1, 1, 1, 128))
+    lay = api.Layout(128, 3)
+    dev = api.DeviceTables(*tb, signs)
+    _, lg = api.decode_attn(lay, dev, torch.from_numpy(q).cuda(), cache, None, 1, logits=True)
+    torch.cuda.synchronize()
+    ref = attention.logits(q[0, 0].astype(np.float64), encs[0].gamma, encs[0].i_xi, encs[0].i_eta, encs[0].i_rho,
+                           signs[0], tb, codec.Layout(128, 3))[0]
+    got = lg.cpu().numpy()[0, 0, 0]
+    tol = 1e-4 * encs[0].gamma * np.linalg.norm(q)
+    assert np.all(np.abs(got - ref) <= tol)
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=1, Hq=8, Hkv=2, Lq=1, d=128, b=3, N=3000),                      # GQA 4, ragged tail
+    dict(B=1, Hq=2, Hkv=2, Lq=8, d=64, b=2, N=5000),                       # 8 query tokens per head
+    dict(B=2, Hq=8, Hkv=2, Lq=1, d=128, b=4, N=2000, qjl=True),            # OCTOPUS-QJL
+    dict(B=1, Hq=4, Hkv=4, Lq=1, d=128, b=3, N=1000, q_dtype=torch.float32),  # MHA (1 row)
+    dict(B=1, Hq=4, Hkv=2, Lq=1, d=256, b=2, N=777),                       # 2 rows, d=256
+    dict(B=1, Hq=2, Hkv=1, Lq=3, d=64, b=4, N=100),                        # 6 rows
+    dict(B=1, Hq=4, Hkv=1, Lq=1, d=256, b=4, N=1500, qjl=True),            # QJL, d=256
+    dict(B=1, Hq=8, Hkv=1, Lq=1, d=64, b=3, N=640, qjl=True),              # QJL, 8 rows
+    dict(B=1, Hq=4, Hkv=1, Lq=1, d=128, b=3, N=300, cap=1000),             # cache larger than kv_len
+    dict(B=1, Hq=4, Hkv=1, Lq=1, d=128, b=3, N=1),                         # a single key
+    dict(B=3, Hq=4, Hkv=1, Lq=1, d=128, b=2, N=64, kv_len=0),              # empty context
+])
+def test_decode_attention_cases(cuda_ok, case):
+    _run_case(**case)
+
+
+def test_decode_llm_shaped_full_size(cuda_ok):
+    """B=1, 32 query / 8 KV heads, d=128, 32768 tokens, b=3: every output and logit."""
+    _run_case(1, 32, 8, 1, 128, 3, 32768)
+
+
+def test_decode_workspace_reuse_and_counters(cuda_ok):
+    """Repeated calls with one workspace give identical results (tickets reset)."""
+    tb = parity.oracle_tables(128, 3)
+    signs = tables.rotation_signs(0, 128, 2)
+    keys = inputs.to_bf16(inputs.llm_keys(3, 2, 20000, 128))
+    encs, cache = _oracle_cache(keys, 128, 3, signs, tb)
+    lay = api.Layout(128, 3)
+    dev = api.DeviceTables(*tb, signs)
+    q = torch.from_numpy(inputs.to_bf16(inputs.normal(4, (1, 8, 1, 128)))).to(torch.bfloat16).cuda()
+    V = torch.from_numpy(inputs.to_bf16(inputs.normal(5, (2, 20000, 128)))).to(torch.bfloat16).cuda()
+    ws = api.Workspace(api.decode_attn_workspace_bytes(lay, 1, 8, 2, 1, 20000))
+    o1, _ = api.decode_attn(lay, dev, q, cache, V, 2, workspace=ws)
+    o2, _ = api.decode_attn(lay, dev, q, cache, V, 2, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+    n_heads = 2
+    assert int(ws.buf[:n_heads].abs().sum()) == 0
+
+
+def test_decode_rejects_small_workspace(cuda_ok):
+    lay = api.Layout(128, 3)
+    tb = parity.oracle_tables(128, 3)
+    dev = api.DeviceTables(*tb, tables.rotation_signs(0, 128, 1))
+    cache = api.Cache.empty(lay, 1, 100000)
+    cache.length = 100000
+    q = torch.zeros((1, 4, 1, 128), dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros((1, 100000, 128), dtype=torch.bfloat16, device="cuda")
+    ws = api.Workspace(256)
+    from rotation_preconditioned_quantization_b200 import _lib
+    need = api.decode_attn_workspace_bytes(lay, 1, 4, 1, 1, 100000)
+    assert need > 256
+    st = _lib.lib().octo_decode_attn(lay.ref, dev.ref, q.data_ptr(), _lib.BF16, 1, 4, 1, 1, 100000, 100000,
+                                     cache.packed.data_ptr(), cache.gamma.data_ptr(), None, None, V.data_ptr(),
+                                     0.1, torch.empty((1, 4, 1, 128), device="cuda").data_ptr(), None,
+                                     ws.buf.data_ptr(), 256, None)
+    assert st == _lib.OCTO_EWORKSPACE
