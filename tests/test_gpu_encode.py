@@ -35,7 +35,8 @@ def _encode_gpu(lay, dev, keys_np, dtype, cap=None, offset=0, keys_view=None):
     return out
 
 
-def _check(keys_np, d, b, rounding, dtype, seed=0, qjl=False, cap=None, offset=0, label=""):
+def _check(keys_np, d, b, rounding, dtype, seed=0, qjl=False, cap=None, offset=0, label="",
+           max_boundary_fraction=MAX_BOUNDARY_FRACTION):
     H, N, _ = keys_np.shape
     tb = parity.oracle_tables(d, b)
     signs = tables.rotation_signs(seed, d, H)
@@ -63,7 +64,7 @@ def _check(keys_np, d, b, rounding, dtype, seed=0, qjl=False, cap=None, offset=0
             assert qf == 0, f"{label} head {h}: {qf} non-boundary sketch mismatches"
             np.testing.assert_allclose(g["qnorm"][h][same], nu[same], rtol=1e-4, atol=1e-6)
             tot["qmis"] += qm; tot["qbnd"] += qb
-    assert tot["bnd"] <= MAX_BOUNDARY_FRACTION * tot["trip"]
+    assert tot["bnd"] <= max_boundary_fraction * tot["trip"]
     print(f"\n[encode parity] {label} d={d} b={b} round={'J' if rounding else 'S'} {dtype}: "
           f"{tot['trip']} triplets, {tot['mis']} mismatches, all at a boundary ({tot['bnd']})"
           + (f"; sketch bits {tot['qmis']} mismatches ({tot['qbnd']} at a boundary)" if qjl else ""))
@@ -139,7 +140,9 @@ def test_encode_special_keys(cuda_ok):
     k[0, 3] = 1e10 * inputs.normal(2, d)               # huge
     k[0, 4] = -1.0                                     # constant
     k[0, 5, ::3] = 2.0                                 # sparse
-    g, _ = _check(k, d, b, api.ROUND_JOINT, torch.float32, seed=9, label="special")
+    # structured keys put many values exactly on ties (equal-magnitude rotated
+    # coordinates), so boundary cases are frequent here; failures must still be zero
+    g, _ = _check(k, d, b, api.ROUND_JOINT, torch.float32, seed=9, label="special", max_boundary_fraction=1.0)
     assert g["gamma"][0, 0] == 0.0
     # zero key -> every triplet is the zero triplet: centre cell, lowest rho level
     lay = codec.Layout(d, b)
