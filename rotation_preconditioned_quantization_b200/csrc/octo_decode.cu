@@ -1,488 +1,13 @@
-// OCTOPUS fused decode attention for sm_100a.
-//
-// One step of decode attention over a compressed key cache (explainer,
-// "engineering implementation": decompression, dot products and online
-// softmax happen on chip, the uncompressed keys are never written out; the
-// abstract: keys are reconstructed on the fly without materialising them).
-//
-// Math per KV head (b, h) with query rows r (GQA group x query tokens):
-//   q_rot_r = (1/sqrt(d)) H (s_h * q_r)                    (rotated once)
-//   logit_rn = gamma_n * sum_i rho_hat_in (q_rot_r,i . n_hat_in)
-//              [+ gamma_n nu_n sqrt(pi/2)/d <S q_rot_r, 2 bits_n - 1>]  (QJL)
-//   out_r = softmax_n(scale * logit_rn) V_n
-// Because R is orthogonal, q . k_hat = gamma q_rot . u_rot_hat, so the keys
-// are never inverse-rotated.
-//
-// Structure (one CTA = one KV head x one contiguous slice of the cache):
-//  * prologue: codebooks -> a shared-memory table of decoded triplets
-//    (rho_hat * n_hat for every full code when 3b+1 <= 10 bits, else n_hat
-//    for every direction code plus a rho_hat lookup), replicated 8x so that
-//    the 8 lanes of a quarter-warp read distinct bank groups (conflict-free
-//    128-bit loads); queries rotated by warp-shuffle WHT into a
-//    triplet-major layout; for QJL, p = S q_rot and a 4-bit lookup table of
-//    signed partial sums of p.
-//  * main loop, one warp per 32-key chunk, one lane per key: coalesced
-//    loads of the token-contiguous code words, gamma (and sketch); logits by
-//    table lookups and FMAs; online softmax (m, l) per query row; P.V on
-//    tensor cores (mma.sync m16n8k16 bf16, P split into bf16 hi + lo parts so
-//    the product keeps ~16 mantissa bits) with V read straight from global
-//    memory into A-fragment registers (16-byte loads + byte permutes).
-//  * epilogue: warps merge (m, l, O) in shared memory; CTAs of a head merge
-//    through the workspace, the last-arriving CTA (atomic ticket, no
-//    spinning) writes the normalised output and resets the ticket.
+// OCTOPUS fused decode attention: host entry points (argument checks,
+// split planning, workspace carve-up, dispatch to the per-D kernels).
 
 #include <cuda_runtime.h>
 
 #include <algorithm>
 
-#include "octo_common.cuh"
+#include "octo_decode_kernel.cuh"
 
 namespace octo {
-
-struct DecodeArgs {
-  const void* q;
-  int q_bf16;
-  int B, Hq, Hkv, Lq, g, Gq;  // g = Hq / Hkv, Gq = g * Lq query rows per KV head
-  int64_t kv_len, cache_cap;
-  const uint32_t* packed;
-  const float* gamma;
-  const uint32_t* qjl_bits;
-  const float* qjl_norm;
-  const __nv_bfloat16* V;
-  float scale_log2;  // scale * log2(e)
-  float* out;
-  float* logits;
-  const float* dir_c;
-  const float* rho_c;
-  const float* signs;
-  const float* qjl_S;
-  int64_t table_heads;
-  int n_splits;
-  int64_t keys_per_split;
-  int* counters;
-  float* part_m;
-  float* part_l;
-  float* part_o;
-};
-
-template <int D, int B, int G, bool QJL>
-struct DecCfg {
-  static constexpr int T = (D + 2) / 3;
-  static constexpr int BD = B + 1, BR = B - 1;
-  static constexpr int C = 2 * BD + BR;
-  static constexpr int W = (T * C + 31) / 32;
-  static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr bool FOLD = C <= 10;                    // table indexed by the full code
-  static constexpr int NE = FOLD ? (1 << C) : (1 << (2 * BD));
-  static constexpr int REP = 8;
-  static constexpr int THREADS = 256, NWARP = THREADS / 32;
-  static constexpr int QW = D / 32;                        // sketch words per key
-  static constexpr int PSTRIDE = 40;                       // floats per P row (bank-conflict-free reads)
-  static constexpr int MT = D / 16;                        // m-tiles of O^T
-  static constexpr int NCH = D / 64;                       // 16-byte V chunks per key per lane
-  static constexpr int GV = (G + 3) / 4;                   // float4 per LUT entry
-  // shared memory carve-up (bytes)
-  // region 0 holds the decoded-triplet table during the main loop and the
-  // warps' (m, l, O) afterwards; scratch holds the rotated query rows (and
-  // p = S q_rot for QJL) during the prologue.
-  static constexpr size_t TABLE = sizeof(float4) * NE * REP;
-  static constexpr size_t MERGE = sizeof(float) * NWARP * G * (D + 2);
-  static constexpr size_t REGION0 = TABLE > MERGE ? TABLE : MERGE;
-  static constexpr size_t QT = sizeof(float4) * T * G;
-  static constexpr size_t PBUF = sizeof(float) * NWARP * G * PSTRIDE;
-  static constexpr size_t LUT = QJL ? sizeof(float4) * (D / 4) * 16 * GV : 0;
-  static constexpr size_t QROW = D + 4;                       // floats per scratch query row
-  static constexpr size_t SCRATCH = sizeof(float) * G * (QROW + (QJL ? D : 0));
-  static constexpr size_t SMEM = REGION0 + QT + PBUF + LUT + SCRATCH;
-};
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-// hi + lo bf16 split of two fp32 values: x ~= hi + lo with |x - hi - lo| <~ 2^-17 |x|.
-__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  hi = pack_bf16x2(x0, x1);
-  const float r0 = x0 - bf16_lo(hi), r1 = x1 - bf16_hi(hi);
-  lo = pack_bf16x2(r0, r1);
-}
-
-template <int D, int B, int G, bool QJL>
-__global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
-  using Cfg = DecCfg<D, B, G, QJL>;
-  constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, BD = Cfg::BD, NDIR = Cfg::NDIR;
-  constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, QW = Cfg::QW;
-  constexpr int PS = Cfg::PSTRIDE, MT = Cfg::MT, NCH = Cfg::NCH, GV = Cfg::GV;
-
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float4* table = reinterpret_cast<float4*>(smem_raw);                                   // [NE*REP]
-  float* merge = reinterpret_cast<float*>(smem_raw);                                     // aliases table
-  float4* qt = reinterpret_cast<float4*>(smem_raw + Cfg::REGION0);                       // [T][G]
-  float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::REGION0 + Cfg::QT);             // [NWARP][G][PS]
-  float4* lut = reinterpret_cast<float4*>(smem_raw + Cfg::REGION0 + Cfg::QT + Cfg::PBUF);  // [D/4][16][GV]
-  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::REGION0 + Cfg::QT + Cfg::PBUF + Cfg::LUT);
-  constexpr int QROW = static_cast<int>(Cfg::QROW);
-  __shared__ float s_rho_c[8];
-  __shared__ float s_dir_c[32];
-  __shared__ int s_last;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int split = blockIdx.x;
-  const int bh = blockIdx.y;  // b * Hkv + h_kv
-  const int bidx = bh / a.Hkv, hkv = bh - bidx * a.Hkv;
-  const int64_t trow = bh % a.table_heads;
-  const bool with_v = a.V != nullptr;
-
-  // ------------------------------------------------ prologue
-  if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
-  if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
-  __syncthreads();
-  for (int j = tid; j < NE * REP; j += Cfg::THREADS) {
-    const int e = j / REP;
-    const int ix = e & (NDIR - 1), iy = (e >> BD) & (NDIR - 1);
-    float3 n = oct_inverse(s_dir_c[ix], s_dir_c[iy]);
-    if constexpr (Cfg::FOLD) {
-      const float r = s_rho_c[e >> (2 * BD)];
-      n.x *= r; n.y *= r; n.z *= r;
-    }
-    table[j] = make_float4(n.x, n.y, n.z, 0.0f);
-  }
-  // rotate the query rows: warp r handles row r
-  for (int r = warp; r < G; r += NWARP) {
-    constexpr int E = D / 32;
-    float v[E];
-    if (r < a.Gq) {
-      const int gi = r / a.Lq, lq = r - gi * a.Lq;
-      const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
-      const float* sg = a.signs + trow * D + lane * E;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float x = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qoff + e])
-                                 : static_cast<const float*>(a.q)[qoff + e];
-        v[e] = x * sg[e];
-      }
-      fwht_warp<E>(v, lane);
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = 0.0f;
-    }
-    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
-    float* qrow = scratch + r * QROW;  // padded rotated row
-#pragma unroll
-    for (int e = 0; e < E; ++e) qrow[lane * E + e] = v[e] * inv_sqrt_d;
-    if (lane < 3 * T - D) qrow[D + lane] = 0.0f;
-  }
-  __syncthreads();
-  for (int j = tid; j < T * G; j += Cfg::THREADS) {
-    const int i = j / G, r = j - i * G;
-    const float* qrow = scratch + r * QROW;
-    qt[j] = make_float4(qrow[3 * i], qrow[3 * i + 1], qrow[3 * i + 2], 0.0f);
-  }
-  if constexpr (QJL) {
-    // p_r = S q_rot_r (D outputs per row), then the 4-bit signed-sum table.
-    float* p = scratch + G * QROW;  // [G][D]
-    const float* S = a.qjl_S + trow * D * D;
-    for (int j = tid; j < G * D; j += Cfg::THREADS) {
-      const int r = j / D, m = j - r * D;
-      const float* qrow = scratch + r * QROW;
-      const float* srow = S + static_cast<int64_t>(m) * D;
-      float acc = 0.0f;
-      for (int t = 0; t < D; ++t) acc = fmaf(__ldg(srow + t), qrow[t], acc);
-      p[j] = acc;
-    }
-    __syncthreads();
-    for (int j = tid; j < (D / 4) * 16; j += Cfg::THREADS) {
-      const int grp = j >> 4, nib = j & 15;
-      float vals[4 * GV];
-#pragma unroll
-      for (int r = 0; r < 4 * GV; ++r) {
-        float s = 0.0f;
-        if (r < G) {
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float pv = p[r * D + 4 * grp + t];
-            s += ((nib >> t) & 1) ? pv : -pv;
-          }
-        }
-        vals[r] = s;
-      }
-#pragma unroll
-      for (int v4 = 0; v4 < GV; ++v4)
-        lut[j * GV + v4] = make_float4(vals[4 * v4], vals[4 * v4 + 1], vals[4 * v4 + 2], vals[4 * v4 + 3]);
-    }
-  }
-  __syncthreads();
-
-  // ------------------------------------------------ main loop
-  const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
-  const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
-  const int g8 = lane >> 2, c4 = lane & 3;
-  const int rep_off = lane & (REP - 1);
-
-  float m_run[G], l_run[G];
-#pragma unroll
-  for (int r = 0; r < G; ++r) { m_run[r] = -INFINITY; l_run[r] = 0.0f; }
-  float acc_o[MT][4];
-#pragma unroll
-  for (int t = 0; t < MT; ++t) acc_o[t][0] = acc_o[t][1] = acc_o[t][2] = acc_o[t][3] = 0.0f;
-
-  const uint32_t* pk = a.packed + static_cast<int64_t>(bh) * W * a.cache_cap;
-  const float* gm = a.gamma + static_cast<int64_t>(bh) * a.cache_cap;
-  const __nv_bfloat16* Vh = with_v ? a.V + static_cast<int64_t>(bh) * a.cache_cap * D : nullptr;
-  float* pw = pbuf + warp * G * PS;
-
-  for (int64_t base = k_begin + 32 * warp; base < k_end; base += 32 * NWARP) {
-    const int64_t key = base + lane;
-    const bool valid = key < k_end;
-
-    // V fragments for both 16-key steps, issued first so their latency hides under the logit math
-    uint4 vreg[2][4][NCH];
-    if (with_v) {
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int64_t vk = base + 16 * ks + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
-#pragma unroll
-          for (int hh = 0; hh < NCH; ++hh) {
-            if (vk < k_end)
-              vreg[ks][kk][hh] = __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8));
-            else
-              vreg[ks][kk][hh] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-      }
-    }
-
-    uint32_t wd[W];
-    float gk = 0.0f;
-    if (valid) {
-#pragma unroll
-      for (int w = 0; w < W; ++w) wd[w] = __ldg(pk + static_cast<int64_t>(w) * a.cache_cap + key);
-      gk = __ldg(gm + key);
-    } else {
-#pragma unroll
-      for (int w = 0; w < W; ++w) wd[w] = 0u;
-    }
-
-    float lg[G];
-#pragma unroll
-    for (int r = 0; r < G; ++r) lg[r] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < T; ++i) {
-      constexpr uint32_t mask = (1u << C) - 1u;
-      const int pos = i * C, wi = pos >> 5, sh = pos & 31;
-      uint32_t code;
-      if (sh + C <= 32) code = (wd[wi] >> sh) & mask;
-      else code = __funnelshift_r(wd[wi], wd[wi + 1], sh) & mask;
-      float4 u;
-      if constexpr (Cfg::FOLD) {
-        u = table[code * REP + rep_off];
-      } else {
-        const float4 n = table[(code & ((1u << (2 * BD)) - 1u)) * REP + rep_off];
-        const float rh = s_rho_c[code >> (2 * BD)];
-        u = make_float4(n.x * rh, n.y * rh, n.z * rh, 0.0f);
-      }
-#pragma unroll
-      for (int r = 0; r < G; ++r) {
-        const float4 qv = qt[i * G + r];
-        lg[r] = fmaf(qv.x, u.x, fmaf(qv.y, u.y, fmaf(qv.z, u.z, lg[r])));
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < G; ++r) lg[r] *= gk;
-
-    if constexpr (QJL) {
-      float corr[4 * GV];
-#pragma unroll
-      for (int r = 0; r < 4 * GV; ++r) corr[r] = 0.0f;
-      uint32_t qb[QW];
-      float nu = 0.0f;
-      if (valid) {
-        const uint32_t* qbp = a.qjl_bits + static_cast<int64_t>(bh) * QW * a.cache_cap;
-#pragma unroll
-        for (int w = 0; w < QW; ++w) qb[w] = __ldg(qbp + static_cast<int64_t>(w) * a.cache_cap + key);
-        nu = __ldg(a.qjl_norm + static_cast<int64_t>(bh) * a.cache_cap + key);
-      } else {
-#pragma unroll
-        for (int w = 0; w < QW; ++w) qb[w] = 0u;
-      }
-#pragma unroll
-      for (int j = 0; j < D / 4; ++j) {
-        const uint32_t nib = (qb[j >> 3] >> (4 * (j & 7))) & 15u;
-#pragma unroll
-        for (int v4 = 0; v4 < GV; ++v4) {
-          const float4 t = lut[(j * 16 + nib) * GV + v4];
-          corr[4 * v4] += t.x; corr[4 * v4 + 1] += t.y; corr[4 * v4 + 2] += t.z; corr[4 * v4 + 3] += t.w;
-        }
-      }
-      const float f = gk * nu * (1.2533141373155003f / static_cast<float>(D));  // sqrt(pi/2)/m, m = d
-#pragma unroll
-      for (int r = 0; r < G; ++r) lg[r] = fmaf(f, corr[r], lg[r]);
-    }
-
-    if (a.logits != nullptr && valid) {
-#pragma unroll
-      for (int r = 0; r < G; ++r) {
-        if (r < a.Gq) {
-          const int gi = r / a.Lq, lq = r - gi * a.Lq;
-          const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-          a.logits[row * a.kv_len + key] = lg[r];
-        }
-      }
-    }
-    if (!with_v) continue;
-
-    // online softmax, base 2
-    float alpha[G];
-#pragma unroll
-    for (int r = 0; r < G; ++r) {
-      const float z = valid ? lg[r] * a.scale_log2 : -INFINITY;
-      const float mn = fmaxf(m_run[r], warp_max(z));
-      alpha[r] = exp2f(m_run[r] - mn);  // m_run = -inf -> 0
-      const float p = valid ? exp2f(z - mn) : 0.0f;
-      l_run[r] = l_run[r] * alpha[r] + p;
-      m_run[r] = mn;
-      pw[r * PS + lane] = p;
-    }
-    // this lane's accumulator columns are query rows 2*c4 and 2*c4+1
-    float sa0 = 0.0f, sa1 = 0.0f;
-#pragma unroll
-    for (int r = 0; r < G; ++r) {
-      sa0 = (r == 2 * c4) ? alpha[r] : sa0;
-      sa1 = (r == 2 * c4 + 1) ? alpha[r] : sa1;
-    }
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      acc_o[t][0] *= sa0; acc_o[t][1] *= sa1; acc_o[t][2] *= sa0; acc_o[t][3] *= sa1;
-    }
-    __syncwarp();
-
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
-      if (g8 < G) {
-        const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
-        const float2 p01 = *reinterpret_cast<const float2*>(prow);
-        const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
-        split_bf16x2(p01.x, p01.y, bh0, bl0);
-        split_bf16x2(p89.x, p89.y, bh1, bl1);
-      }
-#pragma unroll
-      for (int hh = 0; hh < NCH; ++hh) {
-        const uint4 k0 = vreg[ks][0][hh], k1 = vreg[ks][1][hh], k8 = vreg[ks][2][hh], k9 = vreg[ks][3][hh];
-        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-        const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
-          const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
-          const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
-          const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
-          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
-        }
-      }
-    }
-    __syncwarp();
-  }
-
-  if (!with_v) return;
-
-  // ------------------------------------------------ epilogue: merge warps
-#pragma unroll
-  for (int r = 0; r < G; ++r) l_run[r] = warp_sum(l_run[r]);
-  __syncthreads();  // every warp is done with the table that `merge` aliases
-  float* wm = merge;                                // [NWARP][G]
-  float* wl = merge + NWARP * G;                    // [NWARP][G]
-  float* wo = merge + 2 * NWARP * G;                // [NWARP][G][D]
-  if (lane == 0) {
-#pragma unroll
-    for (int r = 0; r < G; ++r) { wm[warp * G + r] = m_run[r]; wl[warp * G + r] = l_run[r]; }
-  }
-#pragma unroll
-  for (int t = 0; t < MT; ++t) {
-    const int hh = t >> 2, e2 = t & 3;
-    const int d0 = 64 * hh + 8 * g8 + 2 * e2;
-    const int q0 = 2 * c4, q1 = 2 * c4 + 1;
-    if (q0 < G) { wo[(warp * G + q0) * D + d0] = acc_o[t][0]; wo[(warp * G + q0) * D + d0 + 1] = acc_o[t][2]; }
-    if (q1 < G) { wo[(warp * G + q1) * D + d0] = acc_o[t][1]; wo[(warp * G + q1) * D + d0 + 1] = acc_o[t][3]; }
-  }
-  __syncthreads();
-
-  const int S = a.n_splits;
-  float* pm = a.part_m + (static_cast<int64_t>(bh) * S + split) * G;
-  float* pl = a.part_l + (static_cast<int64_t>(bh) * S + split) * G;
-  float* po = a.part_o + (static_cast<int64_t>(bh) * S + split) * G * D;
-  for (int j = tid; j < G * D; j += Cfg::THREADS) {
-    const int r = j / D, d = j - r * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NWARP; ++w) M = fmaxf(M, wm[w * G + r]);
-    float o = 0.0f, l = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NWARP; ++w) {
-        const float f = exp2f(wm[w * G + r] - M);
-        o = fmaf(f, wo[(w * G + r) * D + d], o);
-        l = fmaf(f, wl[w * G + r], l);
-      }
-    }
-    if (S == 1) {
-      if (r < a.Gq) {
-        const int gi = r / a.Lq, lq = r - gi * a.Lq;
-        const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-        a.out[row * D + d] = l > 0.0f ? o / l : 0.0f;
-      }
-    } else {
-      po[j] = o;
-      if (d == 0) { pm[r] = M; pl[r] = l; }
-    }
-  }
-  if (S == 1) return;
-
-  // ------------------------------------------------ epilogue: merge splits (last CTA of this head)
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int ticket = atomicAdd(a.counters + bh, 1);
-    s_last = ticket == S - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
-  const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
-  const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
-  for (int j = tid; j < G * D; j += Cfg::THREADS) {
-    const int r = j / D, d = j - r * D;
-    if (r >= a.Gq) continue;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(bm + s * G + r));
-    float o = 0.0f, l = 0.0f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float f = exp2f(__ldcg(bm + s * G + r) - M);
-        o = fmaf(f, __ldcg(bo + (static_cast<int64_t>(s) * G + r) * D + d), o);
-        l = fmaf(f, __ldcg(bl + s * G + r), l);
-      }
-    }
-    const int gi = r / a.Lq, lq = r - gi * a.Lq;
-    const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-    a.out[row * D + d] = l > 0.0f ? o / l : 0.0f;
-  }
-  if (tid == 0) a.counters[bh] = 0;  // ready for the next call
-}
 
 // ---------------------------------------------------------------------------
 // host side
@@ -493,9 +18,6 @@ struct Plan {
   int64_t keys_per_split;
   size_t smem;
 };
-
-template <int D, int B, int G, bool QJL>
-size_t smem_of() { return DecCfg<D, B, G, QJL>::SMEM; }
 
 static int sm_count() {
   int dev = 0, sms = 148;
@@ -517,7 +39,7 @@ static void choose_splits(int64_t heads, int64_t kv_len, int sms, int& n_splits,
     if (cost < best - 1e-12) { best = cost; best_s = s; }
   }
   per = (kv_len + best_s - 1) / best_s;
-  per = ((per + 31) / 32) * 32;
+  per = ((per + 127) / 128) * 128;  // whole warp iterations (128 keys at 4 keys per lane)
   n_splits = static_cast<int>(std::max<int64_t>(1, (kv_len + per - 1) / per));
 }
 
@@ -550,39 +72,6 @@ int check_layout(const octo_layout* L) {
   if (octo_layout_init(&chk, L->d, L->b, L->qjl, L->rounding) != OCTO_OK) return OCTO_EINVAL;
   if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits) return OCTO_EINVAL;
   return OCTO_OK;
-}
-
-template <int D, int B, int G, bool QJL>
-cudaError_t launch(const octo::DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  using Cfg = octo::DecCfg<D, B, G, QJL>;
-  auto k = octo::decode_kernel<D, B, G, QJL>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
-  if (e != cudaSuccess) return e;
-  k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a);
-  return cudaGetLastError();
-}
-
-template <int D, int B, int G>
-cudaError_t launch_q(const octo::DecodeArgs& a, bool qjl, dim3 grid, cudaStream_t st) {
-  return qjl ? launch<D, B, G, true>(a, grid, st) : launch<D, B, G, false>(a, grid, st);
-}
-
-template <int D, int B>
-cudaError_t launch_g(const octo::DecodeArgs& a, int G, bool qjl, dim3 grid, cudaStream_t st) {
-  switch (G) {
-    case 1: return launch_q<D, B, 1>(a, qjl, grid, st);
-    case 4: return launch_q<D, B, 4>(a, qjl, grid, st);
-    default: return launch_q<D, B, 8>(a, qjl, grid, st);
-  }
-}
-
-template <int D>
-cudaError_t launch_b(const octo::DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st) {
-  switch (b) {
-    case 2: return launch_g<D, 2>(a, G, qjl, grid, st);
-    case 3: return launch_g<D, 3>(a, G, qjl, grid, st);
-    default: return launch_g<D, 4>(a, G, qjl, grid, st);
-  }
 }
 
 }  // namespace
@@ -672,9 +161,9 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   const dim3 grid(static_cast<unsigned>(a.n_splits), static_cast<unsigned>(heads));
   cudaError_t e;
   switch (D) {
-    case 64: e = launch_b<64>(a, L->b, G, L->qjl != 0, grid, st); break;
-    case 128: e = launch_b<128>(a, L->b, G, L->qjl != 0, grid, st); break;
-    default: e = launch_b<256>(a, L->b, G, L->qjl != 0, grid, st); break;
+    case 64: e = octo::launch_decode_d64(a, L->b, G, L->qjl != 0, grid, st); break;
+    case 128: e = octo::launch_decode_d128(a, L->b, G, L->qjl != 0, grid, st); break;
+    default: e = octo::launch_decode_d256(a, L->b, G, L->qjl != 0, grid, st); break;
   }
   return e == cudaSuccess ? OCTO_OK : OCTO_ECUDA;
 }
