@@ -156,8 +156,9 @@ OCTO_API int octo_encode(const octo_layout* L, const octo_tables* tables,
                 uint32_t* packed, float* gamma, uint32_t* qjl_bits, float* qjl_norm,
                 octo_stream_t stream);
 
-/* Bytes of device workspace octo_decode_attn needs for these sizes (0 in
- * logits-only use). Returns 0 for unsupported arguments. */
+/* Bytes of device workspace octo_decode_attn needs for these sizes (at
+ * least 256: the workspace also carries a status word). Returns 0 for
+ * unsupported arguments. */
 OCTO_API size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq, int Hkv, int Lq, int64_t kv_len);
 
 /* Device. One fused decode-attention step over a compressed cache
@@ -171,20 +172,25 @@ OCTO_API size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq, 
  *   Hq = g*Hkv; query head hq reads KV head hq / g. Cache head index is
  *   b*Hkv + h_kv in packed / gamma / qjl_* / V.
  *   packed, gamma, qjl_bits, qjl_norm: the cache (layout above), capacity
- *   cache_cap, the first kv_len tokens are attended.
- *   V        device bf16 [B*Hkv][cache_cap][d] (16-byte aligned rows), or
- *            NULL for logits only.
+ *   cache_cap, the first kv_len tokens are attended. The code rows are
+ *   staged into shared memory by 16-byte bulk copies, so cache_cap must be
+ *   a multiple of 4 and these four base addresses 16-byte aligned.
+ *   V        device bf16 [B*Hkv][cache_cap][d] (16-byte aligned), or NULL
+ *            for logits only.
  *   scale    softmax temperature (1/sqrt(d) for standard attention).
  *   out      device fp32 [B][Hq][Lq][d]; required iff V != NULL.
  *   logits   device fp32 [B][Hq][Lq][kv_len] raw (unscaled) logits, or NULL.
- *   workspace device, >= octo_decode_attn_workspace() bytes when V != NULL,
- *            256-byte aligned. Its first 4*B*Hkv bytes are arrival counters
- *            that must be zero before the first call (e.g. cudaMemset);
- *            every completed call leaves them zero again. Calls that share
+ *   workspace device, >= octo_decode_attn_workspace() bytes, 256-byte
+ *            aligned, always required. Bytes [0, 4) are a status word: the
+ *            kernel ORs in 1 if one of its bounded on-chip waits expired
+ *            (the outputs of that call are then invalid). Bytes [256, 256 +
+ *            4*B*Hkv) are arrival counters. Status and counters must be zero
+ *            before the first call (zero the whole workspace once); every
+ *            completed call leaves the counters zero again. Calls that share
  *            a workspace must not overlap on the GPU.
  * kv_len == 0 gives out = 0. Errors: OCTO_EINVAL (NULL required pointer,
  * bad sizes, kv_len > cache_cap, both V and logits NULL, misalignment),
- * OCTO_EUNSUPPORTED (g*Lq > 8), OCTO_EWORKSPACE. */
+ * OCTO_EUNSUPPORTED (g*Lq > 8 or B*Hkv > 65535), OCTO_EWORKSPACE. */
 OCTO_API int octo_decode_attn(const octo_layout* L, const octo_tables* tables,
                      const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
                      int64_t kv_len, int64_t cache_cap,

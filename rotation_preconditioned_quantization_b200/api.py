@@ -122,6 +122,9 @@ class Cache:
 
     @classmethod
     def empty(cls, layout: Layout, n_heads: int, cap: int, device="cuda"):
+        """Zeroed cache; the capacity is rounded up to a multiple of 4 tokens
+        (decode stages code rows with 16-byte copies)."""
+        cap = (int(cap) + 3) // 4 * 4
         packed = torch.zeros((n_heads, layout.words, cap), dtype=torch.int32, device=device)
         gamma = torch.zeros((n_heads, cap), dtype=torch.float32, device=device)
         qb = qn = None
@@ -168,15 +171,23 @@ def decode_attn_workspace_bytes(layout: Layout, B: int, Hq: int, Hkv: int, Lq: i
 
 
 class Workspace:
-    """Device workspace for decode_attn; its ticket counters start (and stay) zero."""
+    """Device workspace for decode_attn: status word, ticket counters (zeroed
+    here, left zero by every completed call) and split partials."""
 
     def __init__(self, nbytes: int, device="cuda"):
-        n = max(256, (int(nbytes) + 255) // 256 * 256)
+        n = max(512, (int(nbytes) + 255) // 256 * 256)
         self.buf = torch.zeros(n // 4, dtype=torch.int32, device=device)
 
     @property
     def nbytes(self) -> int:
         return self.buf.numel() * 4
+
+    def status(self) -> int:
+        """Device status word (synchronises): nonzero if a bounded on-chip wait expired."""
+        return int(self.buf[0].item())
+
+    def counters(self, n_heads: int) -> torch.Tensor:
+        return self.buf[64:64 + n_heads]
 
     def ensure(self, nbytes: int):
         if nbytes > self.nbytes:
@@ -212,13 +223,11 @@ def decode_attn(layout: Layout, tables: DeviceTables, q: torch.Tensor, cache: Ca
         logits = torch.empty((B, Hq, Lq, kv), dtype=torch.float32, device=q.device)
     elif logits is False:
         logits = None
-    ws_ptr, ws_n = None, 0
-    if V is not None:
-        need = decode_attn_workspace_bytes(layout, B, Hq, Hkv, Lq, kv)
-        if workspace is None:
-            workspace = Workspace(need, q.device)
-        workspace.ensure(need)
-        ws_ptr, ws_n = _ptr(workspace.buf), workspace.nbytes
+    need = decode_attn_workspace_bytes(layout, B, Hq, Hkv, Lq, kv)
+    if workspace is None:
+        workspace = Workspace(need, q.device)
+    workspace.ensure(need)
+    ws_ptr, ws_n = _ptr(workspace.buf), workspace.nbytes
     st = _lib.lib().octo_decode_attn(layout.ref, tables.ref, _ptr(q), qdt, B, Hq, Hkv, Lq, kv, cache.cap,
                                      _ptr(cache.packed), _ptr(cache.gamma), _ptr(cache.qjl_bits), _ptr(cache.qjl_norm),
                                      _ptr(V), ctypes.c_float(scale), _ptr(out), _ptr(logits), ws_ptr, ws_n,

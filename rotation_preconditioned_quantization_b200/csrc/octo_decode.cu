@@ -12,13 +12,6 @@ namespace octo {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-struct Plan {
-  int G;          // template rows (1, 4 or 8)
-  int n_splits;
-  int64_t keys_per_split;
-  size_t smem;
-};
-
 static int sm_count() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -39,7 +32,7 @@ static void choose_splits(int64_t heads, int64_t kv_len, int sms, int& n_splits,
     if (cost < best - 1e-12) { best = cost; best_s = s; }
   }
   per = (kv_len + best_s - 1) / best_s;
-  per = ((per + 127) / 128) * 128;  // whole warp iterations (128 keys at 4 keys per lane)
+  per = ((per + 63) / 64) * 64;  // slices start at multiples of 64 keys (16-byte aligned copies)
   n_splits = static_cast<int>(std::max<int64_t>(1, (kv_len + per - 1) / per));
 }
 
@@ -49,15 +42,18 @@ static int rows_template(int Gq) { return Gq <= 1 ? 1 : (Gq <= 4 ? 4 : 8); }
 
 namespace {
 
+// Workspace: a status word (own 256-byte line), the per-head arrival
+// counters, then the per-split (m, l) and O partials.
 struct WsLayout {
-  size_t counters, m, l, o, total;
+  size_t status, counters, m, l, o, total;
 };
 
 WsLayout ws_layout(int64_t heads, int n_splits, int G, int D) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   WsLayout w{};
-  w.counters = 0;
-  w.m = up(sizeof(int) * heads);
+  w.status = 0;
+  w.counters = 256;
+  w.m = w.counters + up(sizeof(int) * heads);
   w.l = w.m + up(sizeof(float) * heads * n_splits * G);
   w.o = w.l + up(sizeof(float) * heads * n_splits * G);
   w.total = w.o + up(sizeof(float) * heads * n_splits * G * D);
@@ -103,7 +99,12 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   if (!V && !logits) return OCTO_EINVAL;
   if (V && !out) return OCTO_EINVAL;
   if (L->qjl && (!qjl_bits || !qjl_norm || !tab->qjl_S)) return OCTO_EINVAL;
-  if (V && (reinterpret_cast<uintptr_t>(V) % 16 != 0)) return OCTO_EINVAL;
+  auto misaligned = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 != 0; };
+  if (V && misaligned(V)) return OCTO_EINVAL;
+  // code rows are staged by 16-byte bulk copies
+  if (cache_cap % 4 != 0 || misaligned(packed) || misaligned(gamma)) return OCTO_EINVAL;
+  if (L->qjl && (misaligned(qjl_bits) || misaligned(qjl_norm))) return OCTO_EINVAL;
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return OCTO_EINVAL;
   if (!(scale == scale)) return OCTO_EINVAL;
   const int g = Hq / Hkv, Gq = g * Lq;
   if (Gq > 8) return OCTO_EUNSUPPORTED;
@@ -141,23 +142,15 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.table_heads = tab->n_heads;
   const int G = octo::rows_template(Gq);
 
-  if (V) {
-    octo::choose_splits(heads, kv_len, octo::sm_count(), a.n_splits, a.keys_per_split);
-    const WsLayout w = ws_layout(heads, a.n_splits, G, D);
-    if (a.n_splits > 1) {
-      if (!workspace) return OCTO_EINVAL;
-      if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return OCTO_EINVAL;
-      if (ws_bytes < w.total) return OCTO_EWORKSPACE;
-      char* base = static_cast<char*>(workspace);
-      a.counters = reinterpret_cast<int*>(base + w.counters);
-      a.part_m = reinterpret_cast<float*>(base + w.m);
-      a.part_l = reinterpret_cast<float*>(base + w.l);
-      a.part_o = reinterpret_cast<float*>(base + w.o);
-    }
-  } else {
-    // logits only: no softmax state, slices just spread the work
-    octo::choose_splits(heads, kv_len, octo::sm_count(), a.n_splits, a.keys_per_split);
-  }
+  octo::choose_splits(heads, kv_len, octo::sm_count(), a.n_splits, a.keys_per_split);
+  const WsLayout w = ws_layout(heads, a.n_splits, G, D);
+  if (ws_bytes < w.total) return OCTO_EWORKSPACE;
+  char* base = static_cast<char*>(workspace);
+  a.status = reinterpret_cast<int*>(base + w.status);
+  a.counters = reinterpret_cast<int*>(base + w.counters);
+  a.part_m = reinterpret_cast<float*>(base + w.m);
+  a.part_l = reinterpret_cast<float*>(base + w.l);
+  a.part_o = reinterpret_cast<float*>(base + w.o);
   const dim3 grid(static_cast<unsigned>(a.n_splits), static_cast<unsigned>(heads));
   cudaError_t e;
   switch (D) {

@@ -1,4 +1,4 @@
-// OCTOPUS fused decode attention for sm_100a.
+// OCTOPUS fused decode attention for sm_100a: the kernel template.
 //
 // One step of decode attention over a compressed key cache (explainer,
 // "engineering implementation": decompression, dot products and online
@@ -13,24 +13,32 @@
 // Because R is orthogonal, q . k_hat = gamma q_rot . u_rot_hat, so the keys
 // are never inverse-rotated.
 //
-// Structure (one CTA = one KV head x one contiguous slice of the cache):
-//  * prologue: codebooks -> a shared-memory table of decoded triplets
-//    (rho_hat * n_hat for every full code when 3b+1 <= 10 bits, else n_hat
-//    for every direction code plus a rho_hat lookup), replicated 8x so that
-//    the 8 lanes of a quarter-warp read distinct bank groups (conflict-free
-//    128-bit loads); queries rotated by warp-shuffle WHT into a
+// Structure (one CTA = one KV head x one contiguous slice of the cache,
+// 8 warps, every warp a consumer, thread 0 also the producer):
+//  * The slice is cut into stages of CK = 512 keys. For each stage thread 0
+//    issues TMA bulk copies (cp.async.bulk, completion on an mbarrier) of the
+//    stage's code words and gammas (and sketch words and residual norms)
+//    into a ring of NS shared-memory buffers, and a bulk L2 prefetch of the
+//    stage's V rows. NS stages are in flight; a buffer is refilled after the
+//    block-wide barrier that ends its stage.
+//  * prologue (overlapping the first copies): codebooks -> a shared-memory
+//    table of decoded triplets, replicated 8x so that the 8 lanes of a
+//    quarter-warp read distinct bank groups (b = 2: rho_hat * n_hat for every
+//    full code; b >= 3: n_hat for every direction code, rho_hat from a
+//    4/8-entry table); queries rotated by warp-shuffle WHT into a compact
 //    triplet-major layout; for QJL, p = S q_rot and a 4-bit lookup table of
 //    signed partial sums of p.
-//  * main loop, one warp per 32-key chunk, one lane per key: coalesced
-//    loads of the token-contiguous code words, gamma (and sketch); logits by
-//    table lookups and FMAs; online softmax (m, l) per query row; P.V on
-//    tensor cores (mma.sync m16n8k16 bf16, P split into bf16 hi + lo parts so
-//    the product keeps ~16 mantissa bits) with V read straight from global
-//    memory into A-fragment registers (16-byte loads + byte permutes).
-//  * epilogue: warps merge (m, l, O) in shared memory; CTAs of a head merge
+//  * per stage and warp: 64 keys, two per lane. Logits by table lookups and
+//    FMAs; online softmax (m, l) per query row in base 2; P.V on tensor
+//    cores (mma.sync m16n8k16 bf16; P split into bf16 hi + lo so the product
+//    keeps ~16 mantissa bits) with V read from L2 straight into A-fragment
+//    registers (16-byte loads + byte permutes).
+//  * epilogue: warps merge (m, l, O) in shared memory (reusing the stage
+//    ring); CTAs of a head merge
 //    through the workspace, the last-arriving CTA (atomic ticket, no
 //    spinning) writes the normalised output and resets the ticket.
-
+//  * Every wait on an mbarrier is bounded; on expiry the kernel records
+//    OCTO_DEVICE_TIMEOUT in the workspace status word and returns.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -40,6 +48,8 @@
 #include "octo_common.cuh"
 
 namespace octo {
+
+constexpr int OCTO_DEVICE_TIMEOUT = 1;  // status-word bit: a bounded device wait expired
 
 struct DecodeArgs {
   const void* q;
@@ -61,6 +71,7 @@ struct DecodeArgs {
   int64_t table_heads;
   int n_splits;
   int64_t keys_per_split;
+  int* status;
   int* counters;
   float* part_m;
   float* part_l;
@@ -74,12 +85,13 @@ struct DecCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr bool FOLD = C <= 10;                    // table indexed by the full code
+  static constexpr bool FOLD = C <= 7;                     // b = 2: table indexed by the full code
   static constexpr int NE = FOLD ? (1 << C) : (1 << (2 * BD));
-  static constexpr int REP = 8;
-  static constexpr int THREADS = 512, NWARP = THREADS / 32;
-  static constexpr int KPL = (G <= 4 && D <= 128) ? 4 : 2;  // keys per lane per iteration
-  static constexpr int KW = 32 * KPL;                      // keys per warp per iteration
+  static constexpr int REP = NE <= 256 ? 8 : 4;           // replicas per entry (bank groups)
+  static constexpr int THREADS = 256, NWARP = THREADS / 32;
+  static constexpr int KPL = D <= 128 ? 2 : 1;             // keys per lane per stage
+  static constexpr int KW = 32 * KPL;                      // keys per warp per stage
+  static constexpr int CK = KW * NWARP;                    // keys per stage (512, 256 for d = 256)
   static constexpr int QF = 3 * G;                         // rotated-query floats per triplet
   static constexpr int QV = (QF + 3) / 4;                  // ... as float4
   static constexpr int QW = D / 32;                        // sketch words per key
@@ -87,20 +99,24 @@ struct DecCfg {
   static constexpr int MT = D / 16;                        // m-tiles of O^T
   static constexpr int NCH = D / 64;                       // 16-byte V chunks per key per lane
   static constexpr int GV = (G + 3) / 4;                   // float4 per LUT entry
-  // shared memory carve-up (bytes)
-  // region 0 holds the decoded-triplet table during the main loop and the
-  // warps' (m, l, O) afterwards; scratch holds the rotated query rows (and
-  // p = S q_rot for QJL) during the prologue.
+  // one stage buffer: W code rows, a gamma row (+ QW sketch rows, a norm row)
+  static constexpr int STAGE_ROWS = W + 1 + (QJL ? QW + 1 : 0);
+  static constexpr size_t STAGE = sizeof(uint32_t) * STAGE_ROWS * CK;
+  // shared memory carve-up (bytes): the stage ring is reused for the warps'
+  // (m, l, O) once the main loop is over
   static constexpr size_t TABLE = sizeof(float4) * NE * REP;
   static constexpr size_t MERGE = sizeof(float) * NWARP * G * (D + 2);
-  static constexpr size_t REGION0 = TABLE > MERGE ? TABLE : MERGE;
   static constexpr size_t QT = sizeof(float4) * T * QV;
   static constexpr size_t PBUF = sizeof(float) * NWARP * G * PSTRIDE;
   static constexpr size_t LUT = QJL ? sizeof(float4) * (D / 4) * 16 * GV : 0;
-  static constexpr size_t QROW = D + 4;                       // floats per scratch query row
+  static constexpr size_t QROW = D + 4;                    // floats per scratch query row
   static constexpr size_t SCRATCH = sizeof(float) * G * (QROW + (QJL ? D : 0));
-  static constexpr size_t SMEM = REGION0 + QT + PBUF + LUT + SCRATCH;
-  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static constexpr size_t FIXED = TABLE + QT + PBUF + LUT + SCRATCH;
+  static constexpr size_t BUDGET = 227 * 1024 - 1024;
+  static constexpr size_t ring(int ns) { return ns * STAGE > MERGE ? ns * STAGE : MERGE; }
+  static constexpr int NS = FIXED + ring(3) <= BUDGET ? 3 : 2;  // stages in flight
+  static constexpr size_t SMEM = FIXED + ring(NS);
+  static_assert(SMEM <= BUDGET, "shared memory budget");
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -132,35 +148,72 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+// ---- mbarrier / bulk-copy helpers (PTX) -----------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// Prefetch [p, p + bytes) into L2, one 128-byte line per lane per step.
-__device__ __forceinline__ void prefetch_range_l2(const void* p, int64_t bytes, int lane) {
-  const char* c = static_cast<const char*>(p);
-  for (int64_t off = static_cast<int64_t>(lane) * 128; off < bytes; off += 32 * 128) prefetch_l2(c + off);
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false if the phase did not complete within the limit.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  for (int it = 0; it < (1 << 22); ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// global -> shared bulk copy completing on `bar`; 16-byte aligned, size % 16 == 0
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 template <int D, int B, int G, bool QJL>
-__global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
   using Cfg = DecCfg<D, B, G, QJL>;
   constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, BD = Cfg::BD, NDIR = Cfg::NDIR;
   constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, QW = Cfg::QW;
   constexpr int PS = Cfg::PSTRIDE, MT = Cfg::MT, NCH = Cfg::NCH, GV = Cfg::GV;
-  constexpr int KPL = Cfg::KPL, KW = Cfg::KW, QV = Cfg::QV;
+  constexpr int KPL = Cfg::KPL, KW = Cfg::KW, CK = Cfg::CK, QV = Cfg::QV, NS = Cfg::NS;
+  constexpr int ROWS = Cfg::STAGE_ROWS;
 
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   float4* table = reinterpret_cast<float4*>(smem_raw);                                   // [NE*REP]
-  float* merge = reinterpret_cast<float*>(smem_raw);                                     // aliases table
-  float4* qt = reinterpret_cast<float4*>(smem_raw + Cfg::REGION0);                       // [T][QV]
-  float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::REGION0 + Cfg::QT);             // [NWARP][G][PS]
-  float4* lut = reinterpret_cast<float4*>(smem_raw + Cfg::REGION0 + Cfg::QT + Cfg::PBUF);  // [D/4][16][GV]
-  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::REGION0 + Cfg::QT + Cfg::PBUF + Cfg::LUT);
+  float4* qt = reinterpret_cast<float4*>(smem_raw + Cfg::TABLE);                         // [T][QV]
+  float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + Cfg::QT);               // [NWARP][G][PS]
+  float4* lut = reinterpret_cast<float4*>(smem_raw + Cfg::TABLE + Cfg::QT + Cfg::PBUF);    // [D/4][16][GV]
+  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + Cfg::QT + Cfg::PBUF + Cfg::LUT);
+  uint32_t* stages = reinterpret_cast<uint32_t*>(smem_raw + Cfg::FIXED);                 // [NS][ROWS][CK]
+  float* merge = reinterpret_cast<float*>(smem_raw + Cfg::FIXED);                        // aliases the ring
   constexpr int QROW = static_cast<int>(Cfg::QROW);
+  __shared__ __align__(8) uint64_t full[NS];
   __shared__ float s_rho_c[8];
   __shared__ float s_dir_c[32];
   __shared__ int s_last;
+  __shared__ int s_abort;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x;
@@ -171,32 +224,47 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
 
   const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
   const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
+  const int n_stages = static_cast<int>((k_end - k_begin + CK - 1) / CK);
   const uint32_t* pk = a.packed + static_cast<int64_t>(bh) * W * a.cache_cap;
   const float* gm = a.gamma + static_cast<int64_t>(bh) * a.cache_cap;
   const __nv_bfloat16* Vh = with_v ? a.V + static_cast<int64_t>(bh) * a.cache_cap * D : nullptr;
   const uint32_t* qbp = QJL ? a.qjl_bits + static_cast<int64_t>(bh) * QW * a.cache_cap : nullptr;
   const float* qnp = QJL ? a.qjl_norm + static_cast<int64_t>(bh) * a.cache_cap : nullptr;
 
-  // Stream this warp's keys [s, e) into L2 ahead of use: code words, gamma
-  // (and sketch) and, with V, the value rows.
-  auto prefetch_keys = [&](int64_t s, int64_t e, bool values) {
-    if (s >= e) return;
-    const int64_t n = e - s;
+  // Producer (thread 0): copy stage st's rows into buffer st % NS. Keys are
+  // copied in groups of 4 (16 bytes); the cache capacity is a multiple of 4
+  // and stages start at multiples of 64, so the rounded-up copy stays
+  // inside the cache rows (keys past kv_len are masked by the consumers).
+  auto issue_stage = [&](int st) {
+    const int64_t s0 = k_begin + static_cast<int64_t>(st) * CK;
+    const int n = static_cast<int>(k_end - s0 < CK ? k_end - s0 : CK);
+    const uint32_t bytes = static_cast<uint32_t>(((n + 3) & ~3) * 4);
+    uint32_t* buf = stages + (st % NS) * ROWS * CK;
+    uint64_t* bar = &full[st % NS];
+    mbar_expect_tx(bar, bytes * ROWS);
 #pragma unroll 1
-    for (int w = 0; w < W; ++w) prefetch_range_l2(pk + w * a.cache_cap + s, n * 4, lane);
-    prefetch_range_l2(gm + s, n * 4, lane);
+    for (int w = 0; w < W; ++w) bulk_g2s(buf + w * CK, pk + w * a.cache_cap + s0, bytes, bar);
+    bulk_g2s(buf + W * CK, gm + s0, bytes, bar);
     if constexpr (QJL) {
 #pragma unroll 1
-      for (int w = 0; w < QW; ++w) prefetch_range_l2(qbp + w * a.cache_cap + s, n * 4, lane);
-      prefetch_range_l2(qnp + s, n * 4, lane);
+      for (int w = 0; w < QW; ++w) bulk_g2s(buf + (W + 1 + w) * CK, qbp + w * a.cache_cap + s0, bytes, bar);
+      bulk_g2s(buf + (W + 1 + QW) * CK, qnp + s0, bytes, bar);
     }
-    if (values && with_v) prefetch_range_l2(Vh + s * D, n * D * 2, lane);
+    if (with_v) bulk_prefetch_l2(Vh + s0 * D, static_cast<uint32_t>(n) * D * 2);
   };
-  // first iteration of every warp: start HBM traffic before the prologue
-  prefetch_keys(k_begin + static_cast<int64_t>(KW) * warp,
-                min(k_end, k_begin + static_cast<int64_t>(KW) * (warp + 1)), true);
 
-  // ------------------------------------------------ prologue
+  if (tid == 0) {
+    s_abort = 0;
+#pragma unroll
+    for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int st = 0; st < NS && st < n_stages; ++st) issue_stage(st);
+  }
+
+  // ------------------------------------------------ prologue (overlaps the first copies)
   if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
   if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
   __syncthreads();
@@ -208,7 +276,7 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
       n.x *= r; n.y *= r; n.z *= r;
     }
     const float4 v = make_float4(n.x, n.y, n.z, 0.0f);
-    // replica order rotated by lane so that each store instruction hits 8 bank groups
+    // replica order rotated by lane so that each store instruction hits distinct bank groups
 #pragma unroll
     for (int k = 0; k < REP; ++k) table[e * REP + ((k + lane) & (REP - 1))] = v;
   }
@@ -279,7 +347,7 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
 
-  // ------------------------------------------------ main loop
+  // ------------------------------------------------ main loop over stages
   const int g8 = lane >> 2, c4 = lane & 3;
   const int rep_off = lane & (REP - 1);
 
@@ -291,23 +359,29 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
   for (int t = 0; t < MT; ++t) acc_o[t][0] = acc_o[t][1] = acc_o[t][2] = acc_o[t][3] = 0.0f;
   float* pw = pbuf + warp * G * PS;
 
-  for (int64_t base = k_begin + static_cast<int64_t>(KW) * warp; base < k_end;
-       base += static_cast<int64_t>(KW) * NWARP) {
-    // next iteration's keys start streaming now; this iteration's values too
-    {
-      const int64_t nb = base + static_cast<int64_t>(KW) * NWARP;
-      prefetch_keys(nb, min(k_end, nb + KW), false);
-      if (base != k_begin + static_cast<int64_t>(KW) * warp && with_v)
-        prefetch_range_l2(Vh + base * D, (min(k_end, base + KW) - base) * D * 2, lane);
+  for (int st = 0; st < n_stages; ++st) {
+    const uint32_t* buf = stages + (st % NS) * ROWS * CK;
+    const int64_t s0 = k_begin + static_cast<int64_t>(st) * CK;
+    // every thread acquires the stage's data; an expired wait aborts the whole CTA
+    if (!mbar_wait_bounded(&full[st % NS], (st / NS) & 1)) s_abort = 1;  // benign race: all write 1
+    __syncthreads();
+    if (s_abort) {
+      if (tid == 0) {
+        atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
+        // let the copies already issued land before the shared memory is released
+        for (int s2 = st + 1; s2 < n_stages && s2 < st + NS; ++s2) mbar_wait_bounded(&full[s2 % NS], (s2 / NS) & 1);
+      }
+      break;
     }
-    int64_t key[KPL];
+    if (s0 + warp * KW < k_end) {  // this warp has keys in the stage (all but the tail stage)
+    int lk[KPL];
     bool valid[KPL];
     float gk[KPL];
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
-      key[k] = base + 32 * k + lane;
-      valid[k] = key[k] < k_end;
-      gk[k] = valid[k] ? __ldg(gm + key[k]) : 0.0f;
+      lk[k] = warp * KW + 32 * k + lane;
+      valid[k] = s0 + lk[k] < k_end;
+      gk[k] = valid[k] ? __uint_as_float(buf[W * CK + lk[k]]) : 0.0f;
     }
 
     float lg[KPL][G];
@@ -315,12 +389,6 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
     for (int k = 0; k < KPL; ++k)
 #pragma unroll
       for (int r = 0; r < G; ++r) lg[k][r] = 0.0f;
-
-    uint32_t wd[KPL][W];
-#pragma unroll
-    for (int w = 0; w < W; ++w)
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) wd[k][w] = valid[k] ? __ldg(pk + static_cast<int64_t>(w) * a.cache_cap + key[k]) : 0u;
 
 #pragma unroll
     for (int i = 0; i < T; ++i) {
@@ -335,8 +403,8 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
 #pragma unroll
       for (int k = 0; k < KPL; ++k) {
         uint32_t code;
-        if (sh + C <= 32) code = (wd[k][wi] >> sh) & mask;
-        else code = __funnelshift_r(wd[k][wi], wd[k][wi + 1], sh) & mask;
+        if (sh + C <= 32) code = (buf[wi * CK + lk[k]] >> sh) & mask;
+        else code = __funnelshift_r(buf[wi * CK + lk[k]], buf[(wi + 1) * CK + lk[k]], sh) & mask;
         float4 u;
         if constexpr (Cfg::FOLD) {
           u = table[code * REP + rep_off];
@@ -356,23 +424,24 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
 #pragma unroll
       for (int r = 0; r < G; ++r) lg[k][r] *= gk[k];
       if constexpr (QJL) {
-        uint32_t qb[QW];
-        float nu = 0.0f;
-#pragma unroll
-        for (int w = 0; w < QW; ++w) qb[w] = valid[k] ? __ldg(qbp + static_cast<int64_t>(w) * a.cache_cap + key[k]) : 0u;
-        if (valid[k]) nu = __ldg(qnp + key[k]);
         float corr[4 * GV];
 #pragma unroll
         for (int r = 0; r < 4 * GV; ++r) corr[r] = 0.0f;
 #pragma unroll
-        for (int j = 0; j < D / 4; ++j) {
-          const uint32_t nib = (qb[j >> 3] >> (4 * (j & 7))) & 15u;
+        for (int w = 0; w < QW; ++w) {
+          const uint32_t word = buf[(W + 1 + w) * CK + lk[k]];
 #pragma unroll
-          for (int v4 = 0; v4 < GV; ++v4) {
-            const float4 t = lut[(j * 16 + nib) * GV + v4];
-            corr[4 * v4] += t.x; corr[4 * v4 + 1] += t.y; corr[4 * v4 + 2] += t.z; corr[4 * v4 + 3] += t.w;
+          for (int j8 = 0; j8 < 8; ++j8) {
+            const uint32_t nib = (word >> (4 * j8)) & 15u;
+            const int j = 8 * w + j8;
+#pragma unroll
+            for (int v4 = 0; v4 < GV; ++v4) {
+              const float4 t = lut[(j * 16 + nib) * GV + v4];
+              corr[4 * v4] += t.x; corr[4 * v4 + 1] += t.y; corr[4 * v4 + 2] += t.z; corr[4 * v4 + 3] += t.w;
+            }
           }
         }
+        const float nu = valid[k] ? __uint_as_float(buf[(W + 1 + QW) * CK + lk[k]]) : 0.0f;
         const float f = gk[k] * nu * (1.2533141373155003f / static_cast<float>(D));  // sqrt(pi/2)/m, m = d
 #pragma unroll
         for (int r = 0; r < G; ++r) lg[k][r] = fmaf(f, corr[r], lg[k][r]);
@@ -388,102 +457,106 @@ __global__ void __launch_bounds__(512, 1) decode_kernel(DecodeArgs a) {
           if (r < a.Gq) {
             const int gi = r / a.Lq, lq = r - gi * a.Lq;
             const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-            a.logits[row * a.kv_len + key[k]] = lg[k][r];
+            a.logits[row * a.kv_len + s0 + lk[k]] = lg[k][r];
           }
         }
       }
     }
-    if (!with_v) continue;
 
-    // online softmax over this iteration's KW keys, base 2
-    bool grew = false;
-    float alpha[G];
-#pragma unroll
-    for (int r = 0; r < G; ++r) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) {
-        lg[k][r] = valid[k] ? lg[k][r] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, lg[k][r]);
-      }
-      const float mn = fmaxf(m_run[r], warp_max(mx));
-      grew |= mn > m_run[r];
-      alpha[r] = fast_exp2(m_run[r] - mn);  // m_run = -inf -> 0
-      float ps = 0.0f;
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) {
-        lg[k][r] = fast_exp2(lg[k][r] - mn);  // invalid keys: 2^-inf = 0
-        ps += lg[k][r];
-      }
-      l_run[r] = l_run[r] * alpha[r] + ps;
-      m_run[r] = mn;
-    }
-    if (grew) {  // warp-uniform: the maxima are warp-wide
-      float sa0 = 0.0f, sa1 = 0.0f;  // this lane's accumulator columns are rows 2*c4, 2*c4+1
+    if (with_v) {
+      // online softmax over this warp's keys of the stage, base 2
+      bool grew = false;
+      float alpha[G];
 #pragma unroll
       for (int r = 0; r < G; ++r) {
-        sa0 = (r == 2 * c4) ? alpha[r] : sa0;
-        sa1 = (r == 2 * c4 + 1) ? alpha[r] : sa1;
-      }
+        float mx = -INFINITY;
 #pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        acc_o[t][0] *= sa0; acc_o[t][1] *= sa1; acc_o[t][2] *= sa0; acc_o[t][3] *= sa1;
+        for (int k = 0; k < KPL; ++k) {
+          lg[k][r] = valid[k] ? lg[k][r] * a.scale_log2 : -INFINITY;
+          mx = fmaxf(mx, lg[k][r]);
+        }
+        const float mn = fmaxf(m_run[r], warp_max(mx));
+        grew |= mn > m_run[r];
+        alpha[r] = fast_exp2(m_run[r] - mn);  // m_run = -inf -> 0
+        float ps = 0.0f;
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) {
+          lg[k][r] = fast_exp2(lg[k][r] - mn);  // invalid keys: 2^-inf = 0
+          ps += lg[k][r];
+        }
+        l_run[r] = l_run[r] * alpha[r] + ps;
+        m_run[r] = mn;
       }
-    }
+      if (grew) {  // warp-uniform: the maxima are warp-wide
+        float sa0 = 0.0f, sa1 = 0.0f;  // this lane's accumulator columns are rows 2*c4, 2*c4+1
+#pragma unroll
+        for (int r = 0; r < G; ++r) {
+          sa0 = (r == 2 * c4) ? alpha[r] : sa0;
+          sa1 = (r == 2 * c4 + 1) ? alpha[r] : sa1;
+        }
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          acc_o[t][0] *= sa0; acc_o[t][1] *= sa1; acc_o[t][2] *= sa0; acc_o[t][3] *= sa1;
+        }
+      }
 
-    // P.V, one 32-key sub-chunk (lane = key) at a time
+      // P.V, one 32-key sub-chunk (lane = key) at a time
 #pragma unroll
-    for (int k = 0; k < KPL; ++k) {
-      const int64_t kb = base + 32 * k;
-      if (kb >= k_end) break;  // warp-uniform
+      for (int k = 0; k < KPL; ++k) {
+        const int64_t kb = s0 + warp * KW + 32 * k;
+        if (kb >= k_end) break;  // warp-uniform
 #pragma unroll
-      for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
-      __syncwarp();
+        for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
+        __syncwarp();
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        uint4 vreg[4][NCH];
+        for (int ks = 0; ks < 2; ++ks) {
+          uint4 vreg[4][NCH];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int64_t vk = kb + 16 * ks + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
+          for (int kk = 0; kk < 4; ++kk) {
+            const int64_t vk = kb + 16 * ks + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
 #pragma unroll
-          for (int hh = 0; hh < NCH; ++hh)
-            vreg[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
-                                      : make_uint4(0u, 0u, 0u, 0u);
-        }
-        uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
-        if (g8 < G) {
-          const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
-          const float2 p01 = *reinterpret_cast<const float2*>(prow);
-          const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
-          split_bf16x2(p01.x, p01.y, bh0, bl0);
-          split_bf16x2(p89.x, p89.y, bh1, bl1);
-        }
+            for (int hh = 0; hh < NCH; ++hh)
+              vreg[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
+                                        : make_uint4(0u, 0u, 0u, 0u);
+          }
+          uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
+          if (g8 < G) {
+            const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
+            const float2 p01 = *reinterpret_cast<const float2*>(prow);
+            const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
+            split_bf16x2(p01.x, p01.y, bh0, bl0);
+            split_bf16x2(p89.x, p89.y, bh1, bl1);
+          }
 #pragma unroll
-        for (int hh = 0; hh < NCH; ++hh) {
-          const uint4 k0 = vreg[0][hh], k1 = vreg[1][hh], k8 = vreg[2][hh], k9 = vreg[3][hh];
-          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-          const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
+          for (int hh = 0; hh < NCH; ++hh) {
+            const uint4 k0 = vreg[0][hh], k1 = vreg[1][hh], k8 = vreg[2][hh], k9 = vreg[3][hh];
+            const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+            const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
-            const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
-            const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
-            const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
-            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
+              const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
+              const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
+              const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
+              mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
+              mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
+            }
           }
         }
+        __syncwarp();
       }
-      __syncwarp();
     }
-  }
+    }  // warp has keys
 
-  if (!with_v) return;
+    __syncthreads();  // every warp is done with this stage's buffer
+    if (tid == 0 && st + NS < n_stages) issue_stage(st + NS);
+  }
+  __syncthreads();  // the ring is free: no copy is in flight after the last stage
+  if (s_abort || !with_v) return;
 
   // ------------------------------------------------ epilogue: merge warps
 #pragma unroll
   for (int r = 0; r < G; ++r) l_run[r] = warp_sum(l_run[r]);
-  __syncthreads();  // every warp is done with the table that `merge` aliases
   float* wm = merge;                                // [NWARP][G]
   float* wl = merge + NWARP * G;                    // [NWARP][G]
   float* wo = merge + 2 * NWARP * G;                // [NWARP][G][D]

@@ -115,13 +115,25 @@ def test_encode_and_decode_validate_before_launch():
                                 ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
     assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 16, 16, null, null, null,
                                 ctypes.c_float(0.1), null, null, null, 0, null) == _lib.OCTO_EINVAL
+    # the workspace is always required (status word), 256-byte aligned
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, 272, 1 << 20, null) == _lib.OCTO_EINVAL
+    # cache rows are staged with 16-byte copies: capacity % 4 and aligned cache pointers
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 6, 6, 16, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, 256, 1 << 20, null) == _lib.OCTO_EINVAL
+    assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 20, 16, null, null, 16,
+                                ctypes.c_float(0.1), 16, null, 256, 1 << 20, null) == _lib.OCTO_EINVAL
+    # too many query rows per KV head
     assert lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 16, 0, 1, 16, 1, 1, 8, 8, 16, 16, null, null, 16,
-                                ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EUNSUPPORTED
+                                ctypes.c_float(0.1), 16, null, 256, 1 << 20, null) == _lib.OCTO_EUNSUPPORTED
     # QJL layout without sketch buffers
     Lq = api.Layout(128, 4, qjl=True)
     assert lib.octo_decode_attn(Lq.ref, ctypes.byref(Tf), 16, 0, 1, 4, 1, 1, 8, 8, 16, 16, null, null, 16,
                                 ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
     assert lib.octo_decode_attn_workspace(L.ref, 1, 16, 1, 1, 8) == 0
+    assert lib.octo_decode_attn_workspace(L.ref, 1, 4, 1, 1, 0) >= 256
 
 
 def test_status_strings():

@@ -158,8 +158,8 @@ def test_decode_workspace_reuse_and_counters(cuda_ok):
     o2, _ = api.decode_attn(lay, dev, q, cache, V, 2, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
-    n_heads = 2
-    assert int(ws.buf[:n_heads].abs().sum()) == 0
+    assert int(ws.counters(2).abs().sum()) == 0
+    assert ws.status() == 0
 
 
 def test_decode_rejects_small_workspace(cuda_ok):
