@@ -88,10 +88,9 @@ struct DecCfg {
   static constexpr bool FOLD = C <= 7;                     // b = 2: table indexed by the full code
   static constexpr int NE = FOLD ? (1 << C) : (1 << (2 * BD));
   static constexpr int REP = NE <= 256 ? 8 : 4;           // replicas per entry (bank groups)
-  static constexpr int THREADS = 256, NWARP = THREADS / 32;
-  static constexpr int KPL = D <= 128 ? 2 : 1;             // keys per lane per stage
-  static constexpr int KW = 32 * KPL;                      // keys per warp per stage
-  static constexpr int CK = KW * NWARP;                    // keys per stage (512, 256 for d = 256)
+  static constexpr int KPL = D <= 128 ? 2 : 1;             // keys per lane per chunk
+  static constexpr int KW = 32 * KPL;                      // keys per chunk (one warp's unit of work)
+  static constexpr int NS = 2;                             // chunks in flight per warp
   static constexpr int QF = 3 * G;                         // rotated-query floats per triplet
   static constexpr int QV = (QF + 3) / 4;                  // ... as float4
   static constexpr int QW = D / 32;                        // sketch words per key
@@ -99,23 +98,25 @@ struct DecCfg {
   static constexpr int MT = D / 16;                        // m-tiles of O^T
   static constexpr int NCH = D / 64;                       // 16-byte V chunks per key per lane
   static constexpr int GV = (G + 3) / 4;                   // float4 per LUT entry
-  // one stage buffer: W code rows, a gamma row (+ QW sketch rows, a norm row)
-  static constexpr int STAGE_ROWS = W + 1 + (QJL ? QW + 1 : 0);
-  static constexpr size_t STAGE = sizeof(uint32_t) * STAGE_ROWS * CK;
-  // shared memory carve-up (bytes): the stage ring is reused for the warps'
-  // (m, l, O) once the main loop is over
+  // one chunk buffer: W code rows, a gamma row (+ QW sketch rows, a norm row)
+  static constexpr int ROWS = W + 1 + (QJL ? QW + 1 : 0);
+  static constexpr size_t CHUNK = sizeof(uint32_t) * ROWS * KW;
   static constexpr size_t TABLE = sizeof(float4) * NE * REP;
-  static constexpr size_t MERGE = sizeof(float) * NWARP * G * (D + 2);
   static constexpr size_t QT = sizeof(float4) * T * QV;
-  static constexpr size_t PBUF = sizeof(float) * NWARP * G * PSTRIDE;
   static constexpr size_t LUT = QJL ? sizeof(float4) * (D / 4) * 16 * GV : 0;
   static constexpr size_t QROW = D + 4;                    // floats per scratch query row
   static constexpr size_t SCRATCH = sizeof(float) * G * (QROW + (QJL ? D : 0));
-  static constexpr size_t FIXED = TABLE + QT + PBUF + LUT + SCRATCH;
-  static constexpr size_t BUDGET = 227 * 1024 - 1024;
-  static constexpr size_t ring(int ns) { return ns * STAGE > MERGE ? ns * STAGE : MERGE; }
-  static constexpr int NS = FIXED + ring(3) <= BUDGET ? 3 : 2;  // stages in flight
-  static constexpr size_t SMEM = FIXED + ring(NS);
+  static constexpr size_t BUDGET = 227 * 1024 - 2048;
+  // per-warp bytes: its P buffer and its chunk ring (the ring is reused for
+  // the warp's (m, l, O) in the epilogue)
+  static constexpr size_t PER_WARP_P = sizeof(float) * G * PSTRIDE;
+  static constexpr size_t RING_RAW = NS * CHUNK > sizeof(float) * G * (D + 2) ? NS * CHUNK : sizeof(float) * G * (D + 2);
+  static constexpr size_t RING = (RING_RAW + 127) / 128 * 128;  // keeps every ring 128-byte aligned
+  static constexpr size_t FIXED = TABLE + QT + LUT + SCRATCH;
+  static constexpr int NWARP = FIXED + 16 * (PER_WARP_P + RING) <= BUDGET ? 16 : 8;
+  static constexpr int THREADS = 32 * NWARP;
+  static constexpr size_t PBUF = PER_WARP_P * NWARP;
+  static constexpr size_t SMEM = FIXED + PBUF + RING * NWARP;
   static_assert(SMEM <= BUDGET, "shared memory budget");
 };
 
@@ -192,24 +193,22 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
 }
 
 template <int D, int B, int G, bool QJL>
-__global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kernel(DecodeArgs a) {
   using Cfg = DecCfg<D, B, G, QJL>;
   constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, BD = Cfg::BD, NDIR = Cfg::NDIR;
   constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, QW = Cfg::QW;
   constexpr int PS = Cfg::PSTRIDE, MT = Cfg::MT, NCH = Cfg::NCH, GV = Cfg::GV;
-  constexpr int KPL = Cfg::KPL, KW = Cfg::KW, CK = Cfg::CK, QV = Cfg::QV, NS = Cfg::NS;
-  constexpr int ROWS = Cfg::STAGE_ROWS;
+  constexpr int KPL = Cfg::KPL, KW = Cfg::KW, QV = Cfg::QV, NS = Cfg::NS, ROWS = Cfg::ROWS;
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
   float4* table = reinterpret_cast<float4*>(smem_raw);                                   // [NE*REP]
   float4* qt = reinterpret_cast<float4*>(smem_raw + Cfg::TABLE);                         // [T][QV]
-  float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + Cfg::QT);               // [NWARP][G][PS]
-  float4* lut = reinterpret_cast<float4*>(smem_raw + Cfg::TABLE + Cfg::QT + Cfg::PBUF);    // [D/4][16][GV]
-  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + Cfg::QT + Cfg::PBUF + Cfg::LUT);
-  uint32_t* stages = reinterpret_cast<uint32_t*>(smem_raw + Cfg::FIXED);                 // [NS][ROWS][CK]
-  float* merge = reinterpret_cast<float*>(smem_raw + Cfg::FIXED);                        // aliases the ring
+  float4* lut = reinterpret_cast<float4*>(smem_raw + Cfg::TABLE + Cfg::QT);              // [D/4][16][GV]
+  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + Cfg::QT + Cfg::LUT);
+  float* pbuf = reinterpret_cast<float*>(smem_raw + Cfg::FIXED);                         // [NWARP][G][PS]
+  unsigned char* rings = smem_raw + Cfg::FIXED + Cfg::PBUF;                              // [NWARP] RING bytes
   constexpr int QROW = static_cast<int>(Cfg::QROW);
-  __shared__ __align__(8) uint64_t full[NS];
+  __shared__ __align__(8) uint64_t full[NWARP][NS];
   __shared__ float s_rho_c[8];
   __shared__ float s_dir_c[32];
   __shared__ int s_last;
@@ -224,45 +223,53 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
 
   const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
   const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
-  const int n_stages = static_cast<int>((k_end - k_begin + CK - 1) / CK);
+  // chunks of KW keys, dealt to warps round-robin: warp w takes chunks w, w + NWARP, ...
+  const int n_chunks = static_cast<int>((k_end - k_begin + KW - 1) / KW);
+  const int my_chunks = warp < n_chunks ? (n_chunks - warp + NWARP - 1) / NWARP : 0;
   const uint32_t* pk = a.packed + static_cast<int64_t>(bh) * W * a.cache_cap;
   const float* gm = a.gamma + static_cast<int64_t>(bh) * a.cache_cap;
   const __nv_bfloat16* Vh = with_v ? a.V + static_cast<int64_t>(bh) * a.cache_cap * D : nullptr;
   const uint32_t* qbp = QJL ? a.qjl_bits + static_cast<int64_t>(bh) * QW * a.cache_cap : nullptr;
   const float* qnp = QJL ? a.qjl_norm + static_cast<int64_t>(bh) * a.cache_cap : nullptr;
+  uint32_t* ring = reinterpret_cast<uint32_t*>(rings + warp * Cfg::RING);                // [NS][ROWS][KW]
 
-  // Producer (thread 0): copy stage st's rows into buffer st % NS. Keys are
-  // copied in groups of 4 (16 bytes); the cache capacity is a multiple of 4
-  // and stages start at multiples of 64, so the rounded-up copy stays
-  // inside the cache rows (keys past kv_len are masked by the consumers).
-  auto issue_stage = [&](int st) {
-    const int64_t s0 = k_begin + static_cast<int64_t>(st) * CK;
-    const int n = static_cast<int>(k_end - s0 < CK ? k_end - s0 : CK);
+  // This warp's i-th chunk: lane 0 arms the barrier, lanes < ROWS each copy
+  // one row (code words, gammas, sketch words, norms) into ring slot i % NS,
+  // lane ROWS prefetches the chunk's V rows into L2. Keys are copied in
+  // groups of 4 (16 bytes); the capacity is a multiple of 4 and chunks start
+  // at multiples of KW, so the rounded-up copy stays inside the cache rows.
+  auto issue_chunk = [&](int i) {
+    const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * i) * KW;
+    const int n = static_cast<int>(k_end - s0 < KW ? k_end - s0 : KW);
     const uint32_t bytes = static_cast<uint32_t>(((n + 3) & ~3) * 4);
-    uint32_t* buf = stages + (st % NS) * ROWS * CK;
-    uint64_t* bar = &full[st % NS];
-    mbar_expect_tx(bar, bytes * ROWS);
-#pragma unroll 1
-    for (int w = 0; w < W; ++w) bulk_g2s(buf + w * CK, pk + w * a.cache_cap + s0, bytes, bar);
-    bulk_g2s(buf + W * CK, gm + s0, bytes, bar);
-    if constexpr (QJL) {
-#pragma unroll 1
-      for (int w = 0; w < QW; ++w) bulk_g2s(buf + (W + 1 + w) * CK, qbp + w * a.cache_cap + s0, bytes, bar);
-      bulk_g2s(buf + (W + 1 + QW) * CK, qnp + s0, bytes, bar);
+    uint32_t* buf = ring + (i % NS) * ROWS * KW;
+    uint64_t* bar = &full[warp][i % NS];
+    if (lane == 0) mbar_expect_tx(bar, bytes * ROWS);
+    __syncwarp();
+    for (int r = lane; r <= ROWS; r += 32) {
+      if (r < W) {
+        bulk_g2s(buf + r * KW, pk + r * a.cache_cap + s0, bytes, bar);
+      } else if (r == W) {
+        bulk_g2s(buf + W * KW, gm + s0, bytes, bar);
+      } else if (QJL && r < W + 1 + QW) {
+        const int w = r - W - 1;
+        bulk_g2s(buf + (W + 1 + w) * KW, qbp + w * a.cache_cap + s0, bytes, bar);
+      } else if (QJL && r == W + 1 + QW) {
+        bulk_g2s(buf + (W + 1 + QW) * KW, qnp + s0, bytes, bar);
+      } else if (r == ROWS && with_v) {
+        bulk_prefetch_l2(Vh + s0 * D, static_cast<uint32_t>(n) * D * 2);
+      }
     }
-    if (with_v) bulk_prefetch_l2(Vh + s0 * D, static_cast<uint32_t>(n) * D * 2);
   };
 
   if (tid == 0) {
     s_abort = 0;
-#pragma unroll
-    for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1);
+    for (int w = 0; w < NWARP; ++w)
+      for (int s = 0; s < NS; ++s) mbar_init(&full[w][s], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int st = 0; st < NS && st < n_stages; ++st) issue_stage(st);
-  }
+  for (int i = 0; i < NS && i < my_chunks; ++i) issue_chunk(i);
 
   // ------------------------------------------------ prologue (overlaps the first copies)
   if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
@@ -347,7 +354,7 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
   }
   __syncthreads();
 
-  // ------------------------------------------------ main loop over stages
+  // ------------------------------------------------ main loop: this warp's chunks
   const int g8 = lane >> 2, c4 = lane & 3;
   const int rep_off = lane & (REP - 1);
 
@@ -358,30 +365,24 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
 #pragma unroll
   for (int t = 0; t < MT; ++t) acc_o[t][0] = acc_o[t][1] = acc_o[t][2] = acc_o[t][3] = 0.0f;
   float* pw = pbuf + warp * G * PS;
+  int aborted_at = -1;
 
-  for (int st = 0; st < n_stages; ++st) {
-    const uint32_t* buf = stages + (st % NS) * ROWS * CK;
-    const int64_t s0 = k_begin + static_cast<int64_t>(st) * CK;
-    // every thread acquires the stage's data; an expired wait aborts the whole CTA
-    if (!mbar_wait_bounded(&full[st % NS], (st / NS) & 1)) s_abort = 1;  // benign race: all write 1
-    __syncthreads();
-    if (s_abort) {
-      if (tid == 0) {
-        atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
-        // let the copies already issued land before the shared memory is released
-        for (int s2 = st + 1; s2 < n_stages && s2 < st + NS; ++s2) mbar_wait_bounded(&full[s2 % NS], (s2 / NS) & 1);
-      }
+  for (int ci = 0; ci < my_chunks; ++ci) {
+    const uint32_t* buf = ring + (ci % NS) * ROWS * KW;
+    const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * ci) * KW;
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[warp][ci % NS], (ci / NS) & 1))) {
+      aborted_at = ci;  // warp-uniform
       break;
     }
-    if (s0 + warp * KW < k_end) {  // this warp has keys in the stage (all but the tail stage)
+
     int lk[KPL];
     bool valid[KPL];
     float gk[KPL];
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
-      lk[k] = warp * KW + 32 * k + lane;
+      lk[k] = 32 * k + lane;
       valid[k] = s0 + lk[k] < k_end;
-      gk[k] = valid[k] ? __uint_as_float(buf[W * CK + lk[k]]) : 0.0f;
+      gk[k] = valid[k] ? __uint_as_float(buf[W * KW + lk[k]]) : 0.0f;
     }
 
     float lg[KPL][G];
@@ -403,8 +404,8 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
 #pragma unroll
       for (int k = 0; k < KPL; ++k) {
         uint32_t code;
-        if (sh + C <= 32) code = (buf[wi * CK + lk[k]] >> sh) & mask;
-        else code = __funnelshift_r(buf[wi * CK + lk[k]], buf[(wi + 1) * CK + lk[k]], sh) & mask;
+        if (sh + C <= 32) code = (buf[wi * KW + lk[k]] >> sh) & mask;
+        else code = __funnelshift_r(buf[wi * KW + lk[k]], buf[(wi + 1) * KW + lk[k]], sh) & mask;
         float4 u;
         if constexpr (Cfg::FOLD) {
           u = table[code * REP + rep_off];
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
         for (int r = 0; r < 4 * GV; ++r) corr[r] = 0.0f;
 #pragma unroll
         for (int w = 0; w < QW; ++w) {
-          const uint32_t word = buf[(W + 1 + w) * CK + lk[k]];
+          const uint32_t word = buf[(W + 1 + w) * KW + lk[k]];
 #pragma unroll
           for (int j8 = 0; j8 < 8; ++j8) {
             const uint32_t nib = (word >> (4 * j8)) & 15u;
@@ -441,12 +442,15 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
             }
           }
         }
-        const float nu = valid[k] ? __uint_as_float(buf[(W + 1 + QW) * CK + lk[k]]) : 0.0f;
+        const float nu = valid[k] ? __uint_as_float(buf[(W + 1 + QW) * KW + lk[k]]) : 0.0f;
         const float f = gk[k] * nu * (1.2533141373155003f / static_cast<float>(D));  // sqrt(pi/2)/m, m = d
 #pragma unroll
         for (int r = 0; r < G; ++r) lg[k][r] = fmaf(f, corr[r], lg[k][r]);
       }
     }
+    // this warp is done with the chunk's rows: refill the slot with chunk ci + NS
+    __syncwarp();
+    if (ci + NS < my_chunks) issue_chunk(ci + NS);
 
     if (a.logits != nullptr) {
 #pragma unroll
@@ -462,115 +466,122 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
         }
       }
     }
+    if (!with_v) continue;
 
-    if (with_v) {
-      // online softmax over this warp's keys of the stage, base 2
-      bool grew = false;
-      float alpha[G];
+    // online softmax over the chunk, base 2
+    bool grew = false;
+    float alpha[G];
 #pragma unroll
-      for (int r = 0; r < G; ++r) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < KPL; ++k) {
-          lg[k][r] = valid[k] ? lg[k][r] * a.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, lg[k][r]);
-        }
-        const float mn = fmaxf(m_run[r], warp_max(mx));
-        grew |= mn > m_run[r];
-        alpha[r] = fast_exp2(m_run[r] - mn);  // m_run = -inf -> 0
-        float ps = 0.0f;
-#pragma unroll
-        for (int k = 0; k < KPL; ++k) {
-          lg[k][r] = fast_exp2(lg[k][r] - mn);  // invalid keys: 2^-inf = 0
-          ps += lg[k][r];
-        }
-        l_run[r] = l_run[r] * alpha[r] + ps;
-        m_run[r] = mn;
-      }
-      if (grew) {  // warp-uniform: the maxima are warp-wide
-        float sa0 = 0.0f, sa1 = 0.0f;  // this lane's accumulator columns are rows 2*c4, 2*c4+1
-#pragma unroll
-        for (int r = 0; r < G; ++r) {
-          sa0 = (r == 2 * c4) ? alpha[r] : sa0;
-          sa1 = (r == 2 * c4 + 1) ? alpha[r] : sa1;
-        }
-#pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          acc_o[t][0] *= sa0; acc_o[t][1] *= sa1; acc_o[t][2] *= sa0; acc_o[t][3] *= sa1;
-        }
-      }
-
-      // P.V, one 32-key sub-chunk (lane = key) at a time
+    for (int r = 0; r < G; ++r) {
+      float mx = -INFINITY;
 #pragma unroll
       for (int k = 0; k < KPL; ++k) {
-        const int64_t kb = s0 + warp * KW + 32 * k;
-        if (kb >= k_end) break;  // warp-uniform
+        lg[k][r] = valid[k] ? lg[k][r] * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, lg[k][r]);
+      }
+      const float mn = fmaxf(m_run[r], warp_max(mx));
+      grew |= mn > m_run[r];
+      alpha[r] = fast_exp2(m_run[r] - mn);  // m_run = -inf -> 0
+      float ps = 0.0f;
 #pragma unroll
-        for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
-        __syncwarp();
+      for (int k = 0; k < KPL; ++k) {
+        lg[k][r] = fast_exp2(lg[k][r] - mn);  // invalid keys: 2^-inf = 0
+        ps += lg[k][r];
+      }
+      l_run[r] = l_run[r] * alpha[r] + ps;
+      m_run[r] = mn;
+    }
+    if (grew) {  // warp-uniform: the maxima are warp-wide
+      float sa0 = 0.0f, sa1 = 0.0f;  // this lane's accumulator columns are rows 2*c4, 2*c4+1
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          uint4 vreg[4][NCH];
+      for (int r = 0; r < G; ++r) {
+        sa0 = (r == 2 * c4) ? alpha[r] : sa0;
+        sa1 = (r == 2 * c4 + 1) ? alpha[r] : sa1;
+      }
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int64_t vk = kb + 16 * ks + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
-#pragma unroll
-            for (int hh = 0; hh < NCH; ++hh)
-              vreg[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
-                                        : make_uint4(0u, 0u, 0u, 0u);
-          }
-          uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
-          if (g8 < G) {
-            const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
-            const float2 p01 = *reinterpret_cast<const float2*>(prow);
-            const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
-            split_bf16x2(p01.x, p01.y, bh0, bl0);
-            split_bf16x2(p89.x, p89.y, bh1, bl1);
-          }
-#pragma unroll
-          for (int hh = 0; hh < NCH; ++hh) {
-            const uint4 k0 = vreg[0][hh], k1 = vreg[1][hh], k8 = vreg[2][hh], k9 = vreg[3][hh];
-            const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-            const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-              const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
-              const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
-              const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
-              const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-              mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
-              mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
-            }
-          }
-        }
-        __syncwarp();
+      for (int t = 0; t < MT; ++t) {
+        acc_o[t][0] *= sa0; acc_o[t][1] *= sa1; acc_o[t][2] *= sa0; acc_o[t][3] *= sa1;
       }
     }
-    }  // warp has keys
 
-    __syncthreads();  // every warp is done with this stage's buffer
-    if (tid == 0 && st + NS < n_stages) issue_stage(st + NS);
+    // P.V, one 32-key sub-chunk (lane = key) at a time
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      const int64_t kb = s0 + 32 * k;
+      if (kb >= k_end) break;  // warp-uniform
+#pragma unroll
+      for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
+      __syncwarp();
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        uint4 vreg[4][NCH];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int64_t vk = kb + 16 * ks + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
+#pragma unroll
+          for (int hh = 0; hh < NCH; ++hh)
+            vreg[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
+                                      : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
+        if (g8 < G) {
+          const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
+          const float2 p01 = *reinterpret_cast<const float2*>(prow);
+          const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
+          split_bf16x2(p01.x, p01.y, bh0, bl0);
+          split_bf16x2(p89.x, p89.y, bh1, bl1);
+        }
+#pragma unroll
+        for (int hh = 0; hh < NCH; ++hh) {
+          const uint4 k0 = vreg[0][hh], k1 = vreg[1][hh], k8 = vreg[2][hh], k9 = vreg[3][hh];
+          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+          const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
+            const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
+            const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
+            const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
+            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
+            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
+          }
+        }
+      }
+      __syncwarp();
+    }
   }
-  __syncthreads();  // the ring is free: no copy is in flight after the last stage
+
+  if (aborted_at >= 0 && lane == 0) {
+    atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
+    s_abort = 1;
+    // chunks issued but not consumed (the one that timed out and up to NS-1
+    // after it) must land before the shared memory is reused or released
+    for (int c = aborted_at; c < aborted_at + NS && c < my_chunks; ++c)
+      mbar_wait_bounded(&full[warp][c % NS], (c / NS) & 1);
+  }
+  __syncthreads();
   if (s_abort || !with_v) return;
 
-  // ------------------------------------------------ epilogue: merge warps
+  // ------------------------------------------------ epilogue: merge warps (in each warp's ring)
 #pragma unroll
   for (int r = 0; r < G; ++r) l_run[r] = warp_sum(l_run[r]);
-  float* wm = merge;                                // [NWARP][G]
-  float* wl = merge + NWARP * G;                    // [NWARP][G]
-  float* wo = merge + 2 * NWARP * G;                // [NWARP][G][D]
+  auto wm = [&](int w) { return reinterpret_cast<float*>(rings + w * Cfg::RING); };          // [G] m
+  auto wl = [&](int w) { return reinterpret_cast<float*>(rings + w * Cfg::RING) + G; };      // [G] l
+  auto wo = [&](int w) { return reinterpret_cast<float*>(rings + w * Cfg::RING) + 2 * G; };  // [G][D] O
   if (lane == 0) {
 #pragma unroll
-    for (int r = 0; r < G; ++r) { wm[warp * G + r] = m_run[r]; wl[warp * G + r] = l_run[r]; }
+    for (int r = 0; r < G; ++r) { wm(warp)[r] = m_run[r]; wl(warp)[r] = l_run[r]; }
   }
+  {
+    float* o = wo(warp);
 #pragma unroll
-  for (int t = 0; t < MT; ++t) {
-    const int hh = t >> 2, e2 = t & 3;
-    const int d0 = 64 * hh + 8 * g8 + 2 * e2;
-    const int q0 = 2 * c4, q1 = 2 * c4 + 1;
-    if (q0 < G) { wo[(warp * G + q0) * D + d0] = acc_o[t][0]; wo[(warp * G + q0) * D + d0 + 1] = acc_o[t][2]; }
-    if (q1 < G) { wo[(warp * G + q1) * D + d0] = acc_o[t][1]; wo[(warp * G + q1) * D + d0 + 1] = acc_o[t][3]; }
+    for (int t = 0; t < MT; ++t) {
+      const int hh = t >> 2, e2 = t & 3;
+      const int d0 = 64 * hh + 8 * g8 + 2 * e2;
+      const int q0 = 2 * c4, q1 = 2 * c4 + 1;
+      if (q0 < G) { o[q0 * D + d0] = acc_o[t][0]; o[q0 * D + d0 + 1] = acc_o[t][2]; }
+      if (q1 < G) { o[q1 * D + d0] = acc_o[t][1]; o[q1 * D + d0 + 1] = acc_o[t][3]; }
+    }
   }
   __syncthreads();
 
@@ -582,14 +593,14 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(DecodeArgs a) {
     const int r = j / D, d = j - r * D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NWARP; ++w) M = fmaxf(M, wm[w * G + r]);
+    for (int w = 0; w < NWARP; ++w) M = fmaxf(M, wm(w)[r]);
     float o = 0.0f, l = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < NWARP; ++w) {
-        const float f = fast_exp2(wm[w * G + r] - M);
-        o = fmaf(f, wo[(w * G + r) * D + d], o);
-        l = fmaf(f, wl[w * G + r], l);
+        const float f = fast_exp2(wm(w)[r] - M);
+        o = fmaf(f, wo(w)[r * D + d], o);
+        l = fmaf(f, wl(w)[r], l);
       }
     }
     if (S == 1) {

@@ -59,6 +59,7 @@ struct EncCfg {
   static constexpr int KT = 8192 / D;              // keys per tile
   static constexpr int US = ((3 * T) % 2 == 0) ? 3 * T + 1 : 3 * T;  // odd row stride (floats)
   static constexpr int THREADS = 256;
+  static constexpr int REP = NDIR * NDIR <= 256 ? 8 : 4;  // n_hat replicas (distinct bank groups per quarter-warp)
 };
 
 template <int D, int B, bool QJL>
@@ -67,9 +68,10 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   constexpr int T = Cfg::T, KT = Cfg::KT, US = Cfg::US, E = Cfg::E, W = Cfg::W, C = Cfg::C;
   constexpr int NDIR = Cfg::NDIR, NRHO = Cfg::NRHO;
 
+  constexpr int REP = Cfg::REP;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float4* nhat = reinterpret_cast<float4*>(smem_raw);                 // [NDIR*NDIR]
-  float* U = reinterpret_cast<float*>(nhat + NDIR * NDIR);            // [KT][US]
+  float4* nhat = reinterpret_cast<float4*>(smem_raw);                 // [NDIR*NDIR][REP]
+  float* U = reinterpret_cast<float*>(nhat + NDIR * NDIR * REP);      // [KT][US]
   uint16_t* codes = reinterpret_cast<uint16_t*>(U + KT * US);         // [KT][T]
   __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[8], s_rho_t[8];
 
@@ -83,9 +85,39 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   __syncthreads();
   for (int e = tid; e < NDIR * NDIR; e += Cfg::THREADS) {
     const float3 n = oct_inverse(s_dir_c[e / NDIR], s_dir_c[e % NDIR]);
-    nhat[e] = make_float4(n.x, n.y, n.z, 0.0f);
+    const float4 v = make_float4(n.x, n.y, n.z, 0.0f);
+#pragma unroll
+    for (int k = 0; k < REP; ++k) nhat[e * REP + ((k + lane) & (REP - 1))] = v;
   }
-  // (the first __syncthreads of the tile loop orders these writes)
+  __syncthreads();
+  // the norm codebook lives in registers: thresholds and centroids
+  float rt[NRHO > 1 ? NRHO - 1 : 1], rc[NRHO];
+#pragma unroll
+  for (int k = 0; k < NRHO - 1; ++k) rt[k] = s_rho_t[k];
+#pragma unroll
+  for (int k = 0; k < NRHO; ++k) rc[k] = s_rho_c[k];
+  const int rep_off = lane & (REP - 1);
+  // Cell of x in the direction codebook: start from the uniform-grid cell
+  // and step to the exact one (cell i has t[i-1] <= x < t[i]; the Lloyd-Max
+  // thresholds are close to uniform, so this takes 0-1 steps).
+  auto dir_index = [&](float x) -> int {
+    int i = __float2int_rd((x + 1.0f) * (0.5f * NDIR));
+    i = i < 0 ? 0 : (i > NDIR - 1 ? NDIR - 1 : i);
+    while (i > 0 && x < s_dir_t[i - 1]) --i;
+    while (i < NDIR - 1 && x >= s_dir_t[i]) ++i;
+    return i;
+  };
+  // Norm level nearest to v (count of thresholds <= v) and its centroid.
+  auto rho_level = [&](float v, int& ir, float& rh) {
+    ir = 0;
+    rh = rc[0];
+#pragma unroll
+    for (int k = 0; k < NRHO - 1; ++k) {
+      const bool up = v >= rt[k];
+      ir += up;
+      rh = up ? rc[k + 1] : rh;
+    }
+  };
 
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
 
@@ -134,8 +166,9 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
       ss = warp_sum(ss);
       const float g = sqrtf(ss);
+      const float ig = g > 0.0f ? 1.0f / g : 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = (g > 0.0f ? v[e] / g : 0.0f) * sgn[e];
+      for (int e = 0; e < E; ++e) v[e] = v[e] * ig * sgn[e];
       fwht_warp<E>(v, lane);
       float* row = U + k * US;
 #pragma unroll
@@ -153,25 +186,26 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       const float rho = sqrtf(x * x + y * y + z * z);
       const float l1 = fabsf(x) + fabsf(y) + fabsf(z);
       float px = 0.0f, py = 0.0f, pz = 1.0f;
-      if (l1 > 0.0f) { px = x / l1; py = y / l1; pz = z / l1; }
+      if (l1 > 0.0f) {
+        const float il = 1.0f / l1;
+        px = x * il; py = y * il; pz = z * il;
+      }
       float xi = px, eta = py;
       if (!(pz >= 0.0f)) {
         xi = (1.0f - fabsf(py)) * (px >= 0.0f ? 1.0f : -1.0f);
         eta = (1.0f - fabsf(px)) * (py >= 0.0f ? 1.0f : -1.0f);
       }
-      int ix = count_le(s_dir_t, NDIR - 1, xi);
-      int iy = count_le(s_dir_t, NDIR - 1, eta);
+      int ix = dir_index(xi);
+      int iy = dir_index(eta);
       int ir;
-      float4 nb;
+      float rh;
+      float4 nb = nhat[(ix * NDIR + iy) * REP + rep_off];
       if (!a.joint) {
-        ir = count_le(s_rho_t, NRHO - 1, rho);
-        nb = nhat[ix * NDIR + iy];
+        rho_level(rho, ir, rh);
       } else {
         // centre first, then (dx, dy) row-major; replace only on strictly smaller error
-        nb = nhat[ix * NDIR + iy];
-        float s = nb.x * x + nb.y * y + nb.z * z;
-        ir = count_le(s_rho_t, NRHO - 1, s);
-        float rh = s_rho_c[ir];
+        const float s = nb.x * x + nb.y * y + nb.z * z;
+        rho_level(s, ir, rh);
         float best = rh * (rh - 2.0f * s);
         const int cx = ix, cy = iy;
 #pragma unroll
@@ -181,19 +215,19 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
             if (dx == 0 && dy == 0) continue;
             const int ux = cx + dx, uy = cy + dy;
             if (ux < 0 || ux >= NDIR || uy < 0 || uy >= NDIR) continue;
-            const float4 n = nhat[ux * NDIR + uy];
+            const float4 n = nhat[(ux * NDIR + uy) * REP + rep_off];
             const float sc = n.x * x + n.y * y + n.z * z;
-            const int rc = count_le(s_rho_t, NRHO - 1, sc);
-            const float rr = s_rho_c[rc];
+            int rci;
+            float rr;
+            rho_level(sc, rci, rr);
             const float err = rr * (rr - 2.0f * sc);
-            if (err < best) { best = err; ix = ux; iy = uy; ir = rc; nb = n; }
+            if (err < best) { best = err; ix = ux; iy = uy; ir = rci; rh = rr; nb = n; }
           }
         }
       }
       codes[k * T + i] = static_cast<uint16_t>(ix | (iy << Cfg::BD) | (ir << (2 * Cfg::BD)));
       if constexpr (QJL) {
         // residual e = t - rho_hat n_hat, in place (the pad coordinate is dropped later)
-        const float rh = s_rho_c[ir];
         tp[0] = x - rh * nb.x;
         tp[1] = y - rh * nb.y;
         tp[2] = z - rh * nb.z;
@@ -257,7 +291,7 @@ static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
   EncodeArgs a = a0;
   a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
   a.n_tiles = a.tiles_per_head * a.n_heads;
-  const size_t smem = sizeof(float4) * Cfg::NDIR * Cfg::NDIR + sizeof(float) * Cfg::KT * Cfg::US +
+  const size_t smem = sizeof(float4) * Cfg::NDIR * Cfg::NDIR * Cfg::REP + sizeof(float) * Cfg::KT * Cfg::US +
                       sizeof(uint16_t) * Cfg::KT * Cfg::T;
   auto kern = encode_kernel<D, B, QJL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
