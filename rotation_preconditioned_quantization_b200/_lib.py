@@ -10,7 +10,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liboctopus_b200.so")
+# OCTO_LIBRARY selects another build of the same library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("OCTO_LIBRARY") or os.path.join(_HERE, "liboctopus_b200.so")
 
 OCTO_OK, OCTO_EINVAL, OCTO_EUNSUPPORTED, OCTO_ECUDA, OCTO_EWORKSPACE = 0, -1, -2, -3, -4
 ROUND_SCALAR, ROUND_JOINT = 0, 1

@@ -72,8 +72,28 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile and link the library; returns its path."""
+def build(force: bool = False, verbose_ptxas: bool = False, defines=(), out: str | None = None,
+          build_dir: str | None = None) -> str:
+    """Compile and link the library; returns its path.
+
+    ``defines`` (e.g. ``["OCTO_DECODE_MAX_WARPS=8"]``) set the kernels'
+    build-time tuning knobs; with them, pass a separate ``build_dir`` and
+    ``out`` so the default build is left untouched.
+    """
+    global BUILD, LIB, NVCC_FLAGS
+    saved = (BUILD, LIB, NVCC_FLAGS)
+    if build_dir:
+        BUILD = build_dir
+    if out:
+        LIB = out
+    NVCC_FLAGS = NVCC_FLAGS + [f"-D{d}" for d in defines]
+    try:
+        return _build(force, verbose_ptxas)
+    finally:
+        BUILD, LIB, NVCC_FLAGS = saved
+
+
+def _build(force: bool, verbose_ptxas: bool) -> str:
     os.makedirs(BUILD, exist_ok=True)
     headers = _headers()
     srcs = _sources()

@@ -78,6 +78,14 @@ struct DecodeArgs {
   float* part_o;
 };
 
+// Build-time tuning knobs (the defaults are the measured best on B200).
+#ifndef OCTO_DECODE_MAX_WARPS
+#define OCTO_DECODE_MAX_WARPS 8   // warps per CTA (16 only if shared memory allows)
+#endif
+#ifndef OCTO_DECODE_FOLD_BITS
+#define OCTO_DECODE_FOLD_BITS 10  // full-code table when a triplet code has at most this many bits
+#endif
+
 template <int D, int B, int G, bool QJL>
 struct DecCfg {
   static constexpr int T = (D + 2) / 3;
@@ -85,12 +93,12 @@ struct DecCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr bool FOLD = C <= 7;                     // b = 2: table indexed by the full code
+  static constexpr bool FOLD = C <= OCTO_DECODE_FOLD_BITS;  // table indexed by the full code (b <= 3)
   static constexpr int NE = FOLD ? (1 << C) : (1 << (2 * BD));
   static constexpr int REP = NE <= 256 ? 8 : 4;           // replicas per entry (bank groups)
   static constexpr int KPL = D <= 128 ? 2 : 1;             // keys per lane per chunk
   static constexpr int KW = 32 * KPL;                      // keys per chunk (one warp's unit of work)
-  static constexpr int NS = 2;                             // chunks in flight per warp
+  static constexpr int NS_MAX = 2;                         // chunks in flight per warp (at most)
   static constexpr int QF = 3 * G;                         // rotated-query floats per triplet
   static constexpr int QV = (QF + 3) / 4;                  // ... as float4
   static constexpr int QW = D / 32;                        // sketch words per key
@@ -110,10 +118,20 @@ struct DecCfg {
   // per-warp bytes: its P buffer and its chunk ring (the ring is reused for
   // the warp's (m, l, O) in the epilogue)
   static constexpr size_t PER_WARP_P = sizeof(float) * G * PSTRIDE;
-  static constexpr size_t RING_RAW = NS * CHUNK > sizeof(float) * G * (D + 2) ? NS * CHUNK : sizeof(float) * G * (D + 2);
-  static constexpr size_t RING = (RING_RAW + 127) / 128 * 128;  // keeps every ring 128-byte aligned
+  // a warp's ring also holds its (m, l, O) in the epilogue, and the rings
+  // together the split-merge weights (G x up to 1024 splits, 8+ warps)
+  static constexpr size_t cmax(size_t x, size_t y) { return x > y ? x : y; }
+  static constexpr size_t ring_bytes(int ns) {
+    return (cmax(cmax(ns * CHUNK, sizeof(float) * G * (D + 2)), sizeof(float) * G * 1024 / 8) + 127) / 128 * 128;
+  }
   static constexpr size_t FIXED = TABLE + QT + LUT + SCRATCH;
-  static constexpr int NWARP = FIXED + 16 * (PER_WARP_P + RING) <= BUDGET ? 16 : 8;
+  static constexpr bool fits(int nw, int ns) { return FIXED + nw * (PER_WARP_P + ring_bytes(ns)) <= BUDGET; }
+  // prefer 16 warps (latency hiding), then double buffering
+  static constexpr int NWARP = (OCTO_DECODE_MAX_WARPS >= 16 && fits(16, 1)) ? 16 : 8;
+  static_assert(fits(8, 1), "shared memory budget");
+  static constexpr int NS = fits(NWARP, NS_MAX) ? NS_MAX : 1;
+  static constexpr size_t RING = ring_bytes(NS);  // keeps every ring 128-byte aligned
+  static_assert(RING * 8 >= sizeof(float) * G * 1024, "split-merge weights fit in the rings");
   static constexpr int THREADS = 32 * NWARP;
   static constexpr size_t PBUF = PER_WARP_P * NWARP;
   static constexpr size_t SMEM = FIXED + PBUF + RING * NWARP;
@@ -262,6 +280,30 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
     }
   };
 
+  // The few small global reads of the prologue go first, ahead of the bulk
+  // traffic that the chunk copies start: codebooks, and one query row per
+  // warp (sign-flipped, in registers).
+  constexpr int E = D / 32;
+  float qraw[E];
+  if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
+  if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
+  {
+    const int r = warp;
+    if (r < G && r < a.Gq) {
+      const int gi = r / a.Lq, lq = r - gi * a.Lq;
+      const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
+      const float* sg = a.signs + trow * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float x = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qoff + e])
+                                 : static_cast<const float*>(a.q)[qoff + e];
+        qraw[e] = x * __ldg(sg + e);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) qraw[e] = 0.0f;
+    }
+  }
   if (tid == 0) {
     s_abort = 0;
     for (int w = 0; w < NWARP; ++w)
@@ -272,9 +314,6 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   for (int i = 0; i < NS && i < my_chunks; ++i) issue_chunk(i);
 
   // ------------------------------------------------ prologue (overlaps the first copies)
-  if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
-  if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
-  __syncthreads();
   for (int e = tid; e < NE; e += Cfg::THREADS) {
     const int ix = e & (NDIR - 1), iy = (e >> BD) & (NDIR - 1);
     float3 n = oct_inverse(s_dir_c[ix], s_dir_c[iy]);
@@ -287,29 +326,14 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 #pragma unroll
     for (int k = 0; k < REP; ++k) table[e * REP + ((k + lane) & (REP - 1))] = v;
   }
-  // rotate the query rows: warp r handles row r
-  for (int r = warp; r < G; r += NWARP) {
-    constexpr int E = D / 32;
-    float v[E];
-    if (r < a.Gq) {
-      const int gi = r / a.Lq, lq = r - gi * a.Lq;
-      const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
-      const float* sg = a.signs + trow * D + lane * E;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float x = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qoff + e])
-                                 : static_cast<const float*>(a.q)[qoff + e];
-        v[e] = x * sg[e];
-      }
-      fwht_warp<E>(v, lane);
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = 0.0f;
-    }
+  // rotate the query rows: warp r handles row r (G <= 8 <= NWARP)
+  static_assert(G <= NWARP, "one warp per query row");
+  if (warp < G) {
+    fwht_warp<E>(qraw, lane);
     const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
-    float* qrow = scratch + r * QROW;  // padded rotated row
+    float* qrow = scratch + warp * QROW;  // padded rotated row
 #pragma unroll
-    for (int e = 0; e < E; ++e) qrow[lane * E + e] = v[e] * inv_sqrt_d;
+    for (int e = 0; e < E; ++e) qrow[lane * E + e] = qraw[e] * inv_sqrt_d;
     if (lane < 3 * T - D) qrow[D + lane] = 0.0f;
   }
   __syncthreads();
@@ -367,9 +391,27 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   float* pw = pbuf + warp * G * PS;
   int aborted_at = -1;
 
+  // V fragments of a whole chunk, all requested at the start of the chunk
+  // (before its logit phase, which hides their latency): k-step j covers
+  // keys s0 + 16 j + {2c4, 2c4+1, 2c4+8, 2c4+9}, 16-byte columns 8 g8 + 64 hh.
+  uint4 vall[2 * KPL][4][NCH];
+  auto load_v = [&](int64_t s0v) {
+#pragma unroll
+    for (int j = 0; j < 2 * KPL; ++j)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int64_t vk = s0v + 16 * j + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
+#pragma unroll
+        for (int hh = 0; hh < NCH; ++hh)
+          vall[j][kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
+                                       : make_uint4(0u, 0u, 0u, 0u);
+      }
+  };
+
   for (int ci = 0; ci < my_chunks; ++ci) {
     const uint32_t* buf = ring + (ci % NS) * ROWS * KW;
     const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * ci) * KW;
+    if (with_v) load_v(s0);  // in flight during the wait and the logits
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[warp][ci % NS], (ci / NS) & 1))) {
       aborted_at = ci;  // warp-uniform
       break;
@@ -504,50 +546,41 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
       }
     }
 
-    // P.V, one 32-key sub-chunk (lane = key) at a time
+    // P.V: KPL sub-chunks of 32 keys (lane = key), each two 16-key k-steps.
 #pragma unroll
-    for (int k = 0; k < KPL; ++k) {
+    for (int j = 0; j < 2 * KPL; ++j) {
+      const int k = j >> 1, ks = j & 1;
       const int64_t kb = s0 + 32 * k;
       if (kb >= k_end) break;  // warp-uniform
+      if (ks == 0) {
 #pragma unroll
-      for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
-      __syncwarp();
+        for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
+        __syncwarp();
+      }
+      uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
+      if (g8 < G) {
+        const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
+        const float2 p01 = *reinterpret_cast<const float2*>(prow);
+        const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
+        split_bf16x2(p01.x, p01.y, bh0, bl0);
+        split_bf16x2(p89.x, p89.y, bh1, bl1);
+      }
 #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        uint4 vreg[4][NCH];
+      for (int hh = 0; hh < NCH; ++hh) {
+        const uint4 k0 = vall[j][0][hh], k1 = vall[j][1][hh], k8 = vall[j][2][hh], k9 = vall[j][3][hh];
+        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+        const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int64_t vk = kb + 16 * ks + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
-#pragma unroll
-          for (int hh = 0; hh < NCH; ++hh)
-            vreg[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
-                                      : make_uint4(0u, 0u, 0u, 0u);
-        }
-        uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
-        if (g8 < G) {
-          const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
-          const float2 p01 = *reinterpret_cast<const float2*>(prow);
-          const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
-          split_bf16x2(p01.x, p01.y, bh0, bl0);
-          split_bf16x2(p89.x, p89.y, bh1, bl1);
-        }
-#pragma unroll
-        for (int hh = 0; hh < NCH; ++hh) {
-          const uint4 k0 = vreg[0][hh], k1 = vreg[1][hh], k8 = vreg[2][hh], k9 = vreg[3][hh];
-          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-          const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
-            const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
-            const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
-            const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
-            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
-          }
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
+          const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
+          const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
+          const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
+          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
+          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
         }
       }
-      __syncwarp();
+      if (ks == 1) __syncwarp();  // the P rows of this sub-chunk are consumed
     }
   }
 
@@ -629,22 +662,34 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
   const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
   const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
-  for (int j = tid; j < G * D; j += Cfg::THREADS) {
-    const int r = j / D, d = j - r * D;
-    if (r >= a.Gq) continue;
+  // 1) per row: M = max_s m_s, weights f_s = 2^(m_s - M) (kept in the free
+  //    ring memory), L = sum_s f_s l_s; one warp per row, lanes over splits
+  float* fw = reinterpret_cast<float*>(rings);  // [G][S]
+  __shared__ float s_L[8];
+  if (warp < a.Gq) {
+    const int r = warp;
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(bm + s * G + r));
-    float o = 0.0f, l = 0.0f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float f = fast_exp2(__ldcg(bm + s * G + r) - M);
-        o = fmaf(f, __ldcg(bo + (static_cast<int64_t>(s) * G + r) * D + d), o);
-        l = fmaf(f, __ldcg(bl + s * G + r), l);
-      }
+    for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, __ldcg(bm + s2 * G + r));
+    M = warp_max(M);
+    float L = 0.0f;
+    for (int s2 = lane; s2 < S; s2 += 32) {
+      const float f = M == -INFINITY ? 0.0f : fast_exp2(__ldcg(bm + s2 * G + r) - M);
+      fw[r * S + s2] = f;
+      L = fmaf(f, __ldcg(bl + s2 * G + r), L);
     }
+    L = warp_sum(L);
+    if (lane == 0) s_L[r] = L;
+  }
+  __syncthreads();
+  // 2) out = sum_s f_s O_s / L; the split loads are independent and coalesced over d
+  for (int j = tid; j < a.Gq * D; j += Cfg::THREADS) {
+    const int r = j / D, d = j - r * D;
+    float o = 0.0f;
+#pragma unroll 8
+    for (int s2 = 0; s2 < S; ++s2) o = fmaf(fw[r * S + s2], __ldcg(bo + (static_cast<int64_t>(s2) * G + r) * D + d), o);
     const int gi = r / a.Lq, lq = r - gi * a.Lq;
     const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-    a.out[row * D + d] = l > 0.0f ? o / l : 0.0f;
+    a.out[row * D + d] = s_L[r] > 0.0f ? o / s_L[r] : 0.0f;
   }
   if (tid == 0) a.counters[bh] = 0;  // ready for the next call
 }
