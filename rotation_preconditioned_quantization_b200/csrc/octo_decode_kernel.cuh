@@ -82,6 +82,9 @@ struct DecodeArgs {
 #ifndef OCTO_DECODE_MAX_WARPS
 #define OCTO_DECODE_MAX_WARPS 8   // warps per CTA (16 only if shared memory allows)
 #endif
+#ifndef OCTO_DECODE_KPL
+#define OCTO_DECODE_KPL 4         // keys per lane per chunk (d <= 128; half of it for d = 256)
+#endif
 #ifndef OCTO_DECODE_FOLD_BITS
 #define OCTO_DECODE_FOLD_BITS 10  // full-code table when a triplet code has at most this many bits
 #endif
@@ -96,7 +99,7 @@ struct DecCfg {
   static constexpr bool FOLD = C <= OCTO_DECODE_FOLD_BITS;  // table indexed by the full code (b <= 3)
   static constexpr int NE = FOLD ? (1 << C) : (1 << (2 * BD));
   static constexpr int REP = NE <= 256 ? 8 : 4;           // replicas per entry (bank groups)
-  static constexpr int KPL = D <= 128 ? 2 : 1;             // keys per lane per chunk
+  static constexpr int KPL = D <= 128 ? OCTO_DECODE_KPL : (OCTO_DECODE_KPL + 1) / 2;  // keys per lane per chunk
   static constexpr int KW = 32 * KPL;                      // keys per chunk (one warp's unit of work)
   static constexpr int NS_MAX = 2;                         // chunks in flight per warp (at most)
   static constexpr int QF = 3 * G;                         // rotated-query floats per triplet
@@ -391,27 +394,26 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   float* pw = pbuf + warp * G * PS;
   int aborted_at = -1;
 
-  // V fragments of a whole chunk, all requested at the start of the chunk
-  // (before its logit phase, which hides their latency): k-step j covers
-  // keys s0 + 16 j + {2c4, 2c4+1, 2c4+8, 2c4+9}, 16-byte columns 8 g8 + 64 hh.
-  uint4 vall[2 * KPL][4][NCH];
-  auto load_v = [&](int64_t s0v) {
+  // V fragments of 16-key step j of a chunk (keys s0 + 16 j + {2c4, 2c4+1,
+  // 2c4+8, 2c4+9}, 16-byte columns 8 g8 + 64 hh); step j + 1 is loaded while
+  // step j multiplies, step 0 while the chunk's logits are computed.
+  constexpr bool VPIPE = NCH <= 2;
+  auto load_v_step = [&](uint4 (&dst)[4][NCH], int64_t s0v, int j) {
 #pragma unroll
-    for (int j = 0; j < 2 * KPL; ++j)
+    for (int kk = 0; kk < 4; ++kk) {
+      const int64_t vk = s0v + 16 * j + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int64_t vk = s0v + 16 * j + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
-#pragma unroll
-        for (int hh = 0; hh < NCH; ++hh)
-          vall[j][kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
-                                       : make_uint4(0u, 0u, 0u, 0u);
-      }
+      for (int hh = 0; hh < NCH; ++hh)
+        dst[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+    }
   };
+  uint4 vcur[4][NCH], vnext[4][NCH];  // vnext is dead unless VPIPE
 
   for (int ci = 0; ci < my_chunks; ++ci) {
     const uint32_t* buf = ring + (ci % NS) * ROWS * KW;
     const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * ci) * KW;
-    if (with_v) load_v(s0);  // in flight during the wait and the logits
+    if (VPIPE && with_v) load_v_step(vcur, s0, 0);  // in flight during the wait and the logits
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[warp][ci % NS], (ci / NS) & 1))) {
       aborted_at = ci;  // warp-uniform
       break;
@@ -557,6 +559,11 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
         for (int r = 0; r < G; ++r) pw[r * PS + lane] = lg[k][r];
         __syncwarp();
       }
+      if constexpr (VPIPE) {
+        if (j + 1 < 2 * KPL) load_v_step(vnext, s0, j + 1);  // keys past the end load as zeros
+      } else {
+        load_v_step(vcur, s0, j);
+      }
       uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
       if (g8 < G) {
         const float* prow = pw + g8 * PS + 16 * ks + 2 * c4;
@@ -567,7 +574,7 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
       }
 #pragma unroll
       for (int hh = 0; hh < NCH; ++hh) {
-        const uint4 k0 = vall[j][0][hh], k1 = vall[j][1][hh], k8 = vall[j][2][hh], k9 = vall[j][3][hh];
+        const uint4 k0 = vcur[0][hh], k1 = vcur[1][hh], k8 = vcur[2][hh], k9 = vcur[3][hh];
         const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
         const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
 #pragma unroll
@@ -579,6 +586,12 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
           mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
           mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
         }
+      }
+      if constexpr (VPIPE) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int hh = 0; hh < NCH; ++hh) vcur[kk][hh] = vnext[kk][hh];
       }
       if (ks == 1) __syncwarp();  // the P rows of this sub-chunk are consumed
     }
@@ -650,48 +663,40 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   if (S == 1) return;
 
   // ------------------------------------------------ epilogue: merge splits (last CTA of this head)
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const int ticket = atomicAdd(a.counters + bh, 1);
+    // release our partials (written by this CTA, ordered by the barrier) and,
+    // for the last arrival, acquire everyone else's
+    int ticket;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(a.counters + bh) : "memory");
     s_last = ticket == S - 1;
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
   const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
   const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
-  // 1) per row: M = max_s m_s, weights f_s = 2^(m_s - M) (kept in the free
-  //    ring memory), L = sum_s f_s l_s; one warp per row, lanes over splits
-  float* fw = reinterpret_cast<float*>(rings);  // [G][S]
-  __shared__ float s_L[8];
-  if (warp < a.Gq) {
-    const int r = warp;
-    float M = -INFINITY;
-    for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, __ldcg(bm + s2 * G + r));
-    M = warp_max(M);
-    float L = 0.0f;
-    for (int s2 = lane; s2 < S; s2 += 32) {
-      const float f = M == -INFINITY ? 0.0f : fast_exp2(__ldcg(bm + s2 * G + r) - M);
-      fw[r * S + s2] = f;
-      L = fmaf(f, __ldcg(bl + s2 * G + r), L);
-    }
-    L = warp_sum(L);
-    if (lane == 0) s_L[r] = L;
-  }
-  __syncthreads();
-  // 2) out = sum_s f_s O_s / L; the split loads are independent and coalesced over d
+  // every thread loads its (row, column)'s S partials plus the row's (m, l)
+  // in one round (independent, coalesced over d), then combines them
   for (int j = tid; j < a.Gq * D; j += Cfg::THREADS) {
     const int r = j / D, d = j - r * D;
-    float o = 0.0f;
+    float M = -INFINITY;
 #pragma unroll 8
-    for (int s2 = 0; s2 < S; ++s2) o = fmaf(fw[r * S + s2], __ldcg(bo + (static_cast<int64_t>(s2) * G + r) * D + d), o);
+    for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, __ldcg(bm + s2 * G + r));
+    float o = 0.0f, l = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll 8
+      for (int s2 = 0; s2 < S; ++s2) {
+        const float f = fast_exp2(__ldcg(bm + s2 * G + r) - M);
+        o = fmaf(f, __ldcg(bo + (static_cast<int64_t>(s2) * G + r) * D + d), o);
+        l = fmaf(f, __ldcg(bl + s2 * G + r), l);
+      }
+    }
     const int gi = r / a.Lq, lq = r - gi * a.Lq;
     const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-    a.out[row * D + d] = s_L[r] > 0.0f ? o / s_L[r] : 0.0f;
+    a.out[row * D + d] = l > 0.0f ? o / l : 0.0f;
   }
-  if (tid == 0) a.counters[bh] = 0;  // ready for the next call
+  if (tid == 0) atomicExch(a.counters + bh, 0);  // ready for the next call
 }
 
 // Launch one decode instantiation for head dimension D (defined in the
