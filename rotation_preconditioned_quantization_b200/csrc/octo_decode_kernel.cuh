@@ -699,19 +699,558 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   if (tid == 0) atomicExch(a.counters + bh, 0);  // ready for the next call
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core logits (codes of at most 10 bits, i.e. b <= 3, and d <= 128).
+//
+// For a GQA group the logits of a tile of keys are a dense contraction,
+// logits[key][row] = sum_c u_hat[key][c] q_rot[row][c], so they run on
+// mma.sync m16n8k16 bf16 with keys as M, query rows as N (padded to 8) and
+// rotated coordinates as K. Each 16-wide k-step holds 4 triplets: lane
+// column c4 carries triplet 4s + c4 as (x, y | z, 0), so a lane decodes one
+// triplet code per key per k-step. The shared-memory table stores every
+// decoded triplet rho_hat * n_hat already split into bf16 hi + lo halves, in
+// exactly the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); the
+// rotated queries are B fragments held in registers for the whole CTA.
+// Three products (hi.hi + hi.lo + lo.hi) keep about 16 mantissa bits, well
+// inside the logit tolerance. With OCTOPUS-QJL the sketch term is a second
+// contraction of the +-1 sign bits against p = S q_rot, on the same units.
+// ---------------------------------------------------------------------------
+template <int D, int B, int G, bool QJL>
+struct TcCfg {
+  static constexpr int T = (D + 2) / 3;
+  static constexpr int BD = B + 1, BR = B - 1;
+  static constexpr int C = 2 * BD + BR;
+  static constexpr int W = (T * C + 31) / 32;
+  static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
+  static constexpr int NE = 1 << C;          // full-code table
+  static constexpr int REP = 8;              // replicas (distinct bank groups per quarter-warp)
+  static constexpr int NKS = (T + 3) / 4;    // logit k-steps (4 triplets each)
+  static constexpr int KW = 64;              // keys per chunk
+  static constexpr int MTL = KW / 16;        // m-tiles per chunk
+  static constexpr int SW = KW + 8;          // padded row stride of a staged chunk (words)
+  static constexpr int QW = D / 32;          // sketch words per key
+  static constexpr int QKS = D / 16;         // sketch k-steps
+  static constexpr int NWARP = 8, THREADS = 256;
+  static constexpr int ROWS = W + 1 + (QJL ? QW + 1 : 0);
+  static constexpr size_t CHUNK = sizeof(uint32_t) * ROWS * SW;
+  static constexpr int PS = KW + 8;          // P row stride (floats)
+  static constexpr int MT = D / 16, NCH = D / 64;
+  static constexpr size_t TABLE = sizeof(uint4) * NE * REP;
+  static constexpr size_t QROW = (12 * NKS > D + 4 ? 12 * NKS : D + 4);  // padded rotated query row
+  static constexpr size_t SCRATCH = (sizeof(float) * G * (QROW + (QJL ? D : 0)) + 15) / 16 * 16;
+  static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per warp
+  static constexpr size_t cmax(size_t x, size_t y) { return x > y ? x : y; }
+  static constexpr size_t ring_bytes(int ns) {
+    return (cmax(cmax(ns * CHUNK, sizeof(float) * G * (D + 2)), sizeof(float) * G * 1024 / 8) + 127) / 128 * 128;
+  }
+  static constexpr size_t FIXED = TABLE + SCRATCH;
+  static constexpr size_t BUDGET = 227 * 1024 - 2048;
+  static constexpr int NS = FIXED + NWARP * (PBUF + ring_bytes(2)) <= BUDGET ? 2 : 1;
+  static constexpr size_t RING = ring_bytes(NS);
+  static constexpr size_t SMEM = FIXED + NWARP * (PBUF + RING);
+  static_assert(SMEM <= BUDGET, "shared memory budget");
+  static_assert(G <= 8 && D <= 128, "tensor-core logits shape");
+};
+
+__device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi) {
+  // +1 / -1 in bf16 (0x3F80 / 0xBF80) for sketch bits 1 / 0
+  return 0xBF80BF80u ^ ((bit_lo & 1u) << 15) ^ ((bit_hi & 1u) << 31);
+}
+
+template <int D, int B, int G, bool QJL>
+__global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
+  using Cfg = TcCfg<D, B, G, QJL>;
+  constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, BD = Cfg::BD, NDIR = Cfg::NDIR;
+  constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, QW = Cfg::QW, NKS = Cfg::NKS;
+  constexpr int KW = Cfg::KW, MTL = Cfg::MTL, SW = Cfg::SW, NS = Cfg::NS, ROWS = Cfg::ROWS;
+  constexpr int PS = Cfg::PS, MT = Cfg::MT, NCH = Cfg::NCH, QKS = Cfg::QKS;
+  constexpr int QROW = static_cast<int>(Cfg::QROW);
+
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  uint4* table = reinterpret_cast<uint4*>(smem_raw);                                     // [NE][REP]
+  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::TABLE);                      // [G][QROW] (+ [G][D])
+  unsigned char* per_warp = smem_raw + Cfg::FIXED;                                       // [NWARP] x (PBUF + RING)
+  __shared__ float s_rho_c[8];
+  __shared__ float s_dir_c[32];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g8 = lane >> 2, c4 = lane & 3;
+  const int split = blockIdx.x;
+  const int bh = blockIdx.y;  // b * Hkv + h_kv
+  const int bidx = bh / a.Hkv, hkv = bh - bidx * a.Hkv;
+  const int64_t trow = bh % a.table_heads;
+  const bool with_v = a.V != nullptr;
+
+  const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
+  const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
+  const int n_chunks = static_cast<int>((k_end - k_begin + KW - 1) / KW);
+  const int my_chunks = warp < n_chunks ? (n_chunks - warp + NWARP - 1) / NWARP : 0;
+  const uint32_t* pk = a.packed + static_cast<int64_t>(bh) * W * a.cache_cap;
+  const float* gm = a.gamma + static_cast<int64_t>(bh) * a.cache_cap;
+  const __nv_bfloat16* Vh = with_v ? a.V + static_cast<int64_t>(bh) * a.cache_cap * D : nullptr;
+  const uint32_t* qbp = QJL ? a.qjl_bits + static_cast<int64_t>(bh) * QW * a.cache_cap : nullptr;
+  const float* qnp = QJL ? a.qjl_norm + static_cast<int64_t>(bh) * a.cache_cap : nullptr;
+  float* pw = reinterpret_cast<float*>(per_warp + warp * (Cfg::PBUF + Cfg::RING));                  // [G][PS]
+  uint32_t* ring = reinterpret_cast<uint32_t*>(per_warp + warp * (Cfg::PBUF + Cfg::RING) + Cfg::PBUF);  // [NS][ROWS][SW]
+
+  // Chunk i of this warp (keys k_begin + (warp + NWARP i) KW ...): the lanes
+  // copy its rows (code words, gammas, sketch words, norms) into ring slot
+  // i % NS with 16-byte cp.async copies (one commit group per chunk), and
+  // prefetch its V rows into L2. Keys are copied in groups of 4; the cache
+  // capacity is a multiple of 4 and chunks start at multiples of KW, so the
+  // rounded-up copy stays inside the cache rows (keys past kv_len are masked).
+  auto issue_chunk = [&](int i) {
+    const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * i) * KW;
+    const int n = static_cast<int>(k_end - s0 < KW ? k_end - s0 : KW);
+    const int groups = (n + 3) >> 2;
+    uint32_t* buf = ring + (i % NS) * ROWS * SW;
+    for (int p = lane; p < ROWS * (KW / 4); p += 32) {
+      const int r = p / (KW / 4), c = p - r * (KW / 4);
+      if (c >= groups) continue;
+      const void* src;
+      if (r < W) src = pk + r * a.cache_cap + s0 + 4 * c;
+      else if (r == W) src = gm + s0 + 4 * c;
+      else if (QJL && r < W + 1 + QW) src = qbp + (r - W - 1) * a.cache_cap + s0 + 4 * c;
+      else src = qnp + s0 + 4 * c;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(buf + r * SW + 4 * c)), "l"(src)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (with_v) {
+      const char* v0 = reinterpret_cast<const char*>(Vh + s0 * D);
+      for (int64_t off = static_cast<int64_t>(lane) * 128; off < static_cast<int64_t>(n) * D * 2; off += 32 * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(v0 + off));
+    }
+  };
+  // small global reads first (codebooks, one sign-flipped query row per warp)
+  constexpr int E = D / 32;
+  float qraw[E];
+  if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
+  if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
+  if (warp < G && warp < a.Gq) {
+    const int gi = warp / a.Lq, lq = warp - gi * a.Lq;
+    const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
+    const float* sg = a.signs + trow * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float x = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qoff + e])
+                               : static_cast<const float*>(a.q)[qoff + e];
+      qraw[e] = x * __ldg(sg + e);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) qraw[e] = 0.0f;
+  }
+  for (int i = 0; i < NS && i < my_chunks; ++i) issue_chunk(i);
+  __syncthreads();
+
+  // ------------------------------------------------ prologue (overlaps the first copies)
+  // decoded-triplet table, pre-split into bf16 hi + lo fragment halves
+  for (int e = tid; e < NE; e += Cfg::THREADS) {
+    const int ix = e & (NDIR - 1), iy = (e >> BD) & (NDIR - 1);
+    float3 n = oct_inverse(s_dir_c[ix], s_dir_c[iy]);
+    const float r = s_rho_c[e >> (2 * BD)];
+    n.x *= r; n.y *= r; n.z *= r;
+    uint32_t xyh, xyl, zh, zl;
+    split_bf16x2(n.x, n.y, xyh, xyl);
+    split_bf16x2(n.z, 0.0f, zh, zl);
+    const uint4 v = make_uint4(xyh, zh, xyl, zl);
+#pragma unroll
+    for (int k = 0; k < REP; ++k) table[e * REP + ((k + lane) & (REP - 1))] = v;
+  }
+  // rotate the query rows: warp r handles row r
+  if (warp < G) {
+    fwht_warp<E>(qraw, lane);
+    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+    float* qrow = scratch + warp * QROW;
+#pragma unroll
+    for (int e = 0; e < E; ++e) qrow[lane * E + e] = qraw[e] * inv_sqrt_d;
+    for (int c = D + lane; c < QROW; c += 32) qrow[c] = 0.0f;  // zero pad to whole k-steps
+  }
+  __syncthreads();
+  if constexpr (QJL) {
+    float* p = scratch + G * QROW;  // [G][D]: p_r = S q_rot_r
+    const float* S = a.qjl_S + trow * D * D;
+    for (int j = tid; j < G * D; j += Cfg::THREADS) {
+      const int r = j / D, m = j - r * D;
+      const float* qrow = scratch + r * QROW;
+      const float* srow = S + static_cast<int64_t>(m) * D;
+      float acc = 0.0f;
+      for (int t = 0; t < D; ++t) acc = fmaf(__ldg(srow + t), qrow[t], acc);
+      p[j] = acc;
+    }
+    __syncthreads();
+  }
+
+  // B fragments of the rotated queries (row g8, triplet 4s + c4 as (x, y | z, 0)), hi and lo
+  uint32_t bq[NKS][4];
+#pragma unroll
+  for (int s = 0; s < NKS; ++s) {
+    const int t = 4 * s + c4;
+    float x = 0.0f, y = 0.0f, z = 0.0f;
+    if (g8 < G) {
+      const float* qrow = scratch + g8 * QROW;
+      x = qrow[3 * t]; y = qrow[3 * t + 1]; z = qrow[3 * t + 2];
+    }
+    split_bf16x2(x, y, bq[s][0], bq[s][2]);
+    split_bf16x2(z, 0.0f, bq[s][1], bq[s][3]);
+  }
+  // sketch B fragments: p row g8, sketch coordinates 16 ks + {2c4, 2c4+1 | 2c4+8, 2c4+9}
+  uint32_t bp[QJL ? QKS : 1][4];
+  if constexpr (QJL) {
+#pragma unroll
+    for (int ks = 0; ks < QKS; ++ks) {
+      float p0 = 0.0f, p1 = 0.0f, p8 = 0.0f, p9 = 0.0f;
+      if (g8 < G) {
+        const float* prow = scratch + G * QROW + g8 * D + 16 * ks + 2 * c4;
+        p0 = prow[0]; p1 = prow[1]; p8 = prow[8]; p9 = prow[9];
+      }
+      split_bf16x2(p0, p1, bp[ks][0], bp[ks][2]);
+      split_bf16x2(p8, p9, bp[ks][1], bp[ks][3]);
+    }
+  }
+  // where this lane's triplet code of each k-step sits in a key's bit stream
+  uint32_t cpos[NKS];  // word << 8 | shift, or 0xFFFF for padding triplets
+#pragma unroll
+  for (int s = 0; s < NKS; ++s) {
+    const int t = 4 * s + c4;
+    cpos[s] = t < T ? (static_cast<uint32_t>((t * C) >> 5) << 8) | static_cast<uint32_t>((t * C) & 31) : 0xFFFFu;
+  }
+  const int rep_off = lane & (REP - 1);
+
+  // ------------------------------------------------ main loop: this warp's chunks
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // this lane's query columns 2c4, 2c4+1
+  float acc_o[MT][4];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) acc_o[t][0] = acc_o[t][1] = acc_o[t][2] = acc_o[t][3] = 0.0f;
+#ifndef OCTO_DECODE_TC_VALL
+#define OCTO_DECODE_TC_VALL 0  // 1: load all of a chunk's V fragments before its logits (spills at d = 128)
+#endif
+  constexpr bool VALL = OCTO_DECODE_TC_VALL && NCH <= 2 && !QJL;  // (the sketch fragments need the registers)
+  constexpr bool VPIPE = !VALL && NCH <= 2;
+  auto load_v_step = [&](uint4 (&dst)[4][NCH], int64_t s0v, int j) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int64_t vk = s0v + 16 * j + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
+#pragma unroll
+      for (int hh = 0; hh < NCH; ++hh)
+        dst[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 vcur[4][NCH], vnext[4][NCH];
+  uint4 vall[VALL ? KW / 16 : 1][4][NCH];
+  const bool q0_real = 2 * c4 < a.Gq, q1_real = 2 * c4 + 1 < a.Gq;
+  for (int ci = 0; ci < my_chunks; ++ci) {
+    const uint32_t* buf = ring + (ci % NS) * ROWS * SW;
+    const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * ci) * KW;
+    if constexpr (VALL) {
+      if (with_v) {  // in flight during the wait and the logits
+#pragma unroll
+        for (int j = 0; j < KW / 16; ++j) load_v_step(vall[j], s0, j);
+      }
+    } else {
+      if (VPIPE && with_v) load_v_step(vcur, s0, 0);  // in flight during the wait and the logits
+    }
+    // this lane's copies of chunk ci are complete (later chunks may still be in
+    // flight), then the warp's: everyone's rows are visible after the syncwarp
+    if (ci + 1 < my_chunks && NS > 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+    else asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+
+    // logits of the chunk in C-fragment layout: lgv[mt] = (kA, q0), (kA, q1), (kB, q0), (kB, q1)
+    float lgv[MTL][4];
+#pragma unroll
+    for (int mt = 0; mt < MTL; ++mt) {
+      const int kA = 16 * mt + g8, kB = kA + 8;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int s = 0; s < NKS; ++s) {
+        uint4 eA = make_uint4(0u, 0u, 0u, 0u), eB = eA;
+        if (cpos[s] != 0xFFFFu) {
+          const int wi = static_cast<int>(cpos[s] >> 8), sh = static_cast<int>(cpos[s] & 31u);
+          const uint32_t* rw = buf + wi * SW;
+          const uint32_t hiA = wi + 1 < W ? rw[SW + kA] : 0u, hiB = wi + 1 < W ? rw[SW + kB] : 0u;
+          const uint32_t cA = __funnelshift_r(rw[kA], hiA, sh) & ((1u << C) - 1u);
+          const uint32_t cB = __funnelshift_r(rw[kB], hiB, sh) & ((1u << C) - 1u);
+          eA = table[cA * REP + rep_off];
+          eB = table[cB * REP + rep_off];
+        }
+        mma_bf16_16816(acc, eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
+        mma_bf16_16816(acc, eA.x, eB.x, eA.y, eB.y, bq[s][2], bq[s][3]);
+        mma_bf16_16816(acc, eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
+      }
+      const float gA = __uint_as_float(buf[W * SW + kA]), gB = __uint_as_float(buf[W * SW + kB]);
+      if constexpr (QJL) {
+        float accq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ks = 0; ks < QKS; ++ks) {
+          const uint32_t wA = buf[(W + 1 + (ks >> 1)) * SW + kA] >> (16 * (ks & 1) + 2 * c4);
+          const uint32_t wB = buf[(W + 1 + (ks >> 1)) * SW + kB] >> (16 * (ks & 1) + 2 * c4);
+          const uint32_t a0 = pm1_bf16x2(wA, wA >> 1), a1 = pm1_bf16x2(wB, wB >> 1);
+          const uint32_t a2 = pm1_bf16x2(wA >> 8, wA >> 9), a3 = pm1_bf16x2(wB >> 8, wB >> 9);
+          mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
+          mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][2], bp[ks][3]);
+        }
+        const float kq = 1.2533141373155003f / static_cast<float>(D);  // sqrt(pi/2)/m, m = d
+        const float fA = kq * __uint_as_float(buf[(W + 1 + QW) * SW + kA]);
+        const float fB = kq * __uint_as_float(buf[(W + 1 + QW) * SW + kB]);
+        acc[0] = fmaf(fA, accq[0], acc[0]); acc[1] = fmaf(fA, accq[1], acc[1]);
+        acc[2] = fmaf(fB, accq[2], acc[2]); acc[3] = fmaf(fB, accq[3], acc[3]);
+      }
+      lgv[mt][0] = acc[0] * gA; lgv[mt][1] = acc[1] * gA;
+      lgv[mt][2] = acc[2] * gB; lgv[mt][3] = acc[3] * gB;
+    }
+    // this warp is done with the chunk's rows: refill the slot with chunk ci + NS
+    __syncwarp();
+    if (ci + NS < my_chunks) issue_chunk(ci + NS);
+
+    if (a.logits != nullptr) {
+#pragma unroll
+      for (int mt = 0; mt < MTL; ++mt) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t key = s0 + 16 * mt + g8 + 8 * h;
+          if (key >= k_end) continue;
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int r = 2 * c4 + qq;
+            if (r < a.Gq) {
+              const int gi = r / a.Lq, lq = r - gi * a.Lq;
+              const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
+              a.logits[row * a.kv_len + key] = lgv[mt][2 * h + qq];
+            }
+          }
+        }
+      }
+    }
+    if (!with_v) continue;
+
+    // online softmax over the chunk, base 2, per query column; keys live on the g8 lanes
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < MTL; ++mt) {
+      const bool vA = s0 + 16 * mt + g8 < k_end, vB = s0 + 16 * mt + g8 + 8 < k_end;
+      lgv[mt][0] = vA ? lgv[mt][0] * a.scale_log2 : -INFINITY;
+      lgv[mt][1] = vA ? lgv[mt][1] * a.scale_log2 : -INFINITY;
+      lgv[mt][2] = vB ? lgv[mt][2] * a.scale_log2 : -INFINITY;
+      lgv[mt][3] = vB ? lgv[mt][3] * a.scale_log2 : -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(lgv[mt][0], lgv[mt][2]));
+      mx1 = fmaxf(mx1, fmaxf(lgv[mt][1], lgv[mt][3]));
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
+    m0 = n0; m1 = n1;
+    float ps0 = 0.0f, ps1 = 0.0f;
+#pragma unroll
+    for (int mt = 0; mt < MTL; ++mt) {
+      lgv[mt][0] = fast_exp2(lgv[mt][0] - n0); lgv[mt][2] = fast_exp2(lgv[mt][2] - n0);
+      lgv[mt][1] = fast_exp2(lgv[mt][1] - n1); lgv[mt][3] = fast_exp2(lgv[mt][3] - n1);
+      ps0 += lgv[mt][0] + lgv[mt][2];
+      ps1 += lgv[mt][1] + lgv[mt][3];
+    }
+    l0 = l0 * al0 + ps0;
+    l1 = l1 * al1 + ps1;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
+    }
+    // P rows (query-major) for the P.V B fragments
+#pragma unroll
+    for (int mt = 0; mt < MTL; ++mt) {
+      const int kA = 16 * mt + g8;
+      if (2 * c4 < G) { pw[(2 * c4) * PS + kA] = lgv[mt][0]; pw[(2 * c4) * PS + kA + 8] = lgv[mt][2]; }
+      if (2 * c4 + 1 < G) { pw[(2 * c4 + 1) * PS + kA] = lgv[mt][1]; pw[(2 * c4 + 1) * PS + kA + 8] = lgv[mt][3]; }
+    }
+    __syncwarp();
+
+    // P.V over the chunk's 16-key steps
+#pragma unroll
+    for (int j = 0; j < KW / 16; ++j) {
+      if (s0 + 16 * j >= k_end) break;  // warp-uniform
+      if constexpr (VALL) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int hh = 0; hh < NCH; ++hh) vcur[kk][hh] = vall[VALL ? j : 0][kk][hh];
+      } else if constexpr (VPIPE) {
+        if (j + 1 < KW / 16) load_v_step(vnext, s0, j + 1);  // keys past the end load as zeros
+      } else {
+        load_v_step(vcur, s0, j);
+      }
+      uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
+      if (g8 < G) {
+        const float* prow = pw + g8 * PS + 16 * j + 2 * c4;
+        const float2 p01 = *reinterpret_cast<const float2*>(prow);
+        const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
+        split_bf16x2(p01.x, p01.y, bh0, bl0);
+        split_bf16x2(p89.x, p89.y, bh1, bl1);
+      }
+#pragma unroll
+      for (int hh = 0; hh < NCH; ++hh) {
+        const uint4 k0 = vcur[0][hh], k1 = vcur[1][hh], k8 = vcur[2][hh], k9 = vcur[3][hh];
+        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+        const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
+          const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
+          const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
+          const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
+          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
+          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
+        }
+      }
+      if constexpr (VPIPE) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int hh = 0; hh < NCH; ++hh) vcur[kk][hh] = vnext[kk][hh];
+      }
+    }
+    __syncwarp();  // P rows consumed before the next chunk overwrites them
+  }
+
+  __syncthreads();  // every ring is free: no copy is in flight after the last chunk
+  if (!with_v) return;
+
+  // ------------------------------------------------ epilogue: merge warps (in each warp's ring)
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  auto wbase = [&](int w) { return reinterpret_cast<float*>(per_warp + w * (Cfg::PBUF + Cfg::RING) + Cfg::PBUF); };
+  {
+    float* wm = wbase(warp);  // [G] m, [G] l, [G][D] O
+    if (g8 == 0) {
+      if (2 * c4 < G) { wm[2 * c4] = m0; wm[G + 2 * c4] = l0; }
+      if (2 * c4 + 1 < G) { wm[2 * c4 + 1] = m1; wm[G + 2 * c4 + 1] = l1; }
+    }
+    float* o = wm + 2 * G;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const int hh = t >> 2, e2 = t & 3;
+      const int d0 = 64 * hh + 8 * g8 + 2 * e2;
+      const int q0 = 2 * c4, q1 = 2 * c4 + 1;
+      if (q0 < G) { o[q0 * D + d0] = acc_o[t][0]; o[q0 * D + d0 + 1] = acc_o[t][2]; }
+      if (q1 < G) { o[q1 * D + d0] = acc_o[t][1]; o[q1 * D + d0 + 1] = acc_o[t][3]; }
+    }
+  }
+  __syncthreads();
+  (void)q0_real; (void)q1_real;
+
+  const int S = a.n_splits;
+  float* pm = a.part_m + (static_cast<int64_t>(bh) * S + split) * G;
+  float* pl = a.part_l + (static_cast<int64_t>(bh) * S + split) * G;
+  float* po = a.part_o + (static_cast<int64_t>(bh) * S + split) * G * D;
+  for (int j = tid; j < G * D; j += Cfg::THREADS) {
+    const int r = j / D, d = j - r * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NWARP; ++w) M = fmaxf(M, wbase(w)[r]);
+    float o = 0.0f, l = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NWARP; ++w) {
+        const float f = fast_exp2(wbase(w)[r] - M);
+        o = fmaf(f, wbase(w)[2 * G + r * D + d], o);
+        l = fmaf(f, wbase(w)[G + r], l);
+      }
+    }
+    if (S == 1) {
+      if (r < a.Gq) {
+        const int gi = r / a.Lq, lq = r - gi * a.Lq;
+        const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
+        a.out[row * D + d] = l > 0.0f ? o / l : 0.0f;
+      }
+    } else {
+      po[j] = o;
+      if (d == 0) { pm[r] = M; pl[r] = l; }
+    }
+  }
+  if (S == 1) return;
+
+  // ------------------------------------------------ epilogue: merge splits (last CTA of this head)
+  __syncthreads();
+  if (tid == 0) {
+    int ticket;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(a.counters + bh) : "memory");
+    s_last = ticket == S - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
+  const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
+  const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
+  // Each thread merges its (row, column) outputs over the S split partials,
+  // 32 splits per round of independent loads (one L2 round trip per round).
+  for (int j = tid; j < a.Gq * D; j += Cfg::THREADS) {
+    const int r = j / D, d = j - r * D;
+    float M = -INFINITY, o = 0.0f, l = 0.0f;
+    for (int sb = 0; sb < S; sb += 32) {
+      float mv[32], lv[32], ov[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const int s2 = sb + k;
+        const bool ok = s2 < S;
+        mv[k] = ok ? __ldcg(bm + s2 * G + r) : -INFINITY;
+        lv[k] = ok ? __ldcg(bl + s2 * G + r) : 0.0f;
+        ov[k] = ok ? __ldcg(bo + (static_cast<int64_t>(s2) * G + r) * D + d) : 0.0f;
+      }
+      float Mb = M;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) Mb = fmaxf(Mb, mv[k]);
+      if (Mb == -INFINITY) continue;
+      const float sc = fast_exp2(M - Mb);  // rescale the rounds merged so far
+      o *= sc;
+      l *= sc;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float f = fast_exp2(mv[k] - Mb);
+        o = fmaf(f, ov[k], o);
+        l = fmaf(f, lv[k], l);
+      }
+      M = Mb;
+    }
+    const int gi = r / a.Lq, lq = r - gi * a.Lq;
+    const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
+    a.out[row * D + d] = l > 0.0f ? o / l : 0.0f;
+  }
+  if (tid == 0) atomicExch(a.counters + bh, 0);  // ready for the next call
+}
+
 // Launch one decode instantiation for head dimension D (defined in the
 // per-D translation units so that the templates compile in parallel).
 cudaError_t launch_decode_d64(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
 cudaError_t launch_decode_d128(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
 cudaError_t launch_decode_d256(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
 
+#ifndef OCTO_DECODE_TC
+#define OCTO_DECODE_TC 1  // tensor-core logits where the shape allows
+#endif
+
 template <int D, int B, int G, bool QJL>
 cudaError_t launch_decode_one(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  using Cfg = DecCfg<D, B, G, QJL>;
-  auto k = decode_kernel<D, B, G, QJL>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
-  if (e != cudaSuccess) return e;
-  k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a);  // grid: (splits, heads)
+  if constexpr (OCTO_DECODE_TC && D <= 128 && 3 * B + 1 <= 10) {
+    using Cfg = TcCfg<D, B, G, QJL>;
+    auto k = decode_tc_kernel<D, B, G, QJL>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
+    if (e != cudaSuccess) return e;
+    k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a);  // grid: (splits, heads)
+  } else {
+    using Cfg = DecCfg<D, B, G, QJL>;
+    auto k = decode_kernel<D, B, G, QJL>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
+    if (e != cudaSuccess) return e;
+    k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a);  // grid: (splits, heads)
+  }
   return cudaGetLastError();
 }
 
