@@ -199,6 +199,35 @@ OCTO_API int octo_decode_attn(const octo_layout* L, const octo_tables* tables,
                      const void* V, float scale, float* out, float* logits,
                      void* workspace, size_t ws_bytes, octo_stream_t stream);
 
+/* Device. octo_decode_attn without a caller-provided workspace, for callers
+ * that cannot allocate device memory themselves: for example a plugin whose
+ * host framework owns every device allocation, or a caller whose allocator
+ * cannot be reached from the code that issues the decode step. It allocates
+ * nothing: the split-merge scratch is a fixed array of
+ * OCTO_STATIC_SCRATCH_BYTES (8 MiB) in the library's own device memory,
+ * reserved on every GPU that loads the library until the process exits.
+ * (Not part of the method: the paper has no counterpart; this is a
+ * deployment convenience.)
+ * Arguments and results are those of octo_decode_attn, minus the workspace.
+ *   - Returns OCTO_EWORKSPACE when the sizes need more scratch than
+ *     OCTO_STATIC_SCRATCH_BYTES (octo_decode_attn_workspace() tells).
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call outside any stream
+ *     capture.
+ *   - Each call zeroes the array's status word and arrival counters on
+ *     `stream` before the decode kernel. All calls on a device share the
+ *     array, which keeps the last call's contents: calls that overlap on
+ *     the GPU (other streams, or other threads) race on it and must not be
+ *     issued. */
+#define OCTO_STATIC_SCRATCH_BYTES (8u << 20)
+OCTO_API int octo_decode_attn_static(const octo_layout* L, const octo_tables* tables,
+                                     const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
+                                     int64_t kv_len, int64_t cache_cap,
+                                     const uint32_t* packed, const float* gamma,
+                                     const uint32_t* qjl_bits, const float* qjl_norm,
+                                     const void* V, float scale, float* out, float* logits,
+                                     octo_stream_t stream);
+
 /* Static string for a status code. */
 OCTO_API const char* octo_status_string(int status);
 
