@@ -22,9 +22,11 @@ the method) on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
+import re
 import sys
 import threading
 import time
@@ -37,6 +39,7 @@ sys.path.insert(0, ROOT)
 # workload
 B, HQ, HKV, D, N, BITS = 1, 32, 8, 128, 32768, 3
 SEED = 0
+METRIC = "compressed-KV decode-attention HBM GB/s (% of ~8 TB/s); encode Mkeys/s"
 WORKLOAD = "llm-decode: B=1, Hq=32, Hkv=8 (GQA 4), d=128, ctx=32768, bf16 K/V/q, b=3 joint"
 
 
@@ -210,7 +213,7 @@ def run_reference(args):
     enc_s = float(np.mean([s["encode_s"] for s in steps]))
     val = float(np.mean([s["value"] for s in steps]))
     line = {
-        "impl": "reference", "metric": "decode-attention HBM GB/s (encode Mkeys/s alongside)", "value": val,
+        "impl": "reference", "metric": METRIC, "value": val,
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * (dec_s + enc_s), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
@@ -336,7 +339,7 @@ def run_gpu(args):
     if rank != 0:
         return 0
     line = {
-        "metric": "decode-attention HBM GB/s (encode Mkeys/s alongside)",
+        "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -364,17 +367,32 @@ def run_gpu(args):
     return 0
 
 
+DECODE_KERNEL_SOURCES = ("octo_common.cuh", "octo_decode_kernel.cuh", "octo_decode.cu")
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_tc_kernel_llm_decode_b1_h32x8_d128_ctx32768_b3.md")
+
+
+def kernel_sources_digest(names=DECODE_KERNEL_SOURCES) -> str:
+    """sha256 over the decode kernel's sources (detects a kernel changed since its ncu capture)."""
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "rotation_preconditioned_quantization_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _ncu_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if it matches the current kernel."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if not os.path.exists(p):
-        return None
+    """DRAM bytes per decode launch from the committed ncu summary, or None when
+    the summary is missing or was taken on other kernel sources."""
     try:
-        with open(p) as f:
-            j = json.load(f)
-        return j.get("dram_bytes_per_launch")
-    except Exception:
+        with open(DECODE_PROFILE) as f:
+            text = f.read()
+    except OSError:
         return None
+    t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", text, re.M)
+    d = re.search(r"^kernel_sources_sha256:\s*([0-9a-f]{64})", text, re.M)
+    if not t or not d or d.group(1) != kernel_sources_digest():
+        return None
+    return int(t.group(1))
 
 
 def main():
