@@ -1,9 +1,13 @@
 // OCTOPUS fused decode attention: host entry points (argument checks,
 // split planning, workspace carve-up, dispatch to the per-D kernels).
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
+#include <cstring>
 
 #include "octo_decode_kernel.cuh"
 
@@ -70,6 +74,71 @@ int check_layout(const octo_layout* L) {
   return OCTO_OK;
 }
 
+// ---- tensor maps of the tensor-core kernel (host) ----------------------------
+// The encoder comes from the driver through the runtime's entry-point query,
+// so the library needs no link against the driver library.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType type, cuuint32_t rank, const void* base, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
+  const auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint32_t elem[3] = {1, 1, 1};
+  return enc(m, type, rank, const_cast<void*>(base), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Token extents are kv_len (not the capacity), so boxes that run past the
+// last token arrive zero-filled.
+bool build_maps(octo::TmaDesc& tm, const octo_layout* L, int64_t heads, int64_t kv_len, int64_t cap,
+                const uint32_t* packed, const float* gamma, const uint32_t* qjl_bits, const float* qjl_norm,
+                const void* V) {
+  std::memset(&tm, 0, sizeof(tm));
+  const cuuint64_t kv = static_cast<cuuint64_t>(kv_len), H = static_cast<cuuint64_t>(heads);
+  const cuuint64_t row = static_cast<cuuint64_t>(cap) * 4;  // bytes between token rows of a plane
+  const cuuint32_t KW = 16;
+  const int W = L->words, QW = L->d / 32, D = L->d;
+  {
+    const cuuint64_t dims[3] = {kv, static_cast<cuuint64_t>(W), H}, str[2] = {row, row * W};
+    const cuuint32_t box[3] = {KW, static_cast<cuuint32_t>(W), 1};
+    if (!make_map(&tm.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, packed, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  {
+    const cuuint64_t dims[2] = {kv, H}, str[1] = {row};
+    const cuuint32_t box[2] = {KW, 1};
+    if (!make_map(&tm.gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, gamma, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+    if (L->qjl &&
+        !make_map(&tm.qnorm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, qjl_norm, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  if (L->qjl) {
+    const cuuint64_t dims[3] = {kv, static_cast<cuuint64_t>(QW), H}, str[2] = {row, row * QW};
+    const cuuint32_t box[3] = {KW, static_cast<cuuint32_t>(QW), 1};
+    if (!make_map(&tm.qbits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, qjl_bits, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  if (V) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), kv, H};
+    const cuuint64_t str[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(cap) * D * 2};
+    const cuuint32_t box[3] = {64, KW, 1};
+    if (!make_map(&tm.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  return true;
+}
+
 }  // namespace
 
 extern "C" size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq, int Hkv, int Lq, int64_t kv_len) {
@@ -109,6 +178,7 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   const int g = Hq / Hkv, Gq = g * Lq;
   if (Gq > 8) return OCTO_EUNSUPPORTED;
   if (static_cast<int64_t>(B) * Hkv > 65535) return OCTO_EUNSUPPORTED;  // grid.y limit
+  if (kv_len > INT_MAX) return OCTO_EUNSUPPORTED;                         // 32-bit token coordinates
   const int D = L->d;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t heads = static_cast<int64_t>(B) * Hkv;
@@ -152,11 +222,17 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.part_l = reinterpret_cast<float*>(base + w.l);
   a.part_o = reinterpret_cast<float*>(base + w.o);
   const dim3 grid(static_cast<unsigned>(a.n_splits), static_cast<unsigned>(heads));
+  // tensor maps for the tensor-core kernel (codes of at most 10 bits, d <= 128)
+  octo::TmaDesc tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (D <= 128 && 3 * L->b + 1 <= 10 &&
+      !build_maps(tm, L, heads, kv_len, cache_cap, packed, gamma, qjl_bits, qjl_norm, V))
+    return OCTO_ECUDA;
   cudaError_t e;
   switch (D) {
-    case 64: e = octo::launch_decode_d64(a, L->b, G, L->qjl != 0, grid, st); break;
-    case 128: e = octo::launch_decode_d128(a, L->b, G, L->qjl != 0, grid, st); break;
-    default: e = octo::launch_decode_d256(a, L->b, G, L->qjl != 0, grid, st); break;
+    case 64: e = octo::launch_decode_d64(a, tm, L->b, G, L->qjl != 0, grid, st); break;
+    case 128: e = octo::launch_decode_d128(a, tm, L->b, G, L->qjl != 0, grid, st); break;
+    default: e = octo::launch_decode_d256(a, tm, L->b, G, L->qjl != 0, grid, st); break;
   }
   return e == cudaSuccess ? OCTO_OK : OCTO_ECUDA;
 }

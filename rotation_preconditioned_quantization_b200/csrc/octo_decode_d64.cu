@@ -3,8 +3,8 @@
 
 namespace octo {
 
-cudaError_t launch_decode_d64(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st) {
-  return launch_decode_d<64>(a, b, G, qjl, grid, st);
+cudaError_t launch_decode_d64(const DecodeArgs& a, const TmaDesc& tm, int b, int G, bool qjl, dim3 grid, cudaStream_t st) {
+  return launch_decode_d<64>(a, tm, b, G, qjl, grid, st);
 }
 
 }  // namespace octo

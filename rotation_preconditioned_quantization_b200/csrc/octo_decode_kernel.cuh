@@ -41,6 +41,7 @@
 //    OCTO_DEVICE_TIMEOUT in the workspace status word and returns.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -704,17 +705,62 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 //
 // For a GQA group the logits of a tile of keys are a dense contraction,
 // logits[key][row] = sum_c u_hat[key][c] q_rot[row][c], so they run on
-// mma.sync m16n8k16 bf16 with keys as M, query rows as N (padded to 8) and
-// rotated coordinates as K. Each 16-wide k-step holds 4 triplets: lane
-// column c4 carries triplet 4s + c4 as (x, y | z, 0), so a lane decodes one
-// triplet code per key per k-step. The shared-memory table stores every
-// decoded triplet rho_hat * n_hat already split into bf16 hi + lo halves, in
-// exactly the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); the
-// rotated queries are B fragments held in registers for the whole CTA.
-// Three products (hi.hi + hi.lo + lo.hi) keep about 16 mantissa bits, well
-// inside the logit tolerance. With OCTOPUS-QJL the sketch term is a second
-// contraction of the +-1 sign bits against p = S q_rot, on the same units.
+// mma.sync m16n8k16 bf16 with keys as M, query rows as N and rotated
+// coordinates as K. Each 16-wide k-step holds 4 triplets: lane column c4
+// carries triplet 4s + c4 as (x, y | z, 0), so a lane decodes one triplet
+// code per key per k-step. The shared-memory table stores every decoded
+// triplet rho_hat * n_hat already split into bf16 hi + lo halves, in exactly
+// the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); the rotated
+// queries are B fragments held in registers for the whole CTA.
+//
+// Precision: with at most 4 query rows (HL layout) the 8 MMA columns hold the
+// rows' bf16 hi halves (columns 0-3) and lo halves (columns 4-7), so two
+// products (A_hi B, A_lo B) give all four hi/lo cross terms and a lane adds
+// its column n and n + 4 (lane c4 and c4 ^ 2) at the end. With 8 rows the
+// columns are all taken and three products (hi.hi + hi.lo + lo.hi) are
+// used. Either way the logits keep about 16 mantissa bits, well inside the
+// logit tolerance. P.V uses the same layouts with P split into hi + lo.
+//
+// Memory pipeline: every warp works through its own 16-key chunks with no
+// block barrier in the main loop. A chunk's code words, gammas (and sketch
+// words and norms) and its V rows arrive by tensor copies (TMA: 4 to 6 per
+// chunk, completion counted on one mbarrier per slot) into one of two
+// shared-memory slots of the warp; L2 prefetches run PF chunks further
+// ahead. The load/store unit then only serves shared-memory reads: no global
+// load of the main loop queues in front of the table lookups. V arrives with
+// the 128-byte swizzle, so the fragment reads are free of bank conflicts.
 // ---------------------------------------------------------------------------
+#ifndef OCTO_DECODE_TC_PF
+#define OCTO_DECODE_TC_PF 4   // chunks a warp prefetches into L2 ahead of its slot copies
+#endif
+
+// Tensor maps of one decode call (built on the host; token extents are
+// kv_len, so rows past the end arrive as zeros).
+struct TmaDesc {
+  CUtensorMap v;      // bf16 [heads][kv_len][D], box 64 x 16 keys, 128-byte swizzle
+  CUtensorMap codes;  // u32 [heads][W][kv_len], box 16 keys x W
+  CUtensorMap gamma;  // f32 [heads][kv_len], box 16
+  CUtensorMap qbits;  // u32 [heads][D/32][kv_len], box 16 x D/32 (OCTOPUS-QJL)
+  CUtensorMap qnorm;  // f32 [heads][kv_len], box 16 (OCTOPUS-QJL)
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
 template <int D, int B, int G, bool QJL>
 struct TcCfg {
   static constexpr int T = (D + 2) / 3;
@@ -725,31 +771,42 @@ struct TcCfg {
   static constexpr int NE = 1 << C;          // full-code table
   static constexpr int REP = 8;              // replicas (distinct bank groups per quarter-warp)
   static constexpr int NKS = (T + 3) / 4;    // logit k-steps (4 triplets each)
-  static constexpr int KW = 64;              // keys per chunk
-  static constexpr int MTL = KW / 16;        // m-tiles per chunk
-  static constexpr int SW = KW + 8;          // padded row stride of a staged chunk (words)
+  static constexpr bool HL = G <= 4;         // hi and lo halves side by side in the MMA columns
+  static constexpr int NB = HL ? 2 : 4;      // query B-fragment registers per k-step
+  static constexpr int KW = 16;              // keys per warp chunk (one m-tile)
   static constexpr int QW = D / 32;          // sketch words per key
   static constexpr int QKS = D / 16;         // sketch k-steps
   static constexpr int NWARP = 8, THREADS = 256;
-  static constexpr int ROWS = W + 1 + (QJL ? QW + 1 : 0);
-  static constexpr size_t CHUNK = sizeof(uint32_t) * ROWS * SW;
-  static constexpr int PS = KW + 8;          // P row stride (floats)
+  static constexpr int NSLOT = 2;
+  static constexpr int PF = OCTO_DECODE_TC_PF;
   static constexpr int MT = D / 16, NCH = D / 64;
+  // a slot's V: NCH swizzled boxes of 16 keys x 128 bytes
+  static constexpr int VBOX = KW * 128;
+  static constexpr int VBYTES = NCH * VBOX;
+  // a slot's rows: code words [W][KW], gammas, sketch words [QW][KW], norms
+  // (each part 128-byte aligned for the tensor copies)
+  static constexpr int G_OFF = (4 * W * KW + 127) / 128 * 128;
+  static constexpr int Q_OFF = G_OFF + 128;
+  static constexpr int N_OFF = Q_OFF + (4 * QW * KW + 127) / 128 * 128;
+  static constexpr int CODES = QJL ? N_OFF + 128 : G_OFF + 128;
+  static constexpr uint32_t TX_CODES = 4u * W * KW + 4u * KW + (QJL ? 4u * QW * KW + 4u * KW : 0u);
+  static constexpr int PS = KW + 8;          // P row stride (floats)
   static constexpr size_t TABLE = sizeof(uint4) * NE * REP;
   static constexpr size_t QROW = (12 * NKS > D + 4 ? 12 * NKS : D + 4);  // padded rotated query row
   static constexpr size_t SCRATCH = (sizeof(float) * G * (QROW + (QJL ? D : 0)) + 15) / 16 * 16;
   static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per warp
-  static constexpr size_t cmax(size_t x, size_t y) { return x > y ? x : y; }
-  static constexpr size_t ring_bytes(int ns) {
-    return (cmax(cmax(ns * CHUNK, sizeof(float) * G * (D + 2)), sizeof(float) * G * 1024 / 8) + 127) / 128 * 128;
-  }
-  static constexpr size_t FIXED = TABLE + SCRATCH;
+  // offsets from a 1024-byte aligned base
+  static constexpr size_t VREG = 0;                                   // [NWARP][NSLOT] V
+  static constexpr size_t CREG = VREG + size_t(NWARP) * NSLOT * VBYTES;  // [NWARP][NSLOT] rows
+  static constexpr size_t PREG = CREG + size_t(NWARP) * NSLOT * CODES;   // [NWARP] P
+  static constexpr size_t TREG = PREG + NWARP * PBUF;                 // table
+  static constexpr size_t SREG = TREG + TABLE;                        // query scratch
   static constexpr size_t BUDGET = 227 * 1024 - 2048;
-  static constexpr int NS = FIXED + NWARP * (PBUF + ring_bytes(2)) <= BUDGET ? 2 : 1;
-  static constexpr size_t RING = ring_bytes(NS);
-  static constexpr size_t SMEM = FIXED + NWARP * (PBUF + RING);
-  static_assert(SMEM <= BUDGET, "shared memory budget");
-  static_assert(G <= 8 && D <= 128, "tensor-core logits shape");
+  static constexpr size_t SMEM = SREG + SCRATCH + 1024;               // + alignment slack
+  static constexpr bool FITS = SMEM <= BUDGET;
+  static_assert(G <= 8 && D <= 128 && NCH >= 1, "tensor-core logits shape");
+  static_assert(VBYTES % 1024 == 0 && CODES % 128 == 0 && PBUF % 16 == 0, "alignment of the slots");
+  static_assert(NSLOT * VBYTES >= static_cast<int>(sizeof(float)) * G * (D + 2), "the warp merge reuses the V slots");
 };
 
 __device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi) {
@@ -758,21 +815,26 @@ __device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi)
 }
 
 template <int D, int B, int G, bool QJL>
-__global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const __grid_constant__ TmaDesc tm) {
   using Cfg = TcCfg<D, B, G, QJL>;
+  static_assert(Cfg::FITS, "shared memory budget");
   constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, BD = Cfg::BD, NDIR = Cfg::NDIR;
   constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, QW = Cfg::QW, NKS = Cfg::NKS;
-  constexpr int KW = Cfg::KW, MTL = Cfg::MTL, SW = Cfg::SW, NS = Cfg::NS, ROWS = Cfg::ROWS;
-  constexpr int PS = Cfg::PS, MT = Cfg::MT, NCH = Cfg::NCH, QKS = Cfg::QKS;
+  constexpr int KW = Cfg::KW, NSLOT = Cfg::NSLOT, PF = Cfg::PF;
+  constexpr int PS = Cfg::PS, MT = Cfg::MT, NCH = Cfg::NCH, QKS = Cfg::QKS, NB = Cfg::NB;
+  constexpr bool HL = Cfg::HL;
   constexpr int QROW = static_cast<int>(Cfg::QROW);
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  uint4* table = reinterpret_cast<uint4*>(smem_raw);                                     // [NE][REP]
-  float* scratch = reinterpret_cast<float*>(smem_raw + Cfg::TABLE);                      // [G][QROW] (+ [G][D])
-  unsigned char* per_warp = smem_raw + Cfg::FIXED;                                       // [NWARP] x (PBUF + RING)
+  // 1024-byte aligned base: the swizzled V boxes follow the address bits
+  unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint4* table = reinterpret_cast<uint4*>(base + Cfg::TREG);        // [NE][REP]
+  float* scratch = reinterpret_cast<float*>(base + Cfg::SREG);      // [G][QROW] (+ [G][D])
+  __shared__ __align__(8) uint64_t full[NWARP][NSLOT];
   __shared__ float s_rho_c[8];
   __shared__ float s_dir_c[32];
   __shared__ int s_last;
+  __shared__ int s_abort;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g8 = lane >> 2, c4 = lane & 3;
@@ -784,50 +846,58 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
 
   const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
   const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
-  const int n_chunks = static_cast<int>((k_end - k_begin + KW - 1) / KW);
+  // chunks of KW keys, dealt to warps round-robin: warp w takes chunks w, w + NWARP, ...
+  const int n_chunks = k_end > k_begin ? static_cast<int>((k_end - k_begin + KW - 1) / KW) : 0;
   const int my_chunks = warp < n_chunks ? (n_chunks - warp + NWARP - 1) / NWARP : 0;
-  const uint32_t* pk = a.packed + static_cast<int64_t>(bh) * W * a.cache_cap;
   const float* gm = a.gamma + static_cast<int64_t>(bh) * a.cache_cap;
   const __nv_bfloat16* Vh = with_v ? a.V + static_cast<int64_t>(bh) * a.cache_cap * D : nullptr;
-  const uint32_t* qbp = QJL ? a.qjl_bits + static_cast<int64_t>(bh) * QW * a.cache_cap : nullptr;
-  const float* qnp = QJL ? a.qjl_norm + static_cast<int64_t>(bh) * a.cache_cap : nullptr;
-  float* pw = reinterpret_cast<float*>(per_warp + warp * (Cfg::PBUF + Cfg::RING));                  // [G][PS]
-  uint32_t* ring = reinterpret_cast<uint32_t*>(per_warp + warp * (Cfg::PBUF + Cfg::RING) + Cfg::PBUF);  // [NS][ROWS][SW]
+  float* pw = reinterpret_cast<float*>(base + Cfg::PREG + warp * Cfg::PBUF);  // [G][PS]
+  auto slot_codes = [&](int s) {
+    return reinterpret_cast<uint32_t*>(base + Cfg::CREG + (warp * NSLOT + s) * Cfg::CODES);
+  };
+  auto slot_v = [&](int s) { return base + Cfg::VREG + (warp * NSLOT + s) * Cfg::VBYTES; };
 
-  // Chunk i of this warp (keys k_begin + (warp + NWARP i) KW ...): the lanes
-  // copy its rows (code words, gammas, sketch words, norms) into ring slot
-  // i % NS with 16-byte cp.async copies (one commit group per chunk), and
-  // prefetch its V rows into L2. Keys are copied in groups of 4; the cache
-  // capacity is a multiple of 4 and chunks start at multiples of KW, so the
-  // rounded-up copy stays inside the cache rows (keys past kv_len are masked).
+  auto chunk_start = [&](int i) { return k_begin + static_cast<int64_t>(warp + NWARP * i) * KW; };
+  auto chunk_len = [&](int64_t s0) { return static_cast<int>(k_end - s0 < KW ? k_end - s0 : KW); };
+  // This warp's i-th chunk into slot i % NSLOT: lane 0 arms the slot's
+  // barrier with the byte count of the boxes (tokens past kv_len arrive as
+  // zeros and count too) and issues the tensor copies: code words, gammas
+  // (sketch words, norms) and the NCH swizzled V boxes.
   auto issue_chunk = [&](int i) {
-    const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * i) * KW;
-    const int n = static_cast<int>(k_end - s0 < KW ? k_end - s0 : KW);
-    const int groups = (n + 3) >> 2;
-    uint32_t* buf = ring + (i % NS) * ROWS * SW;
-    for (int p = lane; p < ROWS * (KW / 4); p += 32) {
-      const int r = p / (KW / 4), c = p - r * (KW / 4);
-      if (c >= groups) continue;
-      const void* src;
-      if (r < W) src = pk + r * a.cache_cap + s0 + 4 * c;
-      else if (r == W) src = gm + s0 + 4 * c;
-      else if (QJL && r < W + 1 + QW) src = qbp + (r - W - 1) * a.cache_cap + s0 + 4 * c;
-      else src = qnp + s0 + 4 * c;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(buf + r * SW + 4 * c)), "l"(src)
-                   : "memory");
+    if (lane != 0) return;
+    const int x = static_cast<int>(chunk_start(i));
+    const int s = i % NSLOT;
+    uint64_t* bar = &full[warp][s];
+    unsigned char* rows = reinterpret_cast<unsigned char*>(slot_codes(s));
+    mbar_expect_tx(bar, Cfg::TX_CODES + (with_v ? static_cast<uint32_t>(Cfg::VBYTES) : 0u));
+    tma_load_3d(rows, &tm.codes, x, 0, bh, bar);
+    tma_load_2d(rows + Cfg::G_OFF, &tm.gamma, x, bh, bar);
+    if constexpr (QJL) {
+      tma_load_3d(rows + Cfg::Q_OFF, &tm.qbits, x, 0, bh, bar);
+      tma_load_2d(rows + Cfg::N_OFF, &tm.qnorm, x, bh, bar);
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
     if (with_v) {
-      const char* v0 = reinterpret_cast<const char*>(Vh + s0 * D);
-      for (int64_t off = static_cast<int64_t>(lane) * 128; off < static_cast<int64_t>(n) * D * 2; off += 32 * 128)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(v0 + off));
+#pragma unroll
+      for (int hh = 0; hh < NCH; ++hh) tma_load_3d(slot_v(s) + hh * Cfg::VBOX, &tm.v, 64 * hh, x, bh, bar);
     }
   };
-  // small global reads first (codebooks, one sign-flipped query row per warp)
+  // Chunk i's rows and V into L2 ahead of its slot copies.
+  auto prefetch_chunk = [&](int i) {
+    if (lane != 0 || i >= my_chunks) return;
+    const int64_t s0 = chunk_start(i);
+    const int n = chunk_len(s0);
+    tma_prefetch_3d(&tm.codes, static_cast<int>(s0), 0, bh);
+    bulk_prefetch_l2(gm + s0, static_cast<uint32_t>(((n + 3) & ~3) * 4));
+    if constexpr (QJL) tma_prefetch_3d(&tm.qbits, static_cast<int>(s0), 0, bh);
+    if (with_v) bulk_prefetch_l2(Vh + s0 * D, static_cast<uint32_t>(n) * 2u * D);
+  };
+
+  // The small global reads (codebooks, one sign-flipped query row per warp)
+  // are issued first, ahead of the bulk copies in the memory queues.
   constexpr int E = D / 32;
   float qraw[E];
-  if (tid < NDIR) s_dir_c[tid] = a.dir_c[tid];
-  if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
+  const float dir_v = tid < NDIR ? __ldg(a.dir_c + tid) : 0.0f;
+  const float rho_v = tid < Cfg::NRHO ? __ldg(a.rho_c + tid) : 0.0f;
   if (warp < G && warp < a.Gq) {
     const int gi = warp / a.Lq, lq = warp - gi * a.Lq;
     const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
@@ -842,7 +912,16 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
 #pragma unroll
     for (int e = 0; e < E; ++e) qraw[e] = 0.0f;
   }
-  for (int i = 0; i < NS && i < my_chunks; ++i) issue_chunk(i);
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < NSLOT; ++s) mbar_init(&full[warp][s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (tid == 0) s_abort = 0;
+  for (int i = 0; i < NSLOT && i < my_chunks; ++i) issue_chunk(i);
+  for (int i = NSLOT; i < NSLOT + PF; ++i) prefetch_chunk(i);
+  if (tid < NDIR) s_dir_c[tid] = dir_v;
+  if (tid < Cfg::NRHO) s_rho_c[tid] = rho_v;
   __syncthreads();
 
   // ------------------------------------------------ prologue (overlaps the first copies)
@@ -883,218 +962,220 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
     __syncthreads();
   }
 
-  // B fragments of the rotated queries (row g8, triplet 4s + c4 as (x, y | z, 0)), hi and lo
-  uint32_t bq[NKS][4];
+  // B fragments of the rotated queries: triplet 4s + c4 as (x, y | z, 0) of
+  // MMA column g8, i.e. query row g8 & 3, lo half for g8 >= 4 (HL), or row
+  // g8 with separate hi and lo registers (8 rows)
+  const int brow = HL ? (g8 & 3) : g8;
+  const bool blo = HL && g8 >= 4;
+  uint32_t bq[NKS][NB];
 #pragma unroll
   for (int s = 0; s < NKS; ++s) {
     const int t = 4 * s + c4;
     float x = 0.0f, y = 0.0f, z = 0.0f;
-    if (g8 < G) {
-      const float* qrow = scratch + g8 * QROW;
+    if (brow < G) {
+      const float* qrow = scratch + brow * QROW;
       x = qrow[3 * t]; y = qrow[3 * t + 1]; z = qrow[3 * t + 2];
     }
-    split_bf16x2(x, y, bq[s][0], bq[s][2]);
-    split_bf16x2(z, 0.0f, bq[s][1], bq[s][3]);
+    uint32_t xyh, xyl, zh, zl;
+    split_bf16x2(x, y, xyh, xyl);
+    split_bf16x2(z, 0.0f, zh, zl);
+    if constexpr (HL) {
+      bq[s][0] = blo ? xyl : xyh;
+      bq[s][1] = blo ? zl : zh;
+    } else {
+      bq[s][0] = xyh; bq[s][1] = zh; bq[s][NB - 2] = xyl; bq[s][NB - 1] = zl;
+    }
   }
-  // sketch B fragments: p row g8, sketch coordinates 16 ks + {2c4, 2c4+1 | 2c4+8, 2c4+9}
-  uint32_t bp[QJL ? QKS : 1][4];
+  // sketch B fragments: p row, sketch coordinates 16 ks + {2c4, 2c4+1 | 2c4+8, 2c4+9}
+  uint32_t bp[QJL ? QKS : 1][NB];
   if constexpr (QJL) {
 #pragma unroll
     for (int ks = 0; ks < QKS; ++ks) {
       float p0 = 0.0f, p1 = 0.0f, p8 = 0.0f, p9 = 0.0f;
-      if (g8 < G) {
-        const float* prow = scratch + G * QROW + g8 * D + 16 * ks + 2 * c4;
+      if (brow < G) {
+        const float* prow = scratch + G * QROW + brow * D + 16 * ks + 2 * c4;
         p0 = prow[0]; p1 = prow[1]; p8 = prow[8]; p9 = prow[9];
       }
-      split_bf16x2(p0, p1, bp[ks][0], bp[ks][2]);
-      split_bf16x2(p8, p9, bp[ks][1], bp[ks][3]);
+      uint32_t h01, l01, h89, l89;
+      split_bf16x2(p0, p1, h01, l01);
+      split_bf16x2(p8, p9, h89, l89);
+      if constexpr (HL) {
+        bp[ks][0] = blo ? l01 : h01;
+        bp[ks][1] = blo ? l89 : h89;
+      } else {
+        bp[ks][0] = h01; bp[ks][1] = h89; bp[ks][NB - 2] = l01; bp[ks][NB - 1] = l89;
+      }
     }
   }
   // where this lane's triplet code of each k-step sits in a key's bit stream
-  uint32_t cpos[NKS];  // word << 8 | shift, or 0xFFFF for padding triplets
+  // (word << 8 | shift). A padding triplet (t >= T) reads code 0's position:
+  // its query coordinates are zero, so whatever entry it finds adds nothing.
+  uint32_t cpos[NKS];
 #pragma unroll
   for (int s = 0; s < NKS; ++s) {
     const int t = 4 * s + c4;
-    cpos[s] = t < T ? (static_cast<uint32_t>((t * C) >> 5) << 8) | static_cast<uint32_t>((t * C) & 31) : 0xFFFFu;
+    cpos[s] = t < T ? (static_cast<uint32_t>((t * C) >> 5) << 8) | static_cast<uint32_t>((t * C) & 31) : 0u;
   }
   const int rep_off = lane & (REP - 1);
 
   // ------------------------------------------------ main loop: this warp's chunks
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // this lane's query columns 2c4, 2c4+1
+  // This lane's query columns: HL lanes c4 and c4 ^ 2 hold the same two rows
+  // (hi and lo columns before the pairwise add), 8-row lanes rows 2c4, 2c4+1.
+  const int q0 = HL ? 2 * (c4 & 1) : 2 * c4, q1 = q0 + 1;
+  const bool owner = !HL || c4 < 2;  // writes this lane's columns (the HL mirror lanes do not)
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
   float acc_o[MT][4];
 #pragma unroll
   for (int t = 0; t < MT; ++t) acc_o[t][0] = acc_o[t][1] = acc_o[t][2] = acc_o[t][3] = 0.0f;
-#ifndef OCTO_DECODE_TC_VALL
-#define OCTO_DECODE_TC_VALL 0  // 1: load all of a chunk's V fragments before its logits (spills at d = 128)
-#endif
-  constexpr bool VALL = OCTO_DECODE_TC_VALL && NCH <= 2 && !QJL;  // (the sketch fragments need the registers)
-  constexpr bool VPIPE = !VALL && NCH <= 2;
-  auto load_v_step = [&](uint4 (&dst)[4][NCH], int64_t s0v, int j) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int64_t vk = s0v + 16 * j + 2 * c4 + (kk & 1) + 8 * (kk >> 1);
-#pragma unroll
-      for (int hh = 0; hh < NCH; ++hh)
-        dst[kk][hh] = vk < k_end ? __ldg(reinterpret_cast<const uint4*>(Vh + vk * D + 64 * hh + 8 * g8))
-                                 : make_uint4(0u, 0u, 0u, 0u);
-    }
-  };
-  uint4 vcur[4][NCH], vnext[4][NCH];
-  uint4 vall[VALL ? KW / 16 : 1][4][NCH];
-  const bool q0_real = 2 * c4 < a.Gq, q1_real = 2 * c4 + 1 < a.Gq;
-  for (int ci = 0; ci < my_chunks; ++ci) {
-    const uint32_t* buf = ring + (ci % NS) * ROWS * SW;
-    const int64_t s0 = k_begin + static_cast<int64_t>(warp + NWARP * ci) * KW;
-    if constexpr (VALL) {
-      if (with_v) {  // in flight during the wait and the logits
-#pragma unroll
-        for (int j = 0; j < KW / 16; ++j) load_v_step(vall[j], s0, j);
-      }
-    } else {
-      if (VPIPE && with_v) load_v_step(vcur, s0, 0);  // in flight during the wait and the logits
-    }
-    // this lane's copies of chunk ci are complete (later chunks may still be in
-    // flight), then the warp's: everyone's rows are visible after the syncwarp
-    if (ci + 1 < my_chunks && NS > 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncwarp();
+  int aborted_at = -1;
 
-    // logits of the chunk in C-fragment layout: lgv[mt] = (kA, q0), (kA, q1), (kB, q0), (kB, q1)
-    float lgv[MTL][4];
+  for (int ci = 0; ci < my_chunks; ++ci) {
+    const int slot = ci % NSLOT;
+    const uint32_t* buf = slot_codes(slot);
+    const unsigned char* vbuf = slot_v(slot);
+    const int64_t s0 = chunk_start(ci);
+    prefetch_chunk(ci + NSLOT + PF);
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[warp][slot], (ci / NSLOT) & 1))) {
+      aborted_at = ci;  // warp-uniform
+      break;
+    }
+
+    // Logits of the chunk in C-fragment layout. Rows are permuted so that a
+    // lane owns 2 consecutive keys: row g8 is key 2 g8, row g8 + 8 is key
+    // 2 g8 + 1; one 8-byte load gives a code word (or gamma, or sketch word)
+    // of both. lgv = (key 2g8, q0), (same, q1), (key 2g8+1, q0), (same, q1).
+    float lgv[4];
+    {
+      constexpr int NC = HL ? 2 : 3;  // independent accumulator chains
+      float acc[NC][4];
 #pragma unroll
-    for (int mt = 0; mt < MTL; ++mt) {
-      const int kA = 16 * mt + g8, kB = kA + 8;
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+      const uint32_t* bk = buf + 2 * g8;  // this lane's 2 keys in row 0
 #pragma unroll
       for (int s = 0; s < NKS; ++s) {
-        uint4 eA = make_uint4(0u, 0u, 0u, 0u), eB = eA;
-        if (cpos[s] != 0xFFFFu) {
-          const int wi = static_cast<int>(cpos[s] >> 8), sh = static_cast<int>(cpos[s] & 31u);
-          const uint32_t* rw = buf + wi * SW;
-          const uint32_t hiA = wi + 1 < W ? rw[SW + kA] : 0u, hiB = wi + 1 < W ? rw[SW + kB] : 0u;
-          const uint32_t cA = __funnelshift_r(rw[kA], hiA, sh) & ((1u << C) - 1u);
-          const uint32_t cB = __funnelshift_r(rw[kB], hiB, sh) & ((1u << C) - 1u);
-          eA = table[cA * REP + rep_off];
-          eB = table[cB * REP + rep_off];
+        // the code may straddle words wi and wi + 1; for the last word the
+        // next row (gamma or padding) supplies bits that the mask drops
+        const int wi = static_cast<int>(cpos[s] >> 8), sh = static_cast<int>(cpos[s] & 31u);
+        const uint2 lo = *reinterpret_cast<const uint2*>(bk + wi * KW);
+        const uint2 hi = *reinterpret_cast<const uint2*>(bk + (wi + 1) * KW);
+        const uint32_t cm = (1u << C) - 1u;
+        const uint4 eA = table[(__funnelshift_r(lo.x, hi.x, sh) & cm) * REP + rep_off];
+        const uint4 eB = table[(__funnelshift_r(lo.y, hi.y, sh) & cm) * REP + rep_off];
+        if constexpr (HL) {
+          mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
+          mma_bf16_16816(acc[1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
+        } else {
+          mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
+          mma_bf16_16816(acc[1], eA.x, eB.x, eA.y, eB.y, bq[s][NB - 2], bq[s][NB - 1]);
+          mma_bf16_16816(acc[NC - 1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
         }
-        mma_bf16_16816(acc, eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
-        mma_bf16_16816(acc, eA.x, eB.x, eA.y, eB.y, bq[s][2], bq[s][3]);
-        mma_bf16_16816(acc, eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
       }
-      const float gA = __uint_as_float(buf[W * SW + kA]), gB = __uint_as_float(buf[W * SW + kB]);
+      float v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[i] = acc[0][i] + acc[1][i];
+        if constexpr (!HL) v[i] += acc[NC - 1][i];
+      }
       if constexpr (QJL) {
         float accq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int ks = 0; ks < QKS; ++ks) {
-          const uint32_t wA = buf[(W + 1 + (ks >> 1)) * SW + kA] >> (16 * (ks & 1) + 2 * c4);
-          const uint32_t wB = buf[(W + 1 + (ks >> 1)) * SW + kB] >> (16 * (ks & 1) + 2 * c4);
+          const uint2 w2 = *reinterpret_cast<const uint2*>(bk + Cfg::Q_OFF / 4 + (ks >> 1) * KW);
+          const int shq = 16 * (ks & 1) + 2 * c4;
+          const uint32_t wA = w2.x >> shq, wB = w2.y >> shq;
           const uint32_t a0 = pm1_bf16x2(wA, wA >> 1), a1 = pm1_bf16x2(wB, wB >> 1);
           const uint32_t a2 = pm1_bf16x2(wA >> 8, wA >> 9), a3 = pm1_bf16x2(wB >> 8, wB >> 9);
           mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
-          mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][2], bp[ks][3]);
+          if constexpr (!HL) mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
         }
         const float kq = 1.2533141373155003f / static_cast<float>(D);  // sqrt(pi/2)/m, m = d
-        const float fA = kq * __uint_as_float(buf[(W + 1 + QW) * SW + kA]);
-        const float fB = kq * __uint_as_float(buf[(W + 1 + QW) * SW + kB]);
-        acc[0] = fmaf(fA, accq[0], acc[0]); acc[1] = fmaf(fA, accq[1], acc[1]);
-        acc[2] = fmaf(fB, accq[2], acc[2]); acc[3] = fmaf(fB, accq[3], acc[3]);
+        const uint2 nu = *reinterpret_cast<const uint2*>(bk + Cfg::N_OFF / 4);
+        const float fA = kq * __uint_as_float(nu.x), fB = kq * __uint_as_float(nu.y);
+        v[0] = fmaf(fA, accq[0], v[0]); v[1] = fmaf(fA, accq[1], v[1]);
+        v[2] = fmaf(fB, accq[2], v[2]); v[3] = fmaf(fB, accq[3], v[3]);
       }
-      lgv[mt][0] = acc[0] * gA; lgv[mt][1] = acc[1] * gA;
-      lgv[mt][2] = acc[2] * gB; lgv[mt][3] = acc[3] * gB;
+      if constexpr (HL) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);  // hi column + lo column
+      }
+      const uint2 g2 = *reinterpret_cast<const uint2*>(bk + Cfg::G_OFF / 4);
+      const float gA = __uint_as_float(g2.x), gB = __uint_as_float(g2.y);
+      lgv[0] = v[0] * gA; lgv[1] = v[1] * gA;
+      lgv[2] = v[2] * gB; lgv[3] = v[3] * gB;
     }
-    // this warp is done with the chunk's rows: refill the slot with chunk ci + NS
-    __syncwarp();
-    if (ci + NS < my_chunks) issue_chunk(ci + NS);
 
-    if (a.logits != nullptr) {
+    const int64_t kown = s0 + 2 * g8;  // lgv[2h + qq] is key kown + h
+    if (a.logits != nullptr && owner) {
 #pragma unroll
-      for (int mt = 0; mt < MTL; ++mt) {
+      for (int h = 0; h < 2; ++h) {
+        const int64_t key = kown + h;
+        if (key >= k_end) continue;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t key = s0 + 16 * mt + g8 + 8 * h;
-          if (key >= k_end) continue;
-#pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const int r = 2 * c4 + qq;
-            if (r < a.Gq) {
-              const int gi = r / a.Lq, lq = r - gi * a.Lq;
-              const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-              a.logits[row * a.kv_len + key] = lgv[mt][2 * h + qq];
-            }
+        for (int qq = 0; qq < 2; ++qq) {
+          const int r = q0 + qq;
+          if (r < a.Gq) {
+            const int gi = r / a.Lq, lq = r - gi * a.Lq;
+            const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
+            a.logits[row * a.kv_len + key] = lgv[2 * h + qq];
           }
         }
       }
     }
-    if (!with_v) continue;
-
-    // online softmax over the chunk, base 2, per query column; keys live on the g8 lanes
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    if (with_v) {
+      // online softmax over the chunk, base 2, per query column; keys live on the g8 lanes
+      const bool vA = kown < k_end, vB = kown + 1 < k_end;
+      lgv[0] = vA ? lgv[0] * a.scale_log2 : -INFINITY;
+      lgv[1] = vA ? lgv[1] * a.scale_log2 : -INFINITY;
+      lgv[2] = vB ? lgv[2] * a.scale_log2 : -INFINITY;
+      lgv[3] = vB ? lgv[3] * a.scale_log2 : -INFINITY;
+      float mx0 = fmaxf(lgv[0], lgv[2]), mx1 = fmaxf(lgv[1], lgv[3]);
 #pragma unroll
-    for (int mt = 0; mt < MTL; ++mt) {
-      const bool vA = s0 + 16 * mt + g8 < k_end, vB = s0 + 16 * mt + g8 + 8 < k_end;
-      lgv[mt][0] = vA ? lgv[mt][0] * a.scale_log2 : -INFINITY;
-      lgv[mt][1] = vA ? lgv[mt][1] * a.scale_log2 : -INFINITY;
-      lgv[mt][2] = vB ? lgv[mt][2] * a.scale_log2 : -INFINITY;
-      lgv[mt][3] = vB ? lgv[mt][3] * a.scale_log2 : -INFINITY;
-      mx0 = fmaxf(mx0, fmaxf(lgv[mt][0], lgv[mt][2]));
-      mx1 = fmaxf(mx1, fmaxf(lgv[mt][1], lgv[mt][3]));
-    }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-    const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
-    m0 = n0; m1 = n1;
-    float ps0 = 0.0f, ps1 = 0.0f;
-#pragma unroll
-    for (int mt = 0; mt < MTL; ++mt) {
-      lgv[mt][0] = fast_exp2(lgv[mt][0] - n0); lgv[mt][2] = fast_exp2(lgv[mt][2] - n0);
-      lgv[mt][1] = fast_exp2(lgv[mt][1] - n1); lgv[mt][3] = fast_exp2(lgv[mt][3] - n1);
-      ps0 += lgv[mt][0] + lgv[mt][2];
-      ps1 += lgv[mt][1] + lgv[mt][3];
-    }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
-    }
-    // P rows (query-major) for the P.V B fragments
-#pragma unroll
-    for (int mt = 0; mt < MTL; ++mt) {
-      const int kA = 16 * mt + g8;
-      if (2 * c4 < G) { pw[(2 * c4) * PS + kA] = lgv[mt][0]; pw[(2 * c4) * PS + kA + 8] = lgv[mt][2]; }
-      if (2 * c4 + 1 < G) { pw[(2 * c4 + 1) * PS + kA] = lgv[mt][1]; pw[(2 * c4 + 1) * PS + kA + 8] = lgv[mt][3]; }
-    }
-    __syncwarp();
-
-    // P.V over the chunk's 16-key steps
-#pragma unroll
-    for (int j = 0; j < KW / 16; ++j) {
-      if (s0 + 16 * j >= k_end) break;  // warp-uniform
-      if constexpr (VALL) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-          for (int hh = 0; hh < NCH; ++hh) vcur[kk][hh] = vall[VALL ? j : 0][kk][hh];
-      } else if constexpr (VPIPE) {
-        if (j + 1 < KW / 16) load_v_step(vnext, s0, j + 1);  // keys past the end load as zeros
-      } else {
-        load_v_step(vcur, s0, j);
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
-      uint32_t bh0 = 0, bl0 = 0, bh1 = 0, bl1 = 0;
-      if (g8 < G) {
-        const float* prow = pw + g8 * PS + 16 * j + 2 * c4;
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
+      m0 = n0; m1 = n1;
+      lgv[0] = fast_exp2(lgv[0] - n0); lgv[2] = fast_exp2(lgv[2] - n0);
+      lgv[1] = fast_exp2(lgv[1] - n1); lgv[3] = fast_exp2(lgv[3] - n1);
+      l0 = l0 * al0 + lgv[0] + lgv[2];
+      l1 = l1 * al1 + lgv[1] + lgv[3];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
+      }
+      // P rows (query-major) for the P.V B fragments: this lane's 2 consecutive keys
+      if (owner) {
+        if (q0 < G) *reinterpret_cast<float2*>(pw + q0 * PS + 2 * g8) = make_float2(lgv[0], lgv[2]);
+        if (q1 < G) *reinterpret_cast<float2*>(pw + q1 * PS + 2 * g8) = make_float2(lgv[1], lgv[3]);
+      }
+      __syncwarp();
+
+      // P.V over the chunk (O^T = V^T P^T: d as M, keys as K)
+      uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;  // (hi | lo) of keys 2c4, 2c4+1 and 2c4+8, 2c4+9
+      if (brow < G) {
+        const float* prow = pw + brow * PS + 2 * c4;
         const float2 p01 = *reinterpret_cast<const float2*>(prow);
         const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
-        split_bf16x2(p01.x, p01.y, bh0, bl0);
-        split_bf16x2(p89.x, p89.y, bh1, bl1);
+        uint32_t h01, l01, h89, l89;
+        split_bf16x2(p01.x, p01.y, h01, l01);
+        split_bf16x2(p89.x, p89.y, h89, l89);
+        if constexpr (HL) {
+          b0 = blo ? l01 : h01; b1 = blo ? l89 : h89;
+        } else {
+          b0 = h01; b1 = h89; b2 = l01; b3 = l89;
+        }
       }
 #pragma unroll
       for (int hh = 0; hh < NCH; ++hh) {
-        const uint4 k0 = vcur[0][hh], k1 = vcur[1][hh], k8 = vcur[2][hh], k9 = vcur[3][hh];
+        // 8 consecutive d (64 hh + 8 g8 ...) of keys 2c4, 2c4+1, 2c4+8, 2c4+9:
+        // in the swizzled box, 16-byte unit g8 of key row k sits at unit g8 ^ (k & 7)
+        const unsigned char* vb = vbuf + hh * Cfg::VBOX;
+        auto vld = [&](int k) {
+          return *reinterpret_cast<const uint4*>(vb + k * 128 + ((g8 ^ (k & 7)) << 4));
+        };
+        const uint4 k0 = vld(2 * c4), k1 = vld(2 * c4 + 1), k8 = vld(2 * c4 + 8), k9 = vld(2 * c4 + 9);
         const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
         const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
 #pragma unroll
@@ -1103,48 +1184,58 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
           const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
           const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
           const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bh0, bh1);
-          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, bl0, bl1);
+          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b0, b1);
+          if constexpr (!HL) mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b2, b3);
         }
       }
-      if constexpr (VPIPE) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-          for (int hh = 0; hh < NCH; ++hh) vcur[kk][hh] = vnext[kk][hh];
-      }
     }
-    __syncwarp();  // P rows consumed before the next chunk overwrites them
+    // the chunk's slot (rows, V, P) is consumed: refill it with chunk ci + NSLOT
+    __syncwarp();
+    if (ci + NSLOT < my_chunks) issue_chunk(ci + NSLOT);
   }
 
-  __syncthreads();  // every ring is free: no copy is in flight after the last chunk
-  if (!with_v) return;
+  // A bounded wait that expired: record it, let this warp's copies in flight
+  // land (again bounded) before the block can exit, and skip the output.
+  if (aborted_at >= 0) {
+    if (lane == 0) {
+      atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
+      s_abort = 1;
+    }
+    for (int c = aborted_at; c < aborted_at + NSLOT && c < my_chunks; ++c)
+      mbar_wait_bounded(&full[warp][c % NSLOT], (c / NSLOT) & 1);
+  }
+  __syncthreads();  // every slot is free: no copy is in flight after the last chunk
+  if (s_abort || !with_v) return;
 
-  // ------------------------------------------------ epilogue: merge warps (in each warp's ring)
+  // ------------------------------------------------ epilogue: merge warps (in each warp's V slots)
+  if constexpr (HL) {  // hi column + lo column of every output
+#pragma unroll
+    for (int t = 0; t < MT; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc_o[t][i] += __shfl_xor_sync(0xffffffffu, acc_o[t][i], 2);
+  }
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
-  auto wbase = [&](int w) { return reinterpret_cast<float*>(per_warp + w * (Cfg::PBUF + Cfg::RING) + Cfg::PBUF); };
-  {
+  auto wbase = [&](int w) { return reinterpret_cast<float*>(base + Cfg::VREG + w * NSLOT * Cfg::VBYTES); };
+  if (owner) {
     float* wm = wbase(warp);  // [G] m, [G] l, [G][D] O
     if (g8 == 0) {
-      if (2 * c4 < G) { wm[2 * c4] = m0; wm[G + 2 * c4] = l0; }
-      if (2 * c4 + 1 < G) { wm[2 * c4 + 1] = m1; wm[G + 2 * c4 + 1] = l1; }
+      if (q0 < G) { wm[q0] = m0; wm[G + q0] = l0; }
+      if (q1 < G) { wm[q1] = m1; wm[G + q1] = l1; }
     }
     float* o = wm + 2 * G;
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
       const int hh = t >> 2, e2 = t & 3;
       const int d0 = 64 * hh + 8 * g8 + 2 * e2;
-      const int q0 = 2 * c4, q1 = 2 * c4 + 1;
       if (q0 < G) { o[q0 * D + d0] = acc_o[t][0]; o[q0 * D + d0 + 1] = acc_o[t][2]; }
       if (q1 < G) { o[q1 * D + d0] = acc_o[t][1]; o[q1 * D + d0 + 1] = acc_o[t][3]; }
     }
   }
   __syncthreads();
-  (void)q0_real; (void)q1_real;
 
   const int S = a.n_splits;
   float* pm = a.part_m + (static_cast<int64_t>(bh) * S + split) * G;
@@ -1228,22 +1319,30 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a) {
 
 // Launch one decode instantiation for head dimension D (defined in the
 // per-D translation units so that the templates compile in parallel).
-cudaError_t launch_decode_d64(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
-cudaError_t launch_decode_d128(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
-cudaError_t launch_decode_d256(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
+cudaError_t launch_decode_d64(const DecodeArgs& a, const TmaDesc& tm, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
+cudaError_t launch_decode_d128(const DecodeArgs& a, const TmaDesc& tm, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
+cudaError_t launch_decode_d256(const DecodeArgs& a, const TmaDesc& tm, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
 
 #ifndef OCTO_DECODE_TC
 #define OCTO_DECODE_TC 1  // tensor-core logits where the shape allows
 #endif
 
+// The tensor-core kernel takes codes of at most 10 bits (b <= 3), d <= 128,
+// and only shapes whose tables and slots fit in shared memory.
 template <int D, int B, int G, bool QJL>
-cudaError_t launch_decode_one(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  if constexpr (OCTO_DECODE_TC && D <= 128 && 3 * B + 1 <= 10) {
+constexpr bool tc_fits() {
+  if constexpr (D <= 128 && 3 * B + 1 <= 10) return TcCfg<D, B, G, QJL>::FITS;
+  else return false;
+}
+
+template <int D, int B, int G, bool QJL>
+cudaError_t launch_decode_one(const DecodeArgs& a, const TmaDesc& tm, dim3 grid, cudaStream_t st) {
+  if constexpr (OCTO_DECODE_TC && tc_fits<D, B, G, QJL>()) {
     using Cfg = TcCfg<D, B, G, QJL>;
     auto k = decode_tc_kernel<D, B, G, QJL>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
     if (e != cudaSuccess) return e;
-    k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a);  // grid: (splits, heads)
+    k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a, tm);  // grid: (splits, heads)
   } else {
     using Cfg = DecCfg<D, B, G, QJL>;
     auto k = decode_kernel<D, B, G, QJL>;
@@ -1255,15 +1354,15 @@ cudaError_t launch_decode_one(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
 }
 
 template <int D>
-cudaError_t launch_decode_d(const DecodeArgs& a, int b, int G, bool qjl, dim3 grid, cudaStream_t st) {
+cudaError_t launch_decode_d(const DecodeArgs& a, const TmaDesc& tm, int b, int G, bool qjl, dim3 grid, cudaStream_t st) {
 #define OCTO_G(BB)                                                                           \
   switch (G) {                                                                               \
-    case 1: return qjl ? launch_decode_one<D, BB, 1, true>(a, grid, st)                      \
-                       : launch_decode_one<D, BB, 1, false>(a, grid, st);                    \
-    case 4: return qjl ? launch_decode_one<D, BB, 4, true>(a, grid, st)                      \
-                       : launch_decode_one<D, BB, 4, false>(a, grid, st);                    \
-    default: return qjl ? launch_decode_one<D, BB, 8, true>(a, grid, st)                     \
-                        : launch_decode_one<D, BB, 8, false>(a, grid, st);                   \
+    case 1: return qjl ? launch_decode_one<D, BB, 1, true>(a, tm, grid, st)                      \
+                       : launch_decode_one<D, BB, 1, false>(a, tm, grid, st);                    \
+    case 4: return qjl ? launch_decode_one<D, BB, 4, true>(a, tm, grid, st)                      \
+                       : launch_decode_one<D, BB, 4, false>(a, tm, grid, st);                    \
+    default: return qjl ? launch_decode_one<D, BB, 8, true>(a, tm, grid, st)                     \
+                        : launch_decode_one<D, BB, 8, false>(a, tm, grid, st);                   \
   }
   switch (b) {
     case 2: OCTO_G(2)
