@@ -212,17 +212,46 @@ def exhaustive_round(t, dir_c, rho_c):
 # --------------------------------------------------------------------------
 # Bit packing (compact bit stream; layout is a reading).
 # --------------------------------------------------------------------------
-def pack(i_xi, i_eta, i_rho, lay: Layout) -> np.ndarray:
-    """[..., T] indices -> [..., W] uint32 words (LSB-first stream).
+def direction_field(i_xi, i_eta, b: int):
+    """Ordered direction cells -> the 2(b+1)-bit direction field of a code.
 
-    The code of triplet i occupies stream bits [i c, i c + c), c = 3b+1;
-    stream bit p is bit p mod 32 of word p // 32, so a code that crosses a
-    word boundary puts its low bits at the top of one word and its high
-    bits at the bottom of the next.
+    Reading: the direction codebook is odd-symmetric (c_k = -c_{L-1-k}, L =
+    2^(b+1)), so each cell index i is stored as a sign and a magnitude rank:
+    s = 1 for the lower half (i < 2^b, negative levels), m = rank of |c_i|
+    among the positive levels (m = i - 2^b above the middle, 2^b - 1 - i
+    below). Field = m_xi | m_eta << b | s_xi << 2b | s_eta << (2b + 1).
     """
-    code = (np.asarray(i_xi, dtype=np.uint64)
-            | (np.asarray(i_eta, dtype=np.uint64) << np.uint64(lay.b_dir))
-            | (np.asarray(i_rho, dtype=np.uint64) << np.uint64(2 * lay.b_dir)))
+    half = 1 << b
+    fields = []
+    for i in (np.asarray(i_xi, dtype=np.int64), np.asarray(i_eta, dtype=np.int64)):
+        s = (i < half).astype(np.int64)
+        m = np.where(i >= half, i - half, half - 1 - i)
+        fields.append((s, m))
+    (sx, mx), (sy, my) = fields
+    return (mx | (my << b) | (sx << (2 * b)) | (sy << (2 * b + 1))).astype(np.uint64)
+
+
+def direction_cells(field, b: int):
+    """Inverse of direction_field: the ordered (i_xi, i_eta) cell indices."""
+    f = np.asarray(field, dtype=np.int64)
+    half = 1 << b
+    mx, my = f & (half - 1), (f >> b) & (half - 1)
+    sx, sy = (f >> (2 * b)) & 1, (f >> (2 * b + 1)) & 1
+    i_xi = np.where(sx == 1, half - 1 - mx, half + mx)
+    i_eta = np.where(sy == 1, half - 1 - my, half + my)
+    return i_xi.astype(np.int64), i_eta.astype(np.int64)
+
+
+def pack(i_xi, i_eta, i_rho, lay: Layout) -> np.ndarray:
+    """[..., T] ordered cell indices -> [..., W] uint32 words (LSB-first stream).
+
+    Triplet code (3b+1 bits) = direction field (2(b+1) bits, see
+    direction_field) | i_rho << 2(b+1). The code of triplet i occupies
+    stream bits [i c, i c + c), c = 3b+1; stream bit p is bit p mod 32 of
+    word p // 32, so a code that crosses a word boundary puts its low bits
+    at the top of one word and its high bits at the bottom of the next.
+    """
+    code = direction_field(i_xi, i_eta, lay.b) | (np.asarray(i_rho, dtype=np.uint64) << np.uint64(2 * lay.b_dir))
     lead = code.shape[:-1]
     words = np.zeros(lead + (lay.words,), dtype=np.uint64)
     c = lay.code_bits
@@ -249,10 +278,9 @@ def unpack(words: np.ndarray, lay: Layout):
         if o + c > 32:
             v = v | (w[..., wi + 1] << np.uint64(32 - o))
         code[..., i] = v & mask
-    m_dir = np.uint64((1 << lay.b_dir) - 1)
+    m_field = np.uint64((1 << (2 * lay.b_dir)) - 1)
     m_rho = np.uint64((1 << lay.b_rho) - 1)
-    i_xi = (code & m_dir).astype(np.int64)
-    i_eta = ((code >> np.uint64(lay.b_dir)) & m_dir).astype(np.int64)
+    i_xi, i_eta = direction_cells(code & m_field, lay.b)
     i_rho = ((code >> np.uint64(2 * lay.b_dir)) & m_rho).astype(np.int64)
     return i_xi, i_eta, i_rho
 

@@ -70,14 +70,17 @@ __device__ __forceinline__ float3 oct_inverse(float a, float b) {
   return make_float3(x * inv, y * inv, r * inv);
 }
 
-// Number of entries of the increasing array t[0..n) that are <= x.
-__device__ __forceinline__ int count_le(const float* t, int n, float x) {
-  int lo = 0, hi = n;  // answer in [lo, hi]
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (t[mid] <= x) lo = mid + 1; else hi = mid;
-  }
-  return lo;
+// Ordered codebook cells (ix, iy) of a code's 2(B+1)-bit direction field
+// m_x | m_y << B | s_x << 2B | s_y << (2B + 1): a cell is stored as its
+// sign (1 = lower half, negative levels) and the rank m of |level| among the
+// positive levels of the odd-symmetric codebook.
+template <int B>
+__device__ __forceinline__ void direction_cells(uint32_t field, int& ix, int& iy) {
+  constexpr uint32_t half = 1u << B, ones = (2u << B) - 1u;
+  const uint32_t mx = field & (half - 1u), my = (field >> B) & (half - 1u);
+  const uint32_t sx = (field >> (2 * B)) & 1u, sy = (field >> (2 * B + 1)) & 1u;
+  ix = static_cast<int>((half | mx) ^ (sx ? ones : 0u));
+  iy = static_cast<int>((half | my) ^ (sy ? ones : 0u));
 }
 
 }  // namespace octo

@@ -106,7 +106,7 @@ bool build_maps(octo::TmaDesc& tm, const octo_layout* L, int64_t heads, int64_t 
   std::memset(&tm, 0, sizeof(tm));
   const cuuint64_t kv = static_cast<cuuint64_t>(kv_len), H = static_cast<cuuint64_t>(heads);
   const cuuint64_t row = static_cast<cuuint64_t>(cap) * 4;  // bytes between token rows of a plane
-  const cuuint32_t KW = 16;
+  const cuuint32_t KW = 16, RK = octo::kTcRoundKeys;
   const int W = L->words, QW = L->d / 32, D = L->d;
   {
     const cuuint64_t dims[3] = {kv, static_cast<cuuint64_t>(W), H}, str[2] = {row, row * W};
@@ -116,7 +116,7 @@ bool build_maps(octo::TmaDesc& tm, const octo_layout* L, int64_t heads, int64_t 
   }
   {
     const cuuint64_t dims[2] = {kv, H}, str[1] = {row};
-    const cuuint32_t box[2] = {KW, 1};
+    const cuuint32_t box[2] = {RK, 1};
     if (!make_map(&tm.gamma, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, gamma, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
     if (L->qjl &&
@@ -125,14 +125,14 @@ bool build_maps(octo::TmaDesc& tm, const octo_layout* L, int64_t heads, int64_t 
   }
   if (L->qjl) {
     const cuuint64_t dims[3] = {kv, static_cast<cuuint64_t>(QW), H}, str[2] = {row, row * QW};
-    const cuuint32_t box[3] = {KW, static_cast<cuuint32_t>(QW), 1};
+    const cuuint32_t box[3] = {RK, static_cast<cuuint32_t>(QW), 1};
     if (!make_map(&tm.qbits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, qjl_bits, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
   }
   if (V) {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), kv, H};
     const cuuint64_t str[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(cap) * D * 2};
-    const cuuint32_t box[3] = {64, KW, 1};
+    const cuuint32_t box[3] = {64, RK, 1};
     if (!make_map(&tm.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return false;
   }

@@ -319,7 +319,8 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 
   // ------------------------------------------------ prologue (overlaps the first copies)
   for (int e = tid; e < NE; e += Cfg::THREADS) {
-    const int ix = e & (NDIR - 1), iy = (e >> BD) & (NDIR - 1);
+    int ix, iy;
+    direction_cells<B>(static_cast<uint32_t>(e), ix, iy);
     float3 n = oct_inverse(s_dir_c[ix], s_dir_c[iy]);
     if constexpr (Cfg::FOLD) {
       const float r = s_rho_c[e >> (2 * BD)];
@@ -708,10 +709,14 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // mma.sync m16n8k16 bf16 with keys as M, query rows as N and rotated
 // coordinates as K. Each 16-wide k-step holds 4 triplets: lane column c4
 // carries triplet 4s + c4 as (x, y | z, 0), so a lane decodes one triplet
-// code per key per k-step. The shared-memory table stores every decoded
-// triplet rho_hat * n_hat already split into bf16 hi + lo halves, in exactly
-// the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); the rotated
-// queries are B fragments held in registers for the whole CTA.
+// code per key per k-step. The shared-memory table holds the decoded
+// triplets rho_hat * n_hat of the positive-level quadrant (codes with both
+// direction signs clear), already split into bf16 hi + lo halves in exactly
+// the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); a code's two
+// direction signs flip the sign bits of x and y in the fragment registers
+// (the codebook is odd-symmetric and the octahedral inverse map is odd in
+// each coordinate, so this is exact). The rotated queries are B fragments
+// held in registers for the whole CTA.
 //
 // Precision: with at most 4 query rows (HL layout) the 8 MMA columns hold the
 // rows' bf16 hi halves (columns 0-3) and lo halves (columns 4-7), so two
@@ -721,27 +726,32 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // used. Either way the logits keep about 16 mantissa bits, well inside the
 // logit tolerance. P.V uses the same layouts with P split into hi + lo.
 //
-// Memory pipeline: every warp works through its own 16-key chunks with no
-// block barrier in the main loop. A chunk's code words, gammas (and sketch
-// words and norms) and its V rows arrive by tensor copies (TMA: 4 to 6 per
-// chunk, completion counted on one mbarrier per slot) into one of two
-// shared-memory slots of the warp; L2 prefetches run PF chunks further
-// ahead. The load/store unit then only serves shared-memory reads: no global
-// load of the main loop queues in front of the table lookups. V arrives with
-// the 128-byte swizzle, so the fragment reads are free of bank conflicts.
+// Memory pipeline: the CTA's key range is cut into rounds of NWARP chunks of
+// 16 keys, one chunk per consumer warp. A producer warp stages whole rounds
+// into a ring of shared-memory stages with a few large tensor copies (TMA:
+// the round's V as two 128-byte-swizzled boxes, its gammas, one code box per
+// chunk), completion counted on the stage's full barrier; the consumer
+// warps release a stage on its empty barrier. The load/store unit then only
+// serves shared-memory reads, and no consumer ever waits on a copy issue.
 // ---------------------------------------------------------------------------
-#ifndef OCTO_DECODE_TC_PF
-#define OCTO_DECODE_TC_PF 4   // chunks a warp prefetches into L2 ahead of its slot copies
+#ifndef OCTO_DECODE_TC_WARPS
+#define OCTO_DECODE_TC_WARPS 8   // consumer warps per CTA (one 16-key chunk of every round each)
 #endif
+#ifndef OCTO_DECODE_TC_STAGES
+#define OCTO_DECODE_TC_STAGES 4  // rounds in flight (shared-memory stages)
+#endif
+
+// Keys of one round (the tensor maps' boxes are built for this size).
+constexpr int kTcRoundKeys = 16 * OCTO_DECODE_TC_WARPS;
 
 // Tensor maps of one decode call (built on the host; token extents are
 // kv_len, so rows past the end arrive as zeros).
 struct TmaDesc {
-  CUtensorMap v;      // bf16 [heads][kv_len][D], box 64 x 16 keys, 128-byte swizzle
+  CUtensorMap v;      // bf16 [heads][kv_len][D], box 64 x round, 128-byte swizzle
   CUtensorMap codes;  // u32 [heads][W][kv_len], box 16 keys x W
-  CUtensorMap gamma;  // f32 [heads][kv_len], box 16
-  CUtensorMap qbits;  // u32 [heads][D/32][kv_len], box 16 x D/32 (OCTOPUS-QJL)
-  CUtensorMap qnorm;  // f32 [heads][kv_len], box 16 (OCTOPUS-QJL)
+  CUtensorMap gamma;  // f32 [heads][kv_len], box round
+  CUtensorMap qbits;  // u32 [heads][D/32][kv_len], box round x D/32 (OCTOPUS-QJL)
+  CUtensorMap qnorm;  // f32 [heads][kv_len], box round (OCTOPUS-QJL)
 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -756,9 +766,8 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z) : "memory");
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 template <int D, int B, int G, bool QJL>
@@ -768,46 +777,66 @@ struct TcCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr int NE = 1 << C;          // full-code table
+  // table over the positive-level quadrant: (m_xi, m_eta, i_rho)
+  static constexpr int NE = 1 << (3 * B - 1);
   static constexpr int REP = 8;              // replicas (distinct bank groups per quarter-warp)
   static constexpr int NKS = (T + 3) / 4;    // logit k-steps (4 triplets each)
   static constexpr bool HL = G <= 4;         // hi and lo halves side by side in the MMA columns
   static constexpr int NB = HL ? 2 : 4;      // query B-fragment registers per k-step
-  static constexpr int KW = 16;              // keys per warp chunk (one m-tile)
+  static constexpr int KW = 16;              // keys per consumer chunk (one m-tile)
   static constexpr int QW = D / 32;          // sketch words per key
   static constexpr int QKS = D / 16;         // sketch k-steps
-  static constexpr int NWARP = 8, THREADS = 256;
-  static constexpr int NSLOT = 2;
-  static constexpr int PF = OCTO_DECODE_TC_PF;
+  static constexpr int NWARP = OCTO_DECODE_TC_WARPS;   // consumer warps
+  static constexpr int THREADS = 32 * (NWARP + 1);     // + the producer warp
+  static constexpr int NS = OCTO_DECODE_TC_STAGES;
+  static constexpr int RK = kTcRoundKeys;    // keys per round
   static constexpr int MT = D / 16, NCH = D / 64;
-  // a slot's V: NCH swizzled boxes of 16 keys x 128 bytes
-  static constexpr int VBOX = KW * 128;
-  static constexpr int VBYTES = NCH * VBOX;
-  // a slot's rows: code words [W][KW], gammas, sketch words [QW][KW], norms
-  // (each part 128-byte aligned for the tensor copies)
-  static constexpr int G_OFF = (4 * W * KW + 127) / 128 * 128;
-  static constexpr int Q_OFF = G_OFF + 128;
-  static constexpr int N_OFF = Q_OFF + (4 * QW * KW + 127) / 128 * 128;
-  static constexpr int CODES = QJL ? N_OFF + 128 : G_OFF + 128;
-  static constexpr uint32_t TX_CODES = 4u * W * KW + 4u * KW + (QJL ? 4u * QW * KW + 4u * KW : 0u);
+  // one stage: V (NCH swizzled boxes of RK rows x 128 bytes), per-warp code
+  // boxes [W][16], gammas, (sketch words [QW][RK], norms); parts 128-byte aligned
+  static constexpr int VHALF = RK * 128;
+  static constexpr int CW = (4 * W * KW + 127) / 128 * 128;
+  static constexpr int ST_V = 0;
+  static constexpr int ST_C = ST_V + NCH * VHALF;
+  static constexpr int ST_G = ST_C + NWARP * CW;
+  static constexpr int ST_Q = ST_G + (4 * RK + 127) / 128 * 128;
+  static constexpr int ST_N = ST_Q + (QJL ? 4 * QW * RK : 0);
+  static constexpr int ST_END = ST_N + (QJL ? (4 * RK + 127) / 128 * 128 : 0);
+  static constexpr int STAGE = (ST_END + 1023) / 1024 * 1024;
   static constexpr int PS = KW + 8;          // P row stride (floats)
   static constexpr size_t TABLE = sizeof(uint4) * NE * REP;
   static constexpr size_t QROW = (12 * NKS > D + 4 ? 12 * NKS : D + 4);  // padded rotated query row
   static constexpr size_t SCRATCH = (sizeof(float) * G * (QROW + (QJL ? D : 0)) + 15) / 16 * 16;
-  static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per warp
+  static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per consumer warp
   // offsets from a 1024-byte aligned base
-  static constexpr size_t VREG = 0;                                   // [NWARP][NSLOT] V
-  static constexpr size_t CREG = VREG + size_t(NWARP) * NSLOT * VBYTES;  // [NWARP][NSLOT] rows
-  static constexpr size_t PREG = CREG + size_t(NWARP) * NSLOT * CODES;   // [NWARP] P
-  static constexpr size_t TREG = PREG + NWARP * PBUF;                 // table
-  static constexpr size_t SREG = TREG + TABLE;                        // query scratch
+  static constexpr size_t SREG = 0;                                  // [NS] stages
+  static constexpr size_t PREG = SREG + size_t(NS) * STAGE;          // [NWARP] P
+  static constexpr size_t TREG = PREG + NWARP * PBUF;                // table
+  static constexpr size_t QREG = TREG + TABLE;                       // query scratch
   static constexpr size_t BUDGET = 227 * 1024 - 2048;
-  static constexpr size_t SMEM = SREG + SCRATCH + 1024;               // + alignment slack
+  static constexpr size_t SMEM = QREG + SCRATCH + 1024;              // + alignment slack
   static constexpr bool FITS = SMEM <= BUDGET;
+  static constexpr uint32_t TX_FIXED = (QJL ? 4u * QW * RK + 4u * RK : 0u) + 4u * RK;  // gammas (+ sketch, norms)
+  static constexpr uint32_t TX_CHUNK = 4u * W * KW;                                     // one code box
   static_assert(G <= 8 && D <= 128 && NCH >= 1, "tensor-core logits shape");
-  static_assert(VBYTES % 1024 == 0 && CODES % 128 == 0 && PBUF % 16 == 0, "alignment of the slots");
-  static_assert(NSLOT * VBYTES >= static_cast<int>(sizeof(float)) * G * (D + 2), "the warp merge reuses the V slots");
+  static_assert(NWARP >= 8 && RK <= 256 && NS >= 2, "consumer warps (one per query row), box rows, stages");
+  static_assert(VHALF % 1024 == 0 && ST_C % 128 == 0 && ST_G % 128 == 0 && ST_Q % 128 == 0 && ST_N % 128 == 0,
+                "alignment of the stage parts");
+  static_assert(size_t(NS) * STAGE >= sizeof(float) * NWARP * G * (D + 2), "the warp merge reuses the stages");
 };
+
+// Table row of a triplet code m_x | m_y << B | s_x << 2B | s_y << (2B+1) |
+// i_rho << (2B+2): the magnitudes and the norm index, signs dropped.
+template <int B>
+__device__ __forceinline__ uint32_t quadrant_index(uint32_t code) {
+  return (code & ((1u << (2 * B)) - 1u)) | ((code >> (2 * B + 2)) << (2 * B));
+}
+// The code's direction signs at the sign bits of the bf16 pair (x, y):
+// s_x -> bit 15, s_y -> bit 31 (the code has at most 13 bits, so neither
+// shift carries other code bits onto those two positions).
+template <int B>
+__device__ __forceinline__ uint32_t quadrant_signs(uint32_t code) {
+  return ((code << (15 - 2 * B)) | (code << (30 - 2 * B))) & 0x80008000u;
+}
 
 __device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi) {
   // +1 / -1 in bf16 (0x3F80 / 0xBF80) for sketch bits 1 / 0
@@ -815,28 +844,31 @@ __device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi)
 }
 
 template <int D, int B, int G, bool QJL>
-__global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const __grid_constant__ TmaDesc tm) {
+__global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
+    decode_tc_kernel(DecodeArgs a, const __grid_constant__ TmaDesc tm) {
   using Cfg = TcCfg<D, B, G, QJL>;
   static_assert(Cfg::FITS, "shared memory budget");
-  constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, BD = Cfg::BD, NDIR = Cfg::NDIR;
-  constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, QW = Cfg::QW, NKS = Cfg::NKS;
-  constexpr int KW = Cfg::KW, NSLOT = Cfg::NSLOT, PF = Cfg::PF;
+  constexpr int T = Cfg::T, C = Cfg::C, NDIR = Cfg::NDIR;
+  constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, NKS = Cfg::NKS;
+  constexpr int KW = Cfg::KW, NS = Cfg::NS, RK = Cfg::RK;
   constexpr int PS = Cfg::PS, MT = Cfg::MT, NCH = Cfg::NCH, QKS = Cfg::QKS, NB = Cfg::NB;
   constexpr bool HL = Cfg::HL;
   constexpr int QROW = static_cast<int>(Cfg::QROW);
+  constexpr uint32_t HALF = 1u << B;
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // 1024-byte aligned base: the swizzled V boxes follow the address bits
   unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint4* table = reinterpret_cast<uint4*>(base + Cfg::TREG);        // [NE][REP]
-  float* scratch = reinterpret_cast<float*>(base + Cfg::SREG);      // [G][QROW] (+ [G][D])
-  __shared__ __align__(8) uint64_t full[NWARP][NSLOT];
+  float* scratch = reinterpret_cast<float*>(base + Cfg::QREG);      // [G][QROW] (+ [G][D])
+  __shared__ __align__(8) uint64_t full[NS], empty[NS];
   __shared__ float s_rho_c[8];
   __shared__ float s_dir_c[32];
   __shared__ int s_last;
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool producer = warp == NWARP;
   const int g8 = lane >> 2, c4 = lane & 3;
   const int split = blockIdx.x;
   const int bh = blockIdx.y;  // b * Hkv + h_kv
@@ -846,50 +878,34 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const _
 
   const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
   const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
-  // chunks of KW keys, dealt to warps round-robin: warp w takes chunks w, w + NWARP, ...
-  const int n_chunks = k_end > k_begin ? static_cast<int>((k_end - k_begin + KW - 1) / KW) : 0;
-  const int my_chunks = warp < n_chunks ? (n_chunks - warp + NWARP - 1) / NWARP : 0;
-  const float* gm = a.gamma + static_cast<int64_t>(bh) * a.cache_cap;
-  const __nv_bfloat16* Vh = with_v ? a.V + static_cast<int64_t>(bh) * a.cache_cap * D : nullptr;
-  float* pw = reinterpret_cast<float*>(base + Cfg::PREG + warp * Cfg::PBUF);  // [G][PS]
-  auto slot_codes = [&](int s) {
-    return reinterpret_cast<uint32_t*>(base + Cfg::CREG + (warp * NSLOT + s) * Cfg::CODES);
-  };
-  auto slot_v = [&](int s) { return base + Cfg::VREG + (warp * NSLOT + s) * Cfg::VBYTES; };
+  // rounds of RK keys; consumer warp w takes keys [16 w, 16 w + 16) of each round
+  const int n_rounds = k_end > k_begin ? static_cast<int>((k_end - k_begin + RK - 1) / RK) : 0;
+  auto stage_base = [&](int s) { return base + Cfg::SREG + static_cast<size_t>(s) * Cfg::STAGE; };
+  float* pw = reinterpret_cast<float*>(base + Cfg::PREG + (producer ? 0 : warp) * Cfg::PBUF);  // [G][PS]
 
-  auto chunk_start = [&](int i) { return k_begin + static_cast<int64_t>(warp + NWARP * i) * KW; };
-  auto chunk_len = [&](int64_t s0) { return static_cast<int>(k_end - s0 < KW ? k_end - s0 : KW); };
-  // This warp's i-th chunk into slot i % NSLOT: lane 0 arms the slot's
-  // barrier with the byte count of the boxes (tokens past kv_len arrive as
-  // zeros and count too) and issues the tensor copies: code words, gammas
-  // (sketch words, norms) and the NCH swizzled V boxes.
-  auto issue_chunk = [&](int i) {
-    if (lane != 0) return;
-    const int x = static_cast<int>(chunk_start(i));
-    const int s = i % NSLOT;
-    uint64_t* bar = &full[warp][s];
-    unsigned char* rows = reinterpret_cast<unsigned char*>(slot_codes(s));
-    mbar_expect_tx(bar, Cfg::TX_CODES + (with_v ? static_cast<uint32_t>(Cfg::VBYTES) : 0u));
-    tma_load_3d(rows, &tm.codes, x, 0, bh, bar);
-    tma_load_2d(rows + Cfg::G_OFF, &tm.gamma, x, bh, bar);
-    if constexpr (QJL) {
-      tma_load_3d(rows + Cfg::Q_OFF, &tm.qbits, x, 0, bh, bar);
-      tma_load_2d(rows + Cfg::N_OFF, &tm.qnorm, x, bh, bar);
-    }
+  // Round r into stage r % NS (producer lane 0): arm the full barrier with
+  // the byte count of the boxes (boxes past kv_len arrive zero-filled and
+  // count in full), then copy the V boxes, the gammas (sketch words, norms)
+  // and one code box per chunk that starts inside the range.
+  auto issue_round = [&](int r) {
+    const int64_t r0 = k_begin + static_cast<int64_t>(r) * RK;
+    const int nch = static_cast<int>((min(k_end - r0, static_cast<int64_t>(RK)) + KW - 1) / KW);
+    const int s = r % NS;
+    unsigned char* st = stage_base(s);
+    uint64_t* bar = &full[s];
+    const int x = static_cast<int>(r0);
+    mbar_expect_tx(bar, Cfg::TX_FIXED + static_cast<uint32_t>(nch) * Cfg::TX_CHUNK +
+                            (with_v ? static_cast<uint32_t>(NCH * Cfg::VHALF) : 0u));
     if (with_v) {
 #pragma unroll
-      for (int hh = 0; hh < NCH; ++hh) tma_load_3d(slot_v(s) + hh * Cfg::VBOX, &tm.v, 64 * hh, x, bh, bar);
+      for (int hh = 0; hh < NCH; ++hh) tma_load_3d(st + Cfg::ST_V + hh * Cfg::VHALF, &tm.v, 64 * hh, x, bh, bar);
     }
-  };
-  // Chunk i's rows and V into L2 ahead of its slot copies.
-  auto prefetch_chunk = [&](int i) {
-    if (lane != 0 || i >= my_chunks) return;
-    const int64_t s0 = chunk_start(i);
-    const int n = chunk_len(s0);
-    tma_prefetch_3d(&tm.codes, static_cast<int>(s0), 0, bh);
-    bulk_prefetch_l2(gm + s0, static_cast<uint32_t>(((n + 3) & ~3) * 4));
-    if constexpr (QJL) tma_prefetch_3d(&tm.qbits, static_cast<int>(s0), 0, bh);
-    if (with_v) bulk_prefetch_l2(Vh + s0 * D, static_cast<uint32_t>(n) * 2u * D);
+    tma_load_2d(st + Cfg::ST_G, &tm.gamma, x, bh, bar);
+    if constexpr (QJL) {
+      tma_load_3d(st + Cfg::ST_Q, &tm.qbits, x, 0, bh, bar);
+      tma_load_2d(st + Cfg::ST_N, &tm.qnorm, x, bh, bar);
+    }
+    for (int c = 0; c < nch; ++c) tma_load_3d(st + Cfg::ST_C + c * Cfg::CW, &tm.codes, x + c * KW, 0, bh, bar);
   };
 
   // The small global reads (codebooks, one sign-flipped query row per warp)
@@ -912,24 +928,27 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const _
 #pragma unroll
     for (int e = 0; e < E; ++e) qraw[e] = 0.0f;
   }
-  if (lane == 0) {
+  if (producer && lane == 0) {
 #pragma unroll
-    for (int s = 0; s < NSLOT; ++s) mbar_init(&full[warp][s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NWARP);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int r = 0; r < NS && r < n_rounds; ++r) issue_round(r);
   }
   if (tid == 0) s_abort = 0;
-  for (int i = 0; i < NSLOT && i < my_chunks; ++i) issue_chunk(i);
-  for (int i = NSLOT; i < NSLOT + PF; ++i) prefetch_chunk(i);
   if (tid < NDIR) s_dir_c[tid] = dir_v;
   if (tid < Cfg::NRHO) s_rho_c[tid] = rho_v;
   __syncthreads();
 
   // ------------------------------------------------ prologue (overlaps the first copies)
-  // decoded-triplet table, pre-split into bf16 hi + lo fragment halves
+  // decoded-triplet table of the positive quadrant (cells HALF + m_xi,
+  // HALF + m_eta), pre-split into bf16 hi + lo fragment halves
   for (int e = tid; e < NE; e += Cfg::THREADS) {
-    const int ix = e & (NDIR - 1), iy = (e >> BD) & (NDIR - 1);
+    const int ix = static_cast<int>(HALF + (e & (HALF - 1))), iy = static_cast<int>(HALF + ((e >> B) & (HALF - 1)));
     float3 n = oct_inverse(s_dir_c[ix], s_dir_c[iy]);
-    const float r = s_rho_c[e >> (2 * BD)];
+    const float r = s_rho_c[e >> (2 * B)];
     n.x *= r; n.y *= r; n.z *= r;
     uint32_t xyh, xyl, zh, zl;
     split_bf16x2(n.x, n.y, xyh, xyl);
@@ -1018,7 +1037,7 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const _
   }
   const int rep_off = lane & (REP - 1);
 
-  // ------------------------------------------------ main loop: this warp's chunks
+  // ------------------------------------------------ main loop
   // This lane's query columns: HL lanes c4 and c4 ^ 2 hold the same two rows
   // (hi and lo columns before the pairwise add), 8-row lanes rows 2c4, 2c4+1.
   const int q0 = HL ? 2 * (c4 & 1) : 2 * c4, q1 = q0 + 1;
@@ -1027,187 +1046,208 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const _
   float acc_o[MT][4];
 #pragma unroll
   for (int t = 0; t < MT; ++t) acc_o[t][0] = acc_o[t][1] = acc_o[t][2] = acc_o[t][3] = 0.0f;
-  int aborted_at = -1;
+  bool aborted = false;
 
-  for (int ci = 0; ci < my_chunks; ++ci) {
-    const int slot = ci % NSLOT;
-    const uint32_t* buf = slot_codes(slot);
-    const unsigned char* vbuf = slot_v(slot);
-    const int64_t s0 = chunk_start(ci);
-    prefetch_chunk(ci + NSLOT + PF);
-    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[warp][slot], (ci / NSLOT) & 1))) {
-      aborted_at = ci;  // warp-uniform
-      break;
+  if (producer) {
+    // Stage round r once the consumers have released its stage (their round
+    // r - NS). Every wait is bounded; on expiry the kernel records the status
+    // and stops issuing. Before the block may exit, the copies of the last
+    // rounds issued have landed (again bounded).
+    if (lane == 0) {
+      int issued = n_rounds < NS ? n_rounds : NS;
+      for (int r = NS; r < n_rounds; ++r) {
+        if (!mbar_wait_bounded(&empty[r % NS], ((r / NS) - 1) & 1)) {
+          aborted = true;
+          break;
+        }
+        issue_round(r);
+        issued = r + 1;
+      }
+      for (int r = issued > NS ? issued - NS : 0; r < issued; ++r)
+        if (!mbar_wait_bounded(&full[r % NS], (r / NS) & 1)) aborted = true;
     }
-
-    // Logits of the chunk in C-fragment layout. Rows are permuted so that a
-    // lane owns 2 consecutive keys: row g8 is key 2 g8, row g8 + 8 is key
-    // 2 g8 + 1; one 8-byte load gives a code word (or gamma, or sketch word)
-    // of both. lgv = (key 2g8, q0), (same, q1), (key 2g8+1, q0), (same, q1).
-    float lgv[4];
-    {
-      constexpr int NC = HL ? 2 : 3;  // independent accumulator chains
-      float acc[NC][4];
-#pragma unroll
-      for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
-      const uint32_t* bk = buf + 2 * g8;  // this lane's 2 keys in row 0
-#pragma unroll
-      for (int s = 0; s < NKS; ++s) {
-        // the code may straddle words wi and wi + 1; for the last word the
-        // next row (gamma or padding) supplies bits that the mask drops
-        const int wi = static_cast<int>(cpos[s] >> 8), sh = static_cast<int>(cpos[s] & 31u);
-        const uint2 lo = *reinterpret_cast<const uint2*>(bk + wi * KW);
-        const uint2 hi = *reinterpret_cast<const uint2*>(bk + (wi + 1) * KW);
-        const uint32_t cm = (1u << C) - 1u;
-        const uint4 eA = table[(__funnelshift_r(lo.x, hi.x, sh) & cm) * REP + rep_off];
-        const uint4 eB = table[(__funnelshift_r(lo.y, hi.y, sh) & cm) * REP + rep_off];
+  } else {
+    for (int r = 0; r < n_rounds; ++r) {
+      const int s = r % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (r / NS) & 1))) {
+        aborted = true;  // warp-uniform
+        break;
+      }
+      const unsigned char* st = stage_base(s);
+      const int64_t s0 = k_begin + static_cast<int64_t>(r) * RK + warp * KW;
+      if (s0 < k_end) {  // warp-uniform: this warp's chunk of the round has keys
+      // Logits of the chunk in C-fragment layout. Rows are permuted so that a
+      // lane owns 2 consecutive keys: row g8 is key 2 g8, row g8 + 8 is key
+      // 2 g8 + 1; one 8-byte load gives a code word (or gamma, or sketch word)
+      // of both. lgv = (key 2g8, q0), (same, q1), (key 2g8+1, q0), (same, q1).
+      float lgv[4];
+      {
+        constexpr int NC = HL ? 2 : 3;  // independent accumulator chains
+        float acc[NC][4];
+  #pragma unroll
+        for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
+        const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + warp * Cfg::CW) + 2 * g8;
+  #pragma unroll
+        for (int s = 0; s < NKS; ++s) {
+          // the code may straddle words wi and wi + 1; for the last word the
+          // next row (the following block of the stage) supplies bits that the mask drops
+          const int wi = static_cast<int>(cpos[s] >> 8), sh = static_cast<int>(cpos[s] & 31u);
+          const uint2 lo = *reinterpret_cast<const uint2*>(bk + wi * KW);
+          const uint2 hi = *reinterpret_cast<const uint2*>(bk + (wi + 1) * KW);
+          const uint32_t cm = (1u << C) - 1u;
+          const uint32_t cA = __funnelshift_r(lo.x, hi.x, sh) & cm, cB = __funnelshift_r(lo.y, hi.y, sh) & cm;
+          uint4 eA = table[quadrant_index<B>(cA) * REP + rep_off];
+          uint4 eB = table[quadrant_index<B>(cB) * REP + rep_off];
+          // the direction signs flip x and y of the hi and lo halves
+          const uint32_t sA = quadrant_signs<B>(cA), sB = quadrant_signs<B>(cB);
+          eA.x ^= sA; eA.z ^= sA;
+          eB.x ^= sB; eB.z ^= sB;
+          if constexpr (HL) {
+            mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
+            mma_bf16_16816(acc[1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
+          } else {
+            mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
+            mma_bf16_16816(acc[1], eA.x, eB.x, eA.y, eB.y, bq[s][NB - 2], bq[s][NB - 1]);
+            mma_bf16_16816(acc[NC - 1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
+          }
+        }
+        float v[4];
+  #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[i] = acc[0][i] + acc[1][i];
+          if constexpr (!HL) v[i] += acc[NC - 1][i];
+        }
+        if constexpr (QJL) {
+          const uint32_t* qk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_Q) + warp * KW + 2 * g8;
+          float accq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  #pragma unroll
+          for (int ks = 0; ks < QKS; ++ks) {
+            const uint2 w2 = *reinterpret_cast<const uint2*>(qk + (ks >> 1) * RK);
+            const int shq = 16 * (ks & 1) + 2 * c4;
+            const uint32_t wA = w2.x >> shq, wB = w2.y >> shq;
+            const uint32_t a0 = pm1_bf16x2(wA, wA >> 1), a1 = pm1_bf16x2(wB, wB >> 1);
+            const uint32_t a2 = pm1_bf16x2(wA >> 8, wA >> 9), a3 = pm1_bf16x2(wB >> 8, wB >> 9);
+            mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
+            if constexpr (!HL) mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
+          }
+          const float kq = 1.2533141373155003f / static_cast<float>(D);  // sqrt(pi/2)/m, m = d
+          const uint2 nu = *reinterpret_cast<const uint2*>(
+              reinterpret_cast<const uint32_t*>(st + Cfg::ST_N) + warp * KW + 2 * g8);
+          const float fA = kq * __uint_as_float(nu.x), fB = kq * __uint_as_float(nu.y);
+          v[0] = fmaf(fA, accq[0], v[0]); v[1] = fmaf(fA, accq[1], v[1]);
+          v[2] = fmaf(fB, accq[2], v[2]); v[3] = fmaf(fB, accq[3], v[3]);
+        }
         if constexpr (HL) {
-          mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
-          mma_bf16_16816(acc[1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
-        } else {
-          mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
-          mma_bf16_16816(acc[1], eA.x, eB.x, eA.y, eB.y, bq[s][NB - 2], bq[s][NB - 1]);
-          mma_bf16_16816(acc[NC - 1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);  // hi column + lo column
         }
+        const uint2 g2 = *reinterpret_cast<const uint2*>(
+            reinterpret_cast<const uint32_t*>(st + Cfg::ST_G) + warp * KW + 2 * g8);
+        const float gA = __uint_as_float(g2.x), gB = __uint_as_float(g2.y);
+        lgv[0] = v[0] * gA; lgv[1] = v[1] * gA;
+        lgv[2] = v[2] * gB; lgv[3] = v[3] * gB;
       }
-      float v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[i] = acc[0][i] + acc[1][i];
-        if constexpr (!HL) v[i] += acc[NC - 1][i];
-      }
-      if constexpr (QJL) {
-        float accq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-        for (int ks = 0; ks < QKS; ++ks) {
-          const uint2 w2 = *reinterpret_cast<const uint2*>(bk + Cfg::Q_OFF / 4 + (ks >> 1) * KW);
-          const int shq = 16 * (ks & 1) + 2 * c4;
-          const uint32_t wA = w2.x >> shq, wB = w2.y >> shq;
-          const uint32_t a0 = pm1_bf16x2(wA, wA >> 1), a1 = pm1_bf16x2(wB, wB >> 1);
-          const uint32_t a2 = pm1_bf16x2(wA >> 8, wA >> 9), a3 = pm1_bf16x2(wB >> 8, wB >> 9);
-          mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
-          if constexpr (!HL) mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
-        }
-        const float kq = 1.2533141373155003f / static_cast<float>(D);  // sqrt(pi/2)/m, m = d
-        const uint2 nu = *reinterpret_cast<const uint2*>(bk + Cfg::N_OFF / 4);
-        const float fA = kq * __uint_as_float(nu.x), fB = kq * __uint_as_float(nu.y);
-        v[0] = fmaf(fA, accq[0], v[0]); v[1] = fmaf(fA, accq[1], v[1]);
-        v[2] = fmaf(fB, accq[2], v[2]); v[3] = fmaf(fB, accq[3], v[3]);
-      }
-      if constexpr (HL) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);  // hi column + lo column
-      }
-      const uint2 g2 = *reinterpret_cast<const uint2*>(bk + Cfg::G_OFF / 4);
-      const float gA = __uint_as_float(g2.x), gB = __uint_as_float(g2.y);
-      lgv[0] = v[0] * gA; lgv[1] = v[1] * gA;
-      lgv[2] = v[2] * gB; lgv[3] = v[3] * gB;
-    }
 
-    const int64_t kown = s0 + 2 * g8;  // lgv[2h + qq] is key kown + h
-    if (a.logits != nullptr && owner) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t key = kown + h;
-        if (key >= k_end) continue;
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int r = q0 + qq;
-          if (r < a.Gq) {
-            const int gi = r / a.Lq, lq = r - gi * a.Lq;
-            const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
-            a.logits[row * a.kv_len + key] = lgv[2 * h + qq];
+      const int64_t kown = s0 + 2 * g8;  // lgv[2h + qq] is key kown + h
+      if (a.logits != nullptr && owner) {
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t key = kown + h;
+          if (key >= k_end) continue;
+  #pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const int r = q0 + qq;
+            if (r < a.Gq) {
+              const int gi = r / a.Lq, lq = r - gi * a.Lq;
+              const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
+              a.logits[row * a.kv_len + key] = lgv[2 * h + qq];
+            }
           }
         }
       }
-    }
-    if (with_v) {
-      // online softmax over the chunk, base 2, per query column; keys live on the g8 lanes
-      const bool vA = kown < k_end, vB = kown + 1 < k_end;
-      lgv[0] = vA ? lgv[0] * a.scale_log2 : -INFINITY;
-      lgv[1] = vA ? lgv[1] * a.scale_log2 : -INFINITY;
-      lgv[2] = vB ? lgv[2] * a.scale_log2 : -INFINITY;
-      lgv[3] = vB ? lgv[3] * a.scale_log2 : -INFINITY;
-      float mx0 = fmaxf(lgv[0], lgv[2]), mx1 = fmaxf(lgv[1], lgv[3]);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      if (with_v) {
+        // online softmax over the chunk, base 2, per query column; keys live on the g8 lanes
+        const bool vA = kown < k_end, vB = kown + 1 < k_end;
+        lgv[0] = vA ? lgv[0] * a.scale_log2 : -INFINITY;
+        lgv[1] = vA ? lgv[1] * a.scale_log2 : -INFINITY;
+        lgv[2] = vB ? lgv[2] * a.scale_log2 : -INFINITY;
+        lgv[3] = vB ? lgv[3] * a.scale_log2 : -INFINITY;
+        float mx0 = fmaxf(lgv[0], lgv[2]), mx1 = fmaxf(lgv[1], lgv[3]);
+  #pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
+        m0 = n0; m1 = n1;
+        lgv[0] = fast_exp2(lgv[0] - n0); lgv[2] = fast_exp2(lgv[2] - n0);
+        lgv[1] = fast_exp2(lgv[1] - n1); lgv[3] = fast_exp2(lgv[3] - n1);
+        l0 = l0 * al0 + lgv[0] + lgv[2];
+        l1 = l1 * al1 + lgv[1] + lgv[3];
+  #pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
+        }
+        // P rows (query-major) for the P.V B fragments: this lane's 2 consecutive keys
+        if (owner) {
+          if (q0 < G) *reinterpret_cast<float2*>(pw + q0 * PS + 2 * g8) = make_float2(lgv[0], lgv[2]);
+          if (q1 < G) *reinterpret_cast<float2*>(pw + q1 * PS + 2 * g8) = make_float2(lgv[1], lgv[3]);
+        }
+        __syncwarp();
+
+        // P.V over the chunk (O^T = V^T P^T: d as M, keys as K)
+        uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;  // (hi | lo) of keys 2c4, 2c4+1 and 2c4+8, 2c4+9
+        if (brow < G) {
+          const float* prow = pw + brow * PS + 2 * c4;
+          const float2 p01 = *reinterpret_cast<const float2*>(prow);
+          const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
+          uint32_t h01, l01, h89, l89;
+          split_bf16x2(p01.x, p01.y, h01, l01);
+          split_bf16x2(p89.x, p89.y, h89, l89);
+          if constexpr (HL) {
+            b0 = blo ? l01 : h01; b1 = blo ? l89 : h89;
+          } else {
+            b0 = h01; b1 = h89; b2 = l01; b3 = l89;
+          }
+        }
+  #pragma unroll
+        for (int hh = 0; hh < NCH; ++hh) {
+          // 8 consecutive d (64 hh + 8 g8 ...) of keys 2c4, 2c4+1, 2c4+8, 2c4+9:
+          // in the swizzled box, 16-byte unit g8 of row k sits at unit g8 ^ (k & 7)
+          // (this warp's rows start at a multiple of 8)
+          const unsigned char* vb = st + Cfg::ST_V + hh * Cfg::VHALF + warp * KW * 128;
+          auto vld = [&](int k) {
+            return *reinterpret_cast<const uint4*>(vb + k * 128 + ((g8 ^ (k & 7)) << 4));
+          };
+          const uint4 k0 = vld(2 * c4), k1 = vld(2 * c4 + 1), k8 = vld(2 * c4 + 8), k9 = vld(2 * c4 + 9);
+          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
+          const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
+  #pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
+            const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
+            const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
+            const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
+            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b0, b1);
+            if constexpr (!HL) mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b2, b3);
+          }
+        }
       }
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
-      m0 = n0; m1 = n1;
-      lgv[0] = fast_exp2(lgv[0] - n0); lgv[2] = fast_exp2(lgv[2] - n0);
-      lgv[1] = fast_exp2(lgv[1] - n1); lgv[3] = fast_exp2(lgv[3] - n1);
-      l0 = l0 * al0 + lgv[0] + lgv[2];
-      l1 = l1 * al1 + lgv[1] + lgv[3];
-#pragma unroll
-      for (int t = 0; t < MT; ++t) {
-        acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
       }
-      // P rows (query-major) for the P.V B fragments: this lane's 2 consecutive keys
-      if (owner) {
-        if (q0 < G) *reinterpret_cast<float2*>(pw + q0 * PS + 2 * g8) = make_float2(lgv[0], lgv[2]);
-        if (q1 < G) *reinterpret_cast<float2*>(pw + q1 * PS + 2 * g8) = make_float2(lgv[1], lgv[3]);
-      }
+      // this warp is done with the stage: release it to the producer
       __syncwarp();
-
-      // P.V over the chunk (O^T = V^T P^T: d as M, keys as K)
-      uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;  // (hi | lo) of keys 2c4, 2c4+1 and 2c4+8, 2c4+9
-      if (brow < G) {
-        const float* prow = pw + brow * PS + 2 * c4;
-        const float2 p01 = *reinterpret_cast<const float2*>(prow);
-        const float2 p89 = *reinterpret_cast<const float2*>(prow + 8);
-        uint32_t h01, l01, h89, l89;
-        split_bf16x2(p01.x, p01.y, h01, l01);
-        split_bf16x2(p89.x, p89.y, h89, l89);
-        if constexpr (HL) {
-          b0 = blo ? l01 : h01; b1 = blo ? l89 : h89;
-        } else {
-          b0 = h01; b1 = h89; b2 = l01; b3 = l89;
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < NCH; ++hh) {
-        // 8 consecutive d (64 hh + 8 g8 ...) of keys 2c4, 2c4+1, 2c4+8, 2c4+9:
-        // in the swizzled box, 16-byte unit g8 of key row k sits at unit g8 ^ (k & 7)
-        const unsigned char* vb = vbuf + hh * Cfg::VBOX;
-        auto vld = [&](int k) {
-          return *reinterpret_cast<const uint4*>(vb + k * 128 + ((g8 ^ (k & 7)) << 4));
-        };
-        const uint4 k0 = vld(2 * c4), k1 = vld(2 * c4 + 1), k8 = vld(2 * c4 + 8), k9 = vld(2 * c4 + 9);
-        const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-        const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
-          const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
-          const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
-          const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-          mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b0, b1);
-          if constexpr (!HL) mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b2, b3);
-        }
-      }
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-    // the chunk's slot (rows, V, P) is consumed: refill it with chunk ci + NSLOT
-    __syncwarp();
-    if (ci + NSLOT < my_chunks) issue_chunk(ci + NSLOT);
   }
-
-  // A bounded wait that expired: record it, let this warp's copies in flight
-  // land (again bounded) before the block can exit, and skip the output.
-  if (aborted_at >= 0) {
-    if (lane == 0) {
-      atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
-      s_abort = 1;
-    }
-    for (int c = aborted_at; c < aborted_at + NSLOT && c < my_chunks; ++c)
-      mbar_wait_bounded(&full[warp][c % NSLOT], (c / NSLOT) & 1);
+  if (aborted && lane == 0) {
+    atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
+    s_abort = 1;
   }
-  __syncthreads();  // every slot is free: no copy is in flight after the last chunk
+  __syncthreads();  // every stage is free: no copy is in flight after the last round
   if (s_abort || !with_v) return;
 
-  // ------------------------------------------------ epilogue: merge warps (in each warp's V slots)
+  // ------------------------------------------------ epilogue: merge warps (in the stage memory)
   if constexpr (HL) {  // hi column + lo column of every output
 #pragma unroll
     for (int t = 0; t < MT; ++t)
@@ -1219,8 +1259,8 @@ __global__ void __launch_bounds__(256, 1) decode_tc_kernel(DecodeArgs a, const _
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
-  auto wbase = [&](int w) { return reinterpret_cast<float*>(base + Cfg::VREG + w * NSLOT * Cfg::VBYTES); };
-  if (owner) {
+  auto wbase = [&](int w) { return reinterpret_cast<float*>(base + Cfg::SREG) + w * G * (D + 2); };
+  if (!producer && owner) {
     float* wm = wbase(warp);  // [G] m, [G] l, [G][D] O
     if (g8 == 0) {
       if (q0 < G) { wm[q0] = m0; wm[G + q0] = l0; }

@@ -62,6 +62,20 @@ struct EncCfg {
   static constexpr int REP = NDIR * NDIR <= 256 ? 8 : 4;  // n_hat replicas (distinct bank groups per quarter-warp)
 };
 
+// Direction field of a triplet code from the ordered cells (ix, iy): the
+// symmetric codebook's cell i is stored as a sign s (1 for the lower half,
+// i < 2^B) and the rank m of |level| among the positive levels, as
+// m_x | m_y << B | s_x << 2B | s_y << (2B + 1); XOR with all ones maps a
+// lower-half cell onto its mirror.
+template <int B>
+__device__ __forceinline__ uint32_t direction_field(int ix, int iy) {
+  constexpr uint32_t half = 1u << B, ones = (2u << B) - 1u;
+  const uint32_t sx = static_cast<uint32_t>(ix) < half, sy = static_cast<uint32_t>(iy) < half;
+  const uint32_t mx = (static_cast<uint32_t>(ix) ^ (sx ? ones : 0u)) & (half - 1u);
+  const uint32_t my = (static_cast<uint32_t>(iy) ^ (sy ? ones : 0u)) & (half - 1u);
+  return mx | (my << B) | (sx << (2 * B)) | (sy << (2 * B + 1));
+}
+
 template <int D, int B, bool QJL>
 __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   using Cfg = EncCfg<D, B>;
@@ -225,7 +239,7 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
           }
         }
       }
-      codes[k * T + i] = static_cast<uint16_t>(ix | (iy << Cfg::BD) | (ir << (2 * Cfg::BD)));
+      codes[k * T + i] = static_cast<uint16_t>(direction_field<B>(ix, iy) | (ir << (2 * Cfg::BD)));
       if constexpr (QJL) {
         // residual e = t - rho_hat n_hat, in place (the pad coordinate is dropped later)
         tp[0] = x - rh * nb.x;

@@ -130,20 +130,27 @@ def test_joint_rho_is_nearest_to_projection():
 
 # ---------------------------------------------------------------- packing
 def test_pack_by_hand():
-    # b=2: c = 7 bits; triplet codes 93 (xi 5, eta 3, rho 1) and 71 (xi 7, eta 0, rho 1)
+    # b=2 (c = 7 bits, half = 4): cells (xi 5, eta 3, rho 1) -> m_xi 1, s_xi 0, m_eta 0, s_eta 1:
+    # 1 | 0 << 2 | 0 << 4 | 1 << 5 | 1 << 6 = 97; (7, 0, 1) -> 3 | 3 << 2 | 0 | 1 << 5 | 1 << 6 = 111
     lay = codec.Layout(6, 2)
     w = codec.pack(np.array([[5, 7]]), np.array([[3, 0]]), np.array([[1, 1]]), lay)
-    assert lay.words == 1 and int(w[0, 0]) == 93 + (71 << 7)
-    # b=4: c = 13 bits; the third code crosses into word 1
+    assert lay.words == 1 and int(w[0, 0]) == 97 + (111 << 7)
+    # b=4 (c = 13 bits, half = 16): (28, 5, 5) -> 12 | 10 << 4 | 1 << 9 | 5 << 10 = 0x16AC,
+    # (16, 15, 0) -> 0 | 0 | 1 << 9 = 0x200, (0, 31, 7) -> 15 | 15 << 4 | 1 << 8 | 7 << 10 = 0x1DFF;
+    # the third code crosses into word 1
     lay = codec.Layout(9, 4)
-    code = [0x1ABC, 0x0F0F, 0x1FFF]
-    ix = np.array([[v & 31 for v in code]])
-    iy = np.array([[(v >> 5) & 31 for v in code]])
-    ir = np.array([[(v >> 10) & 7 for v in code]])
-    w = codec.pack(ix, iy, ir, lay)
+    w = codec.pack(np.array([[28, 16, 0]]), np.array([[5, 15, 31]]), np.array([[5, 0, 7]]), lay)
     assert lay.words == 2
-    assert int(w[0, 0]) == (0x1ABC | (0x0F0F << 13) | ((0x1FFF & 63) << 26))
-    assert int(w[0, 1]) == 0x1FFF >> 6
+    assert int(w[0, 0]) == (0x16AC | (0x200 << 13) | ((0x1DFF & 63) << 26))
+    assert int(w[0, 1]) == 0x1DFF >> 6
+
+
+def _code_by_hand(ix, iy, ir, b):
+    half = 1 << b
+    sx, sy = int(ix < half), int(iy < half)
+    mx = ix - half if ix >= half else half - 1 - ix
+    my = iy - half if iy >= half else half - 1 - iy
+    return mx | my << b | sx << 2 * b | sy << (2 * b + 1) | ir << (2 * b + 2)
 
 
 @pytest.mark.parametrize("d,b", [(64, 2), (128, 3), (128, 4), (256, 2), (256, 4)])
@@ -159,10 +166,22 @@ def test_pack_round_trip_and_sizes(d, b):
     for r in range(7):
         stream = 0
         for i in range(lay.T):
-            stream |= (int(ix[r, i]) | int(iy[r, i]) << lay.b_dir | int(ir[r, i]) << 2 * lay.b_dir) << (i * lay.code_bits)
+            stream |= _code_by_hand(int(ix[r, i]), int(iy[r, i]), int(ir[r, i]), b) << (i * lay.code_bits)
         assert [int(x) for x in w[r]] == [(stream >> (32 * j)) & 0xFFFFFFFF for j in range(lay.words)]
     a, bb, c = codec.unpack(w, lay)
     assert np.array_equal(a, ix) and np.array_equal(bb, iy) and np.array_equal(c, ir)
+
+
+def test_direction_field_pairs_opposite_cells():
+    # cells i and L-1-i (levels c and -c) share the magnitude and differ only in the sign bit
+    for b in (2, 3, 4):
+        L = 1 << (b + 1)
+        i = np.arange(L)
+        f = codec.direction_field(i, np.zeros_like(i), b).astype(np.int64)
+        g = codec.direction_field(L - 1 - i, np.zeros_like(i), b).astype(np.int64)
+        sign = 1 << (2 * b)
+        assert np.array_equal(f ^ g, np.full(L, sign))
+        assert np.array_equal(np.sort(f & ((1 << b) - 1)), np.repeat(np.arange(1 << b), 2))
 
 
 # ---------------------------------------------------------------- quality
