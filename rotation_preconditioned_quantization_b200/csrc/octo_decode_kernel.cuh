@@ -144,7 +144,8 @@ struct DecCfg {
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
-  asm volatile(
+  // a pure register operation: not volatile, so the scheduler may interleave it
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -831,11 +832,23 @@ __device__ __forceinline__ uint32_t quadrant_index(uint32_t code) {
   return (code & ((1u << (2 * B)) - 1u)) | ((code >> (2 * B + 2)) << (2 * B));
 }
 // The code's direction signs at the sign bits of the bf16 pair (x, y):
-// s_x -> bit 15, s_y -> bit 31 (the code has at most 13 bits, so neither
-// shift carries other code bits onto those two positions).
+// s_x -> bit 15, s_y -> bit 31. One multiply forms code << (15 - 2B) plus
+// code << (30 - 2B); for a code of at most 13 bits (b <= 4) the two copies
+// do not overlap, so the sum is their OR and nothing else lands on bit 15
+// or bit 31.
 template <int B>
 __device__ __forceinline__ uint32_t quadrant_signs(uint32_t code) {
-  return ((code << (15 - 2 * B)) | (code << (30 - 2 * B))) & 0x80008000u;
+  static_assert(B <= 4, "non-overlapping shifted copies");
+  return (code * ((1u << (15 - 2 * B)) + (1u << (30 - 2 * B)))) & 0x80008000u;
+}
+
+// Four 8x8 b16 matrices from shared memory, transposed (ldmatrix): lanes
+// 8i .. 8i+7 give the row addresses of matrix i, register i receives it.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                              const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p)));
 }
 
 __device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi) {
@@ -1211,27 +1224,20 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
             b0 = h01; b1 = h89; b2 = l01; b3 = l89;
           }
         }
+        // A fragments of V^T by transposed matrix loads from the swizzled
+        // box: d-tile t (16 dims) x the chunk's 16 keys. Lane L addresses key
+        // (L & 7) + 8 (L >> 4) at 16-byte unit 2t + ((L >> 3) & 1) of the
+        // row, which the swizzle keeps at unit ^ (key & 7) (this warp's rows
+        // start at a multiple of 8); units 8.. are the second 64-dim box.
+        const int vkey = (lane & 7) + ((lane >> 4) << 3);
+        const unsigned char* vrow = st + Cfg::ST_V + (warp * KW + vkey) * 128;
   #pragma unroll
-        for (int hh = 0; hh < NCH; ++hh) {
-          // 8 consecutive d (64 hh + 8 g8 ...) of keys 2c4, 2c4+1, 2c4+8, 2c4+9:
-          // in the swizzled box, 16-byte unit g8 of row k sits at unit g8 ^ (k & 7)
-          // (this warp's rows start at a multiple of 8)
-          const unsigned char* vb = st + Cfg::ST_V + hh * Cfg::VHALF + warp * KW * 128;
-          auto vld = [&](int k) {
-            return *reinterpret_cast<const uint4*>(vb + k * 128 + ((g8 ^ (k & 7)) << 4));
-          };
-          const uint4 k0 = vld(2 * c4), k1 = vld(2 * c4 + 1), k8 = vld(2 * c4 + 8), k9 = vld(2 * c4 + 9);
-          const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
-          const uint32_t w8[4] = {k8.x, k8.y, k8.z, k8.w}, w9[4] = {k9.x, k9.y, k9.z, k9.w};
-  #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const uint32_t a0 = __byte_perm(w0[e2], w1[e2], 0x5410);
-            const uint32_t a1 = __byte_perm(w0[e2], w1[e2], 0x7632);
-            const uint32_t a2 = __byte_perm(w8[e2], w9[e2], 0x5410);
-            const uint32_t a3 = __byte_perm(w8[e2], w9[e2], 0x7632);
-            mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b0, b1);
-            if constexpr (!HL) mma_bf16_16816(acc_o[hh * 4 + e2], a0, a1, a2, a3, b2, b3);
-          }
+        for (int t = 0; t < MT; ++t) {
+          const int unit = 2 * t + ((lane >> 3) & 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(a0, a1, a2, a3, vrow + (unit >> 3) * Cfg::VHALF + (((unit & 7) ^ (vkey & 7)) << 4));
+          mma_bf16_16816(acc_o[t], a0, a1, a2, a3, b0, b1);
+          if constexpr (!HL) mma_bf16_16816(acc_o[t], a0, a1, a2, a3, b2, b3);
         }
       }
       }
@@ -1268,11 +1274,10 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
     }
     float* o = wm + 2 * G;
 #pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      const int hh = t >> 2, e2 = t & 3;
-      const int d0 = 64 * hh + 8 * g8 + 2 * e2;
-      if (q0 < G) { o[q0 * D + d0] = acc_o[t][0]; o[q0 * D + d0 + 1] = acc_o[t][2]; }
-      if (q1 < G) { o[q1 * D + d0] = acc_o[t][1]; o[q1 * D + d0 + 1] = acc_o[t][3]; }
+    for (int t = 0; t < MT; ++t) {  // rows g8 and g8 + 8 of d-tile t
+      const int d0 = 16 * t + g8;
+      if (q0 < G) { o[q0 * D + d0] = acc_o[t][0]; o[q0 * D + d0 + 8] = acc_o[t][2]; }
+      if (q1 < G) { o[q1 * D + d0] = acc_o[t][1]; o[q1 * D + d0 + 8] = acc_o[t][3]; }
     }
   }
   __syncthreads();

@@ -70,8 +70,10 @@ def _run_case(B, Hq, Hkv, Lq, d, b, N, qjl=False, q_dtype=torch.bfloat16, cap=No
     dev = api.DeviceTables(*tb, signs, S)
     qt = torch.from_numpy(q).to(q_dtype).cuda()
     Vt = None if logits_only else torch.from_numpy(Vn).to(torch.bfloat16).cuda()
-    out, lg = api.decode_attn(lay, dev, qt, cache, Vt, Hkv, kv_len=kv, logits=check_logits)
+    ws = api.Workspace(api.decode_attn_workspace_bytes(lay, B, Hq, Hkv, Lq, kv))
+    out, lg = api.decode_attn(lay, dev, qt, cache, Vt, Hkv, kv_len=kv, logits=check_logits, workspace=ws)
     torch.cuda.synchronize()
+    assert ws.status() == 0, "a bounded device wait expired"
     olay = codec.Layout(d, b)
     g = Hq // Hkv
     if kv == 0:
