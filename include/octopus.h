@@ -37,7 +37,11 @@
  * Word w of token n's bit stream is packed[h][w][n]. Within the stream,
  * the (3b+1)-bit code of triplet i starts at bit i(3b+1), LSB first (bit p
  * of the stream is bit p mod 32 of word p / 32); a code is
- * i_xi | i_eta << (b+1) | i_rho << 2(b+1).
+ *   m_xi | m_eta << b | s_xi << 2b | s_eta << (2b+1) | i_rho << 2(b+1),
+ * where a direction cell index i in [0, 2^(b+1)) of the odd-symmetric
+ * codebook is stored as a sign s (1 for the lower half, i < 2^b) and the
+ * rank m of |level| among the positive levels (m = i - 2^b above the
+ * middle, 2^b - 1 - i below).
  */
 #ifndef OCTOPUS_B200_H
 #define OCTOPUS_B200_H

@@ -1198,9 +1198,11 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         lgv[1] = fast_exp2(lgv[1] - n1); lgv[3] = fast_exp2(lgv[3] - n1);
         l0 = l0 * al0 + lgv[0] + lgv[2];
         l1 = l1 * al1 + lgv[1] + lgv[3];
+        if (__any_sync(0xffffffffu, al0 != 1.0f || al1 != 1.0f)) {  // some running max moved
   #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
+          for (int t = 0; t < MT; ++t) {
+            acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
+          }
         }
         // P rows (query-major) for the P.V B fragments: this lane's 2 consecutive keys
         if (owner) {
