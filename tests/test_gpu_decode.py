@@ -181,3 +181,76 @@ def test_decode_rejects_small_workspace(cuda_ok):
                                      0.1, torch.empty((1, 4, 1, 128), device="cuda").data_ptr(), None,
                                      ws.buf.data_ptr(), 256, None)
     assert st == _lib.OCTO_EWORKSPACE
+
+
+def _run_sampled_full_size(B, Hq, Hkv, Lq, d, b, N, qjl, sample, keys_fn, seed=11):
+    """Full-size decode; every output and logit of the sampled KV heads is checked.
+
+    The sampled heads hold the oracle's encoding of seeded keys and seeded V.
+    The other heads hold arbitrary code words and V, drawn on the device,
+    since decode attention is independent per (batch, KV head).
+    """
+    tb = parity.oracle_tables(d, b)
+    H = B * Hkv
+    lay = api.Layout(d, b, qjl=qjl)
+    olay = codec.Layout(d, b)
+    signs = tables.rotation_signs(seed, d, Hkv)
+    S = tables.qjl_matrix(seed + 7, d, Hkv) if qjl else None
+    cache = api.Cache.empty(lay, H, N)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    cache.packed.random_(generator=g)
+    cache.gamma.uniform_(0.5, 2.0, generator=g)
+    if qjl:
+        cache.qjl_bits.random_(generator=g)
+        cache.qjl_norm.uniform_(0.0, 0.3, generator=g)
+    V = torch.randn((H, N, d), device="cuda", generator=g).to(torch.bfloat16)
+    cache.length = N
+    refs = {}
+    for h in sample:
+        keys = keys_fn(seed + 100 + h, N, d)
+        e = codec.encode(keys.astype(np.float64), signs[h % Hkv], tb, olay)
+        cache.packed[h, :, :N] = torch.from_numpy(parity.to_planar(e.words[None])[0].view(np.int32)).cuda()
+        cache.gamma[h, :N] = torch.from_numpy(e.gamma.astype(np.float32)).cuda()
+        if qjl:
+            uh = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, olay)
+            bits, nu, _ = codec.qjl_encode(e.u_rot, uh, S[h % Hkv])
+            e.qbits, e.nu = bits, nu
+            cache.qjl_bits[h, :, :N] = torch.from_numpy(parity.to_planar(codec.qjl_pack(bits)[None])[0].view(np.int32)).cuda()
+            cache.qjl_norm[h, :N] = torch.from_numpy(nu.astype(np.float32)).cuda()
+        vh = inputs.to_bf16(inputs.normal(seed + 200 + h, (N, d)))
+        V[h] = torch.from_numpy(vh).to(torch.bfloat16).cuda()
+        refs[h] = (e, vh)
+    q = inputs.to_bf16(inputs.normal(seed + 2, (B, Hq, Lq, d)))
+    dev = api.DeviceTables(*tb, signs, S)
+    ws = api.Workspace(api.decode_attn_workspace_bytes(lay, B, Hq, Hkv, Lq, N))
+    out, lg = api.decode_attn(lay, dev, torch.from_numpy(q).to(torch.bfloat16).cuda(), cache, V, Hkv,
+                              logits=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0, "a bounded device wait expired"
+    grp = Hq // Hkv
+    for h, (e, vh) in refs.items():
+        bi, hk = divmod(h, Hkv)
+        qq = q[bi, hk * grp:(hk + 1) * grp].reshape(grp * Lq, d).astype(np.float64)
+        qjl_args = (e.qbits, e.nu, S[hk]) if qjl else None
+        ref_o, ref_l = attention.decode_attention(qq, e.gamma, e.i_xi, e.i_eta, e.i_rho, vh.astype(np.float64),
+                                                  signs[hk], tb, olay, qjl=qjl_args)
+        got_l = lg[bi, hk * grp:(hk + 1) * grp].reshape(grp * Lq, N).cpu().numpy()
+        tol_l = 1e-4 * e.gamma[None, :] * np.linalg.norm(qq, axis=1)[:, None]
+        assert np.all(np.abs(got_l - ref_l) <= tol_l), f"head {h}: logit error"
+        got_o = out[bi, hk * grp:(hk + 1) * grp].reshape(grp * Lq, d).cpu().numpy()
+        tol_o = 2e-3 * np.max(np.abs(ref_o), axis=1, keepdims=True)
+        assert np.all(np.abs(got_o - ref_o) <= tol_o), f"head {h}: output error {np.max(np.abs(got_o - ref_o) / tol_o)} x tol"
+
+
+def test_decode_video_audio_shaped_full_size(cuda_ok):
+    """16 heads, d=64 (22 triplets, last padded), 65536 tokens, b=2, 8 query tokens per head;
+    bf16 keys ~ N(0,1). Heads 0 and 9 are checked in full."""
+    _run_sampled_full_size(1, 16, 16, 8, 64, 2, 65536, False, (0, 9),
+                           lambda s, n, d: inputs.to_bf16(inputs.gaussian_keys(s, 1, n, d)[0]))
+
+
+def test_decode_qjl_long_context_full_size(cuda_ok):
+    """Batch 8, 32 query / 8 KV heads, d=128, 131072 tokens, b=4 + OCTOPUS-QJL sketch;
+    LLM-shaped bf16 keys. KV heads 0 and 43 (batch 5) are checked in full."""
+    _run_sampled_full_size(8, 32, 8, 1, 128, 4, 131072, True, (0, 43),
+                           lambda s, n, d: inputs.to_bf16(inputs.llm_keys(s, 1, n, d)[0]))

@@ -154,3 +154,42 @@ def test_encode_llm_prefill_full_size(cuda_ok):
     """Full LLM-shaped prefill: 8 KV heads x 32768 bf16 keys, d=128, b=3, joint."""
     k = inputs.to_bf16(inputs.llm_keys(2, 8, 32768, 128))
     _check(k, 128, 3, api.ROUND_JOINT, torch.bfloat16, seed=0, label="llm-prefill-full")
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_encode_sweep_appends(cuda_ok, d, b):
+    """Encode sweep: 4 heads x 2^18 fp32 keys ~ N(0,1) (2^20 keys) streamed in appends of
+    1-4096 tokens, seeded rotation per head. The appended cache equals a one-shot encode
+    bit for bit, and 512 sampled tokens per head match the oracle (boundary cases counted)."""
+    H, N = 4, 1 << 18
+    k = inputs.gaussian_keys(1000 + 10 * d + b, H, N, d)
+    tb = parity.oracle_tables(d, b)
+    signs = tables.rotation_signs(d * 7 + b, d, H)
+    lay = api.Layout(d, b)
+    dev = api.DeviceTables(*tb, signs)
+    kt = torch.from_numpy(k).cuda()
+    app = api.Cache.empty(lay, H, N)
+    for n in inputs.append_lengths(d + b, N, 1, 4096):
+        s = app.length
+        api.encode(lay, dev, kt[:, s:s + n], app)
+    one = api.Cache.empty(lay, H, N)
+    api.encode(lay, dev, kt, one, 0)
+    torch.cuda.synchronize()
+    assert app.length == N
+    assert torch.equal(one.packed, app.packed) and torch.equal(one.gamma, app.gamma)
+    olay = codec.Layout(d, b)
+    rng = np.random.default_rng(d * 10 + b)
+    tot = dict(mis=0, bnd=0, trip=0)
+    for h in range(H):
+        idx = np.sort(rng.choice(N, 512, replace=False))
+        enc = codec.encode(k[h, idx].astype(np.float64), signs[h], tb, olay)
+        words = parity.from_planar(app.packed[h:h + 1].cpu().numpy(), N)[0][idx]
+        gam = app.gamma[h].cpu().numpy()[idx]
+        np.testing.assert_allclose(gam, enc.gamma, rtol=1e-4, atol=0)
+        m, bn, f, fails = parity.classify_codes(enc, words, tb, olay, True)
+        assert f == 0, f"head {h}: {f} non-boundary code mismatches, e.g. {fails}"
+        tot["mis"] += m; tot["bnd"] += bn; tot["trip"] += len(idx) * olay.T
+    assert tot["bnd"] <= MAX_BOUNDARY_FRACTION * tot["trip"]
+    print(f"\n[encode sweep] d={d} b={b}: {H}x{N} keys appended; sampled {tot['trip']} triplets, "
+          f"{tot['mis']} mismatches, all at a boundary ({tot['bnd']})")
