@@ -227,6 +227,56 @@ def run_reference(args):
     return 0
 
 
+# Decode throughput on the other workload shapes (reported next to the main
+# metric). Codes, gammas, sketches, V and queries are drawn on the device:
+# the decode's work and traffic do not depend on their values.
+OTHER_WORKLOADS = (
+    ("video_audio: B=1, 16/16 heads, d=64, ctx=65536, b=2, 8 query tokens", 1, 16, 16, 8, 64, 2, 65536, False),
+    ("qjl_long_context: B=8, 32/8 heads, d=128, ctx=131072, b=4 + QJL sketch", 8, 32, 8, 1, 128, 4, 131072, True),
+    ("llm_decode_large: B=8, 32/8 heads, d=128, ctx=131072, b=3", 8, 32, 8, 1, 128, 3, 131072, False),
+)
+
+
+def other_workloads(dev, peak, iters=6):
+    out = {}
+    flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)  # > L2 between timed calls
+    for name, B_, HQ_, HKV_, LQ_, D_, BITS_, N_, qjl in OTHER_WORKLOADS:
+        lay = api.Layout(D_, BITS_, qjl=qjl)
+        H = B_ * HKV_
+        tabs = api.DeviceTables.build(lay, SEED, HKV_, device=dev)
+        g = torch.Generator(device=dev).manual_seed(SEED)
+        cache = api.Cache.empty(lay, H, N_, dev)
+        cache.packed.random_(generator=g)
+        cache.gamma.uniform_(0.5, 2.0, generator=g)
+        if qjl:
+            cache.qjl_bits.random_(generator=g)
+            cache.qjl_norm.uniform_(0.0, 0.3, generator=g)
+        cache.length = N_
+        V = torch.randn((H, N_, D_), device=dev, generator=g).to(torch.bfloat16)
+        q = torch.randn((B_, HQ_, LQ_, D_), device=dev, generator=g).to(torch.bfloat16)
+        o = torch.empty((B_, HQ_, LQ_, D_), device=dev)
+        wsp = api.Workspace(api.decode_attn_workspace_bytes(lay, B_, HQ_, HKV_, LQ_, N_), dev)
+        ts = []
+        for i in range(iters + 2):
+            flush.sum()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            api.decode_attn(lay, tabs, q, cache, V, HKV_, out=o, workspace=wsp)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        unit = 4 * lay.words + 4 + 2 * D_ + (4 * (D_ // 32) + 4 if qjl else 0)
+        nbytes = H * N_ * unit
+        ms = float(np.mean(ts))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"GB/s": gbs, "frac": gbs / peak, "ms": ms, "MB": nbytes / 1e6,
+                     "kernel": "tensor-core" if (BITS_ <= 3 and D_ <= 128) else "ffma"}
+        del cache, V
+    return out
+
+
 def run_gpu(args):
     import torch
     from rotation_preconditioned_quantization_b200 import api, inputs
@@ -338,6 +388,7 @@ def run_gpu(args):
     traffic = _ncu_traffic()
     if rank != 0:
         return 0
+    extra = None if args.no_extra else other_workloads(dev, peak)
     line = {
         "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -356,6 +407,7 @@ def run_gpu(args):
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,
+        "other_workloads": extra,
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and ws == 1:
@@ -402,6 +454,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="octopus", choices=["octopus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the decode timings of the other workload shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -23,21 +23,33 @@ static int sm_count() {
   return sms;
 }
 
-// Split the cache of each head into n_splits contiguous slices so that the
-// grid (heads x splits) fills the SMs in whole waves: minimise
-// ceil(heads * s / sms) / s over s, slices of at least 256 keys.
-static void choose_splits(int64_t heads, int64_t kv_len, int sms, int& n_splits, int64_t& per) {
-  const int64_t max_s = std::max<int64_t>(1, std::min<int64_t>(1024, (kv_len + 255) / 256));
+// Split the cache of each head into n_splits contiguous slices. A CTA
+// (one per SM) pays a fixed cost (prologue, first data, split merge: about
+// 8 us measured on B200) plus its slice's bytes at about 30 GB/s per SM, and
+// CTAs run in waves of the SM count; pick the split count that minimises
+//   waves(s) * (fixed + (kv_len / s) * unit_bytes / per_sm_rate).
+// Slices start at multiples of 64 keys (whole rounds of the kernels).
+static void choose_splits(int64_t heads, int64_t kv_len, int sms, int64_t unit_bytes, int& n_splits,
+                          int64_t& per) {
+  constexpr double kFixedUs = 8.0, kBytesPerUs = 30.0e3;
+  const int64_t max_s = std::max<int64_t>(1, std::min<int64_t>(1024, (kv_len + 63) / 64));
   double best = 1e300;
   int64_t best_s = 1;
   for (int64_t s = 1; s <= max_s; ++s) {
     const int64_t waves = (heads * s + sms - 1) / sms;
-    const double cost = static_cast<double>(waves) / s + 1e-4 * s;  // tiny bias against needless splits
-    if (cost < best - 1e-12) { best = cost; best_s = s; }
+    const double keys = static_cast<double>((kv_len + s - 1) / s);
+    const double cost = static_cast<double>(waves) * (kFixedUs + keys * static_cast<double>(unit_bytes) / kBytesPerUs);
+    if (cost < best * (1.0 - 1e-9)) { best = cost; best_s = s; }
   }
   per = (kv_len + best_s - 1) / best_s;
-  per = ((per + 63) / 64) * 64;  // slices start at multiples of 64 keys (16-byte aligned copies)
+  per = ((per + 63) / 64) * 64;
   n_splits = static_cast<int>(std::max<int64_t>(1, (kv_len + per - 1) / per));
+}
+
+// Bytes one (token, KV head) costs decode: code words, gamma, V row (and
+// the sketch words and residual norm).
+static int64_t unit_bytes(const octo_layout* L) {
+  return 4 * L->words + 4 + 2 * L->d + (L->qjl ? 4 * (L->d / 32) + 4 : 0);
 }
 
 static int rows_template(int Gq) { return Gq <= 1 ? 1 : (Gq <= 4 ? 4 : 8); }
@@ -149,7 +161,8 @@ extern "C" size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq
   const int G = octo::rows_template(Gq);
   int n_splits;
   int64_t per;
-  octo::choose_splits(static_cast<int64_t>(B) * Hkv, std::max<int64_t>(kv_len, 1), octo::sm_count(), n_splits, per);
+  octo::choose_splits(static_cast<int64_t>(B) * Hkv, std::max<int64_t>(kv_len, 1), octo::sm_count(), octo::unit_bytes(L),
+                      n_splits, per);
   return ws_layout(static_cast<int64_t>(B) * Hkv, n_splits, G, L->d).total;
 }
 
@@ -212,7 +225,7 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.table_heads = tab->n_heads;
   const int G = octo::rows_template(Gq);
 
-  octo::choose_splits(heads, kv_len, octo::sm_count(), a.n_splits, a.keys_per_split);
+  octo::choose_splits(heads, kv_len, octo::sm_count(), octo::unit_bytes(L), a.n_splits, a.keys_per_split);
   const WsLayout w = ws_layout(heads, a.n_splits, G, D);
   if (ws_bytes < w.total) return OCTO_EWORKSPACE;
   char* base = static_cast<char*>(workspace);

@@ -59,9 +59,9 @@ def test_static_scratch_matches_workspace_entry_point(cuda_ok, B, Hq, Hkv, N):
 
 def test_static_scratch_rejects_sizes_beyond_its_maximum(cuda_ok):
     lay = api.Layout(128, 3)
-    need = api.decode_attn_workspace_bytes(lay, 8, 64, 8, 1, 131072)
-    assert need > 8 << 20
+    # the smallest batch (of 8 KV heads, 8 query rows each, 131072 tokens) whose workspace is over the limit
+    B = next(b for b in (8, 64, 512, 4096) if api.decode_attn_workspace_bytes(lay, b, 64, 8, 1, 131072) > 8 << 20)
     t = _lib.OctoTables(256, 256, 256, 256, 256, None, 8)
-    st = _lib.lib().octo_decode_attn_static(lay.ref, ctypes.byref(t), 256, _lib.BF16, 8, 64, 8, 1, 131072, 131072,
+    st = _lib.lib().octo_decode_attn_static(lay.ref, ctypes.byref(t), 256, _lib.BF16, B, 64, 8, 1, 131072, 131072,
                                             256, 256, None, None, 256, ctypes.c_float(0.1), 256, None, None)
     assert st == _lib.OCTO_EWORKSPACE
