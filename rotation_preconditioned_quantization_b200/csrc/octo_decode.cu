@@ -235,10 +235,10 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.part_l = reinterpret_cast<float*>(base + w.l);
   a.part_o = reinterpret_cast<float*>(base + w.o);
   const dim3 grid(static_cast<unsigned>(a.n_splits), static_cast<unsigned>(heads));
-  // tensor maps for the tensor-core kernel (codes of at most 10 bits, d <= 128)
+  // tensor maps for the tensor-core kernel (d <= 128)
   octo::TmaDesc tm;
   std::memset(&tm, 0, sizeof(tm));
-  if (D <= 128 && 3 * L->b + 1 <= 10 &&
+  if (D <= 128 &&
       !build_maps(tm, L, heads, kv_len, cache_cap, packed, gamma, qjl_bits, qjl_norm, V))
     return OCTO_ECUDA;
   cudaError_t e;

@@ -703,7 +703,7 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core logits (codes of at most 10 bits, i.e. b <= 3, and d <= 128).
+// Tensor-core logits (d <= 128, every bit budget b in {2, 3, 4}).
 //
 // For a GQA group the logits of a tile of keys are a dense contraction,
 // logits[key][row] = sum_c u_hat[key][c] q_rot[row][c], so they run on
@@ -780,7 +780,9 @@ struct TcCfg {
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
   // table over the positive-level quadrant: (m_xi, m_eta, i_rho)
   static constexpr int NE = 1 << (3 * B - 1);
-  static constexpr int REP = 8;              // replicas (distinct bank groups per quarter-warp)
+  // replicas: 8 give every lane of a quarter-warp its own bank group (no
+  // conflicts); the 2048-entry b = 4 table keeps 2 to stay in shared memory
+  static constexpr int REP = NE <= 256 ? 8 : 2;
   static constexpr int NKS = (T + 3) / 4;    // logit k-steps (4 triplets each)
   static constexpr bool HL = G <= 4;         // hi and lo halves side by side in the MMA columns
   static constexpr int NB = HL ? 2 : 4;      // query B-fragment registers per k-step
@@ -789,7 +791,7 @@ struct TcCfg {
   static constexpr int QKS = D / 16;         // sketch k-steps
   static constexpr int NWARP = OCTO_DECODE_TC_WARPS;   // consumer warps
   static constexpr int THREADS = 32 * (NWARP + 1);     // + the producer warp
-  static constexpr int NS = OCTO_DECODE_TC_STAGES;
+  static constexpr int NS_MAX = OCTO_DECODE_TC_STAGES;
   static constexpr int RK = kTcRoundKeys;    // keys per round
   static constexpr int MT = D / 16, NCH = D / 64;
   // one stage: V (NCH swizzled boxes of RK rows x 128 bytes), per-warp code
@@ -809,17 +811,22 @@ struct TcCfg {
   static constexpr size_t SCRATCH = (sizeof(float) * G * (QROW + (QJL ? D : 0)) + 15) / 16 * 16;
   static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per consumer warp
   // offsets from a 1024-byte aligned base
+  static constexpr size_t BUDGET = 227 * 1024 - 2048;
+  // shared memory without the stages (+ alignment slack)
+  static constexpr size_t REST = NWARP * PBUF + TABLE + SCRATCH + 1024;
+  // as many stages as fit, up to NS_MAX
+  static constexpr int NS = REST + size_t(NS_MAX) * STAGE <= BUDGET ? NS_MAX
+                            : REST + 3 * size_t(STAGE) <= BUDGET ? 3 : 2;
   static constexpr size_t SREG = 0;                                  // [NS] stages
   static constexpr size_t PREG = SREG + size_t(NS) * STAGE;          // [NWARP] P
   static constexpr size_t TREG = PREG + NWARP * PBUF;                // table
   static constexpr size_t QREG = TREG + TABLE;                       // query scratch
-  static constexpr size_t BUDGET = 227 * 1024 - 2048;
   static constexpr size_t SMEM = QREG + SCRATCH + 1024;              // + alignment slack
-  static constexpr bool FITS = SMEM <= BUDGET;
+  static constexpr bool FITS = SMEM <= BUDGET && NWARP >= G;  // (one warp per query row in the prologue)
   static constexpr uint32_t TX_FIXED = (QJL ? 4u * QW * RK + 4u * RK : 0u) + 4u * RK;  // gammas (+ sketch, norms)
   static constexpr uint32_t TX_CHUNK = 4u * W * KW;                                     // one code box
   static_assert(G <= 8 && D <= 128 && NCH >= 1, "tensor-core logits shape");
-  static_assert(NWARP >= 8 && RK <= 256 && NS >= 2, "consumer warps (one per query row), box rows, stages");
+  static_assert(NWARP >= 4 && RK <= 256 && NS >= 2, "consumer warps, box rows, stages");
   static_assert(VHALF % 1024 == 0 && ST_C % 128 == 0 && ST_G % 128 == 0 && ST_Q % 128 == 0 && ST_N % 128 == 0,
                 "alignment of the stage parts");
   static_assert(size_t(NS) * STAGE >= sizeof(float) * NWARP * G * (D + 2), "the warp merge reuses the stages");
@@ -1374,11 +1381,11 @@ cudaError_t launch_decode_d256(const DecodeArgs& a, const TmaDesc& tm, int b, in
 #define OCTO_DECODE_TC 1  // tensor-core logits where the shape allows
 #endif
 
-// The tensor-core kernel takes codes of at most 10 bits (b <= 3), d <= 128,
+// The tensor-core kernel takes d <= 128 (b <= 4),
 // and only shapes whose tables and slots fit in shared memory.
 template <int D, int B, int G, bool QJL>
 constexpr bool tc_fits() {
-  if constexpr (D <= 128 && 3 * B + 1 <= 10) return TcCfg<D, B, G, QJL>::FITS;
+  if constexpr (D <= 128 && B <= 4) return TcCfg<D, B, G, QJL>::FITS;
   else return false;
 }
 
