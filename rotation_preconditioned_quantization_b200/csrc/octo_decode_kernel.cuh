@@ -1334,6 +1334,53 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
   const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
   const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
+  if (S <= 32) {
+    // Up to 32 splits (the usual case), one L2 round trip: every thread
+    // issues the partial-O loads of its (at most) two outputs; meanwhile
+    // warp r forms row r's split weights w_s = 2^(m_s - M) / L in shared
+    // memory (lane s = split s), then the outputs are the weighted sums.
+    float* wsm = reinterpret_cast<float*>(base + Cfg::SREG);  // [G][32] weights (the stages are free)
+    for (int j0 = 0; j0 < a.Gq * D; j0 += 2 * Cfg::THREADS) {
+      float ov[2][32];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int j = j0 + tid + k * Cfg::THREADS;
+        const int r = j < a.Gq * D ? j / D : 0, d = j - r * D;
+#pragma unroll
+        for (int s2 = 0; s2 < 32; ++s2)
+          ov[k][s2] = (j < a.Gq * D && s2 < S) ? __ldcg(bo + (static_cast<int64_t>(s2) * G + r) * D + d) : 0.0f;
+      }
+      if (j0 == 0) {
+        if (warp < a.Gq) {
+          const float m = lane < S ? __ldcg(bm + lane * G + warp) : -INFINITY;
+          const float l = lane < S ? __ldcg(bl + lane * G + warp) : 0.0f;
+          float M = m;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+          const float f = M == -INFINITY || m == -INFINITY ? 0.0f : fast_exp2(m - M);
+          float L = f * l;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+          wsm[warp * 32 + lane] = L > 0.0f ? f / L : 0.0f;
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int j = j0 + tid + k * Cfg::THREADS;
+        if (j >= a.Gq * D) continue;
+        const int r = j / D, d = j - r * D;
+        float o = 0.0f;
+#pragma unroll
+        for (int s2 = 0; s2 < 32; ++s2) o = fmaf(wsm[r * 32 + s2], ov[k][s2], o);
+        const int gi = r / a.Lq, lq = r - gi * a.Lq;
+        const int64_t row = (static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq;
+        a.out[row * D + d] = o;
+      }
+    }
+    if (tid == 0) atomicExch(a.counters + bh, 0);  // ready for the next call
+    return;
+  }
   // Each thread merges its (row, column) outputs over the S split partials,
   // 32 splits per round of independent loads (one L2 round trip per round).
   for (int j = tid; j < a.Gq * D; j += Cfg::THREADS) {
