@@ -238,6 +238,9 @@ OTHER_WORKLOADS = (
 
 
 def other_workloads(dev, peak, iters=6):
+    import torch
+    from rotation_preconditioned_quantization_b200 import api
+
     out = {}
     flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)  # > L2 between timed calls
     for name, B_, HQ_, HKV_, LQ_, D_, BITS_, N_, qjl in OTHER_WORKLOADS:
@@ -272,7 +275,7 @@ def other_workloads(dev, peak, iters=6):
         ms = float(np.mean(ts))
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[name] = {"GB/s": gbs, "frac": gbs / peak, "ms": ms, "MB": nbytes / 1e6,
-                     "kernel": "tensor-core" if (BITS_ <= 3 and D_ <= 128) else "ffma"}
+                     "kernel": "tensor-core" if D_ <= 128 else "ffma"}
         del cache, V
     return out
 
