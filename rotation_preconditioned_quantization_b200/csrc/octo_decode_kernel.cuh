@@ -1192,25 +1192,33 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         lgv[1] = vA ? lgv[1] * a.scale_log2 : -INFINITY;
         lgv[2] = vB ? lgv[2] * a.scale_log2 : -INFINITY;
         lgv[3] = vB ? lgv[3] * a.scale_log2 : -INFINITY;
+        // The reference maximum m of a column only has to bound its logits
+        // loosely (softmax does not depend on it): it is raised to the
+        // chunk's maximum, with a rescale of l and O, only when some logit
+        // exceeds it by more than kSlack (so every p = 2^(s - m) <= 2^kSlack).
+        // Most chunks then skip the cross-lane reduction. The first chunk
+        // always raises it (m = -inf), and it has a valid key on lanes g8 = 0.
+        constexpr float kSlack = 8.0f;
         float mx0 = fmaxf(lgv[0], lgv[2]), mx1 = fmaxf(lgv[1], lgv[3]);
+        if (__any_sync(0xffffffffu, mx0 > m0 + kSlack || mx1 > m1 + kSlack)) {
   #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
-        m0 = n0; m1 = n1;
-        lgv[0] = fast_exp2(lgv[0] - n0); lgv[2] = fast_exp2(lgv[2] - n0);
-        lgv[1] = fast_exp2(lgv[1] - n1); lgv[3] = fast_exp2(lgv[3] - n1);
-        l0 = l0 * al0 + lgv[0] + lgv[2];
-        l1 = l1 * al1 + lgv[1] + lgv[3];
-        if (__any_sync(0xffffffffu, al0 != 1.0f || al1 != 1.0f)) {  // some running max moved
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+          const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);  // m = -inf -> 0
+          m0 = n0; m1 = n1;
+          l0 *= al0; l1 *= al1;
   #pragma unroll
           for (int t = 0; t < MT; ++t) {
             acc_o[t][0] *= al0; acc_o[t][1] *= al1; acc_o[t][2] *= al0; acc_o[t][3] *= al1;
           }
         }
+        lgv[0] = fast_exp2(lgv[0] - m0); lgv[2] = fast_exp2(lgv[2] - m0);
+        lgv[1] = fast_exp2(lgv[1] - m1); lgv[3] = fast_exp2(lgv[3] - m1);
+        l0 += lgv[0] + lgv[2];
+        l1 += lgv[1] + lgv[3];
         // P rows (query-major) for the P.V B fragments: this lane's 2 consecutive keys
         if (owner) {
           if (q0 < G) *reinterpret_cast<float2*>(pw + q0 * PS + 2 * g8) = make_float2(lgv[0], lgv[2]);
