@@ -118,7 +118,7 @@ bool build_maps(octo::TmaDesc& tm, const octo_layout* L, int64_t heads, int64_t 
   std::memset(&tm, 0, sizeof(tm));
   const cuuint64_t kv = static_cast<cuuint64_t>(kv_len), H = static_cast<cuuint64_t>(heads);
   const cuuint64_t row = static_cast<cuuint64_t>(cap) * 4;  // bytes between token rows of a plane
-  const cuuint32_t KW = 16, RK = octo::kTcRoundKeys;
+  const cuuint32_t KW = 16, RK = static_cast<cuuint32_t>(octo::tc_round_keys(L->d, L->b));
   const int W = L->words, QW = L->d / 32, D = L->d;
   {
     const cuuint64_t dims[3] = {kv, static_cast<cuuint64_t>(W), H}, str[2] = {row, row * W};

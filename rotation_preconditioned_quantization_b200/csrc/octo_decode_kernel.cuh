@@ -735,15 +735,24 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // warps release a stage on its empty barrier. The load/store unit then only
 // serves shared-memory reads, and no consumer ever waits on a copy issue.
 // ---------------------------------------------------------------------------
-#ifndef OCTO_DECODE_TC_WARPS
-#define OCTO_DECODE_TC_WARPS 8   // consumer warps per CTA (one 16-key chunk of every round each)
-#endif
 #ifndef OCTO_DECODE_TC_STAGES
-#define OCTO_DECODE_TC_STAGES 4  // rounds in flight (shared-memory stages)
+#define OCTO_DECODE_TC_STAGES 4  // rounds in flight at most (shared-memory stages; fewer when they do not fit)
+#endif
+
+// Consumer warps per CTA (one 16-key chunk of every round each). A warp's
+// chunk is a long dependent sequence (code and table reads, MMAs, softmax,
+// P.V), so more warps hide more of it, as far as the stages still fit.
+// Measured best: 10 for d = 128 with b <= 3 (3 stages), 12 for d = 64, and 8
+// for b = 4, whose 64 KB table leaves room for fewer or smaller stages.
+// OCTO_DECODE_TC_WARPS overrides the choice for every configuration.
+#ifdef OCTO_DECODE_TC_WARPS
+constexpr int tc_warps(int, int) { return OCTO_DECODE_TC_WARPS; }
+#else
+constexpr int tc_warps(int d, int b) { return b >= 4 ? 8 : (d <= 64 ? 12 : 10); }
 #endif
 
 // Keys of one round (the tensor maps' boxes are built for this size).
-constexpr int kTcRoundKeys = 16 * OCTO_DECODE_TC_WARPS;
+constexpr int tc_round_keys(int d, int b) { return 16 * tc_warps(d, b); }
 
 // Tensor maps of one decode call (built on the host; token extents are
 // kv_len, so rows past the end arrive as zeros).
@@ -789,10 +798,10 @@ struct TcCfg {
   static constexpr int KW = 16;              // keys per consumer chunk (one m-tile)
   static constexpr int QW = D / 32;          // sketch words per key
   static constexpr int QKS = D / 16;         // sketch k-steps
-  static constexpr int NWARP = OCTO_DECODE_TC_WARPS;   // consumer warps
+  static constexpr int NWARP = tc_warps(D, B);         // consumer warps
   static constexpr int THREADS = 32 * (NWARP + 1);     // + the producer warp
   static constexpr int NS_MAX = OCTO_DECODE_TC_STAGES;
-  static constexpr int RK = kTcRoundKeys;    // keys per round
+  static constexpr int RK = tc_round_keys(D, B);  // keys per round
   static constexpr int MT = D / 16, NCH = D / 64;
   // one stage: V (NCH swizzled boxes of RK rows x 128 bytes), per-warp code
   // boxes [W][16], gammas, (sketch words [QW][RK], norms); parts 128-byte aligned
