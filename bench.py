@@ -280,6 +280,43 @@ def other_workloads(dev, peak, iters=6):
     return out
 
 
+def dequant_workload(dev, peak, iters=6):
+    """octo_dequant (key reconstruction) of the bench workload's cache
+    (8 KV heads x 32768 tokens, d=128, b=3) into fp32 and bf16 rows.
+    Algorithmic bytes per key: 4W + 4 read, 4d or 2d written."""
+    import torch
+    from rotation_preconditioned_quantization_b200 import api
+
+    lay = api.Layout(D, BITS)
+    H = B * HKV
+    tabs = api.DeviceTables.build(lay, SEED, HKV, device=dev)
+    g = torch.Generator(device=dev).manual_seed(SEED + 5)
+    cache = api.Cache.empty(lay, H, N, dev)
+    cache.packed.random_(generator=g)
+    cache.gamma.uniform_(0.5, 2.0, generator=g)
+    cache.length = N
+    flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)  # > L2 between timed calls
+    out = {}
+    for name, dt, esz in (("f32", torch.float32, 4), ("bf16", torch.bfloat16, 2)):
+        o = torch.empty((H, N, D), dtype=dt, device=dev)
+        ts = []
+        for i in range(iters + 2):
+            flush.sum()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            api.dequant(lay, tabs, cache, out=o)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        nbytes = H * N * (4 * lay.words + 4 + esz * D)
+        ms = float(np.mean(ts))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"GB/s": gbs, "frac": gbs / peak, "ms": ms, "MB": nbytes / 1e6, "Mkeys/s": H * N / (ms * 1e-3) / 1e6}
+    return out
+
+
 def run_gpu(args):
     import torch
     from rotation_preconditioned_quantization_b200 import api, inputs
@@ -392,6 +429,7 @@ def run_gpu(args):
     if rank != 0:
         return 0
     extra = None if args.no_extra else other_workloads(dev, peak)
+    dq = None if args.no_extra else dequant_workload(dev, peak)
     line = {
         "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -411,6 +449,7 @@ def run_gpu(args):
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,
         "other_workloads": extra,
+        "dequant": dq,
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and ws == 1:
@@ -458,11 +497,19 @@ def main():
     ap.add_argument("--impl", default="octopus", choices=["octopus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode timings of the other workload shapes")
+    ap.add_argument("--only", choices=["dequant"], help="time only this kernel on the bench cache (one GPU; prints its JSON)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.only == "dequant":
+        import torch
+
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"dequant": dequant_workload(dev, _peaks()[0])}))
+        return 0
     return run_gpu(args)
 
 

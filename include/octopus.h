@@ -232,6 +232,30 @@ OCTO_API int octo_decode_attn_static(const octo_layout* L, const octo_tables* ta
                                      const void* V, float scale, float* out, float* logits,
                                      octo_stream_t stream);
 
+/* Device. Reconstructs keys from the cache: k_hat = gamma * R^T u_hat
+ * (explainer, "triplet decomposition" steps 1-4 undone, for the codec's
+ * compress-and-reconstruct use). u_hat concatenates rho_hat_i * n_hat_i over
+ * the T triplets (inverse octahedral map of section "octahedral folding"),
+ * padding dropped; R = (1/sqrt(d)) H diag(s_h) is the encoder's rotation, so
+ * k_hat_j = gamma * s_h[j] * (H u_hat)_j / sqrt(d). The QJL sketch, if the
+ * layout keeps one, is not read: it estimates inner products, it does not
+ * correct keys.
+ *   packed, gamma  device cache (layout above), cache_cap tokens per head;
+ *                  tokens [token_offset, token_offset + n_tokens) of each of
+ *                  the first n_heads cache heads are read. Cache head h uses
+ *                  sign row h mod tables->n_heads.
+ *   out            device [n_heads][n_tokens][d], row-major, out_dtype
+ *                  OCTO_F32 or OCTO_BF16 (round to nearest even); 16-byte
+ *                  aligned. Computed in fp32.
+ * Errors: OCTO_EINVAL (NULL pointer, negative sizes, token_offset +
+ * n_tokens > cache_cap, misaligned out, bad out_dtype), OCTO_EUNSUPPORTED
+ * (d or b outside the supported set). n_heads == 0 or n_tokens == 0
+ * launches nothing. */
+OCTO_API int octo_dequant(const octo_layout* L, const octo_tables* tables,
+                          int64_t n_heads, int64_t n_tokens, int64_t cache_cap, int64_t token_offset,
+                          const uint32_t* packed, const float* gamma, void* out, int out_dtype,
+                          octo_stream_t stream);
+
 /* Static string for a status code. */
 OCTO_API const char* octo_status_string(int status);
 

@@ -63,6 +63,9 @@ _SIGS = {
                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_void_p]),
+    "octo_dequant": (ctypes.c_int, [ctypes.POINTER(OctoLayout), ctypes.POINTER(OctoTables), ctypes.c_int64, ctypes.c_int64,
+                                    ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_int, ctypes.c_void_p]),
     "octo_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "octo_abi_version": (ctypes.c_int, []),
 }

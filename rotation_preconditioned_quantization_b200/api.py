@@ -166,6 +166,31 @@ def encode(layout: Layout, tables: DeviceTables, keys: torch.Tensor, cache: Cach
     return cache
 
 
+def dequant(layout: Layout, tables: DeviceTables, cache: Cache, n_tokens: int | None = None, token_offset: int = 0,
+            n_heads: int | None = None, dtype=torch.float32, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Reconstructed keys k_hat = gamma R^T u_hat of tokens [token_offset, token_offset + n_tokens)
+    of the first n_heads cache heads, as [n_heads][n_tokens][d] (float32 or bfloat16).
+
+    n_tokens defaults to ``cache.length - token_offset``, n_heads to all cache heads.
+    """
+    dt = {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16}.get(dtype if out is None else out.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported output dtype {dtype if out is None else out.dtype}")
+    n = cache.length - int(token_offset) if n_tokens is None else int(n_tokens)
+    h = cache.n_heads if n_heads is None else int(n_heads)
+    if h > cache.n_heads:
+        raise ValueError(f"n_heads {h} > cache heads {cache.n_heads}")
+    shape = (h, max(n, 0), layout.d)
+    if out is None:
+        out = torch.empty(shape, dtype=dtype, device=cache.gamma.device)
+    elif tuple(out.shape) != shape or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {shape} tensor")
+    st = _lib.lib().octo_dequant(layout.ref, tables.ref, h, n, cache.cap, int(token_offset), _ptr(cache.packed),
+                                 _ptr(cache.gamma), _ptr(out), dt, _stream_ptr(stream))
+    _lib.check(st, "octo_dequant")
+    return out
+
+
 def decode_attn_workspace_bytes(layout: Layout, B: int, Hq: int, Hkv: int, Lq: int, kv_len: int) -> int:
     return int(_lib.lib().octo_decode_attn_workspace(layout.ref, B, Hq, Hkv, Lq, kv_len))
 

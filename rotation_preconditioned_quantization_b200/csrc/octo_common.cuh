@@ -46,12 +46,11 @@ __device__ __forceinline__ void fwht_warp(float (&v)[E], int lane) {
   }
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
+    // lower lane: v + o, upper lane: o - v, as one fma with a +-1 factor
+    // (the product is exact, so the result is the correctly rounded sum)
+    const float sg = (lane & m) != 0 ? -1.0f : 1.0f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[e], m);
-      v[e] = upper ? (o - v[e]) : (v[e] + o);
-    }
+    for (int e = 0; e < E; ++e) v[e] = fmaf(sg, v[e], __shfl_xor_sync(0xffffffffu, v[e], m));
   }
 }
 

@@ -42,7 +42,7 @@ static void choose_splits(int64_t heads, int64_t kv_len, int sms, int64_t unit_b
     if (cost < best * (1.0 - 1e-9)) { best = cost; best_s = s; }
   }
   per = (kv_len + best_s - 1) / best_s;
-  per = ((per + 63) / 64) * 64;
+  per = ((per + 15) / 16) * 16;  // slices start on 16-key boundaries (the copies need 4)
   n_splits = static_cast<int>(std::max<int64_t>(1, (kv_len + per - 1) / per));
 }
 

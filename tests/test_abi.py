@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_lib.exported_symbols())
-    assert L.octo_abi_version() == 100
+    assert L.octo_abi_version() == 101
 
 
 @pytest.mark.parametrize("d,b", [(64, 2), (64, 4), (128, 3), (128, 4), (256, 2), (256, 4)])
@@ -134,6 +134,30 @@ def test_encode_and_decode_validate_before_launch():
                                 ctypes.c_float(0.1), 16, null, null, 0, null) == _lib.OCTO_EINVAL
     assert lib.octo_decode_attn_workspace(L.ref, 1, 16, 1, 1, 8) == 0
     assert lib.octo_decode_attn_workspace(L.ref, 1, 4, 1, 1, 0) >= 256
+
+
+def test_dequant_validates_before_launch():
+    L = api.Layout(128, 3)
+    lib = _lib.lib()
+    null = None
+    Tf = _lib.OctoTables(16, 16, 16, 16, 16, None, 1)
+
+    def dq(tab=ctypes.byref(Tf), heads=1, n=4, cap=8, off=0, packed=16, gamma=16, out=16, dt=_lib.F32, lay=L):
+        return lib.octo_dequant(lay.ref, tab, heads, n, cap, off, packed, gamma, out, dt, null)
+    assert dq(tab=None) == _lib.OCTO_EINVAL
+    assert dq(tab=ctypes.byref(_lib.OctoTables())) == _lib.OCTO_EINVAL   # tables hold NULL pointers
+    assert dq(off=5) == _lib.OCTO_EINVAL                                  # token_offset + n_tokens > cache_cap
+    assert dq(n=-1) == _lib.OCTO_EINVAL and dq(heads=-1) == _lib.OCTO_EINVAL
+    assert dq(dt=7) == _lib.OCTO_EINVAL                                   # output dtype
+    assert dq(out=24) == _lib.OCTO_EINVAL                                 # out not 16-byte aligned
+    assert dq(packed=null) == _lib.OCTO_EINVAL and dq(gamma=null) == _lib.OCTO_EINVAL and dq(out=null) == _lib.OCTO_EINVAL
+    bad = _lib.OctoLayout()
+    ctypes.memmove(ctypes.byref(bad), L.ref, ctypes.sizeof(bad))
+    bad.words += 1                                                        # a layout that init would not produce
+    assert lib.octo_dequant(ctypes.byref(bad), ctypes.byref(Tf), 1, 4, 8, 0, 16, 16, 16, _lib.F32, null) == _lib.OCTO_EINVAL
+    # nothing to do: no launch, even with NULL buffers
+    assert dq(n=0, packed=null, gamma=null, out=null) == _lib.OCTO_OK
+    assert dq(heads=0, packed=null, gamma=null, out=null) == _lib.OCTO_OK
 
 
 def test_status_strings():

@@ -334,6 +334,50 @@ def test_attention_of_decoded_keys_equals_sdpa_on_materialised_keys():
     assert np.max(np.abs(out - ref)) < 1e-13
 
 
+# ---------------------------------------------------------------- key reconstruction
+@pytest.mark.parametrize("d,b", [(64, 2), (128, 3), (256, 4)])
+def test_decode_keys_matches_library_hadamard(d, b):
+    """k_hat = gamma R^T u_hat with R = (1/sqrt(d)) H diag(s): rebuilt here from
+    scipy's Sylvester Hadamard matrix (independent of the oracle's own H and
+    of the orientation of its rotation matrix)."""
+    import scipy.linalg
+
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    s = tables.rotation_signs(4, d, 1)[0]
+    k = inputs.llm_keys(3, 1, 64, d)[0].astype(np.float64)
+    e = codec.encode(k, s, tb, lay)
+    ur = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, lay)
+    H = scipy.linalg.hadamard(d).astype(np.float64)
+    ref = e.gamma[:, None] * (ur @ H) * s[None, :] / math.sqrt(d)
+    kh = codec.decode_keys(e.gamma, e.i_xi, e.i_eta, e.i_rho, s, tb, lay)
+    assert np.max(np.abs(kh - ref)) < 1e-12 * np.max(np.abs(ref))
+    # and the reconstruction is close to the key (relative MSE of the b-bit codec)
+    rel = np.sum((kh - k) ** 2, axis=1) / np.sum(k ** 2, axis=1)
+    assert np.mean(rel) < {2: 0.12, 3: 0.035, 4: 0.01}[b]
+
+
+def test_decode_keys_norm_is_gamma_times_the_norm_of_the_decoded_triplets():
+    """R is orthogonal and every n_hat is a unit vector, so ||k_hat||^2 =
+    gamma^2 sum_i rho_hat_i^2 over the triplets that survive the padding
+    (only the last one can lose coordinates)."""
+    for d, b in ((64, 2), (128, 4), (256, 3)):
+        lay = codec.Layout(d, b)
+        tb = tables.codebooks(d, b)
+        dc, _, rc, _ = (np.asarray(x, dtype=np.float64) for x in tb)
+        s = tables.rotation_signs(6, d, 1)[0]
+        rng = np.random.default_rng(d + b)
+        n = 50
+        i_xi = rng.integers(0, lay.n_dir, (n, lay.T)); i_eta = rng.integers(0, lay.n_dir, (n, lay.T))
+        i_rho = rng.integers(0, lay.n_rho, (n, lay.T))
+        gamma = rng.uniform(0.5, 3.0, n)
+        kh = codec.decode_keys(gamma, i_xi, i_eta, i_rho, s, tb, lay)
+        keep = 3 * lay.T - d                      # coordinates of the last triplet that are dropped
+        last = codec.oct_inverse(dc[i_xi[:, -1]], dc[i_eta[:, -1]])[:, : 3 - keep]
+        sq = np.sum(rc[i_rho[:, :-1]] ** 2, axis=1) + rc[i_rho[:, -1]] ** 2 * np.sum(last ** 2, axis=1)
+        assert np.allclose(np.sum(kh ** 2, axis=1), gamma ** 2 * sq, rtol=1e-12)
+
+
 # ---------------------------------------------------------------- QJL
 def test_qjl_estimator_is_unbiased_over_seeds():
     """[EXPL] "optional residual correction": the sketch makes the inner-product estimate unbiased."""
