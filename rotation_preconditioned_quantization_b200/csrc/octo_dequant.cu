@@ -11,17 +11,18 @@
 // gamma * s_j / sqrt(d). The QJL sketch plays no part: it estimates inner
 // products, it does not correct the key.
 //
-// Kernel structure: a persistent grid walks tiles of KT consecutive tokens
-// of one head. Phase 1 stages the tile's code words ([W][KT], token-
+// Kernel structure: each block walks a contiguous range of tiles of KT
+// consecutive tokens of one head. A tile's code words ([W][KT], token-
 // contiguous in the cache, so each word plane is one coalesced row) and
-// gammas in shared memory; it is issued one tile ahead, into registers, so
-// the loads overlap the previous tile's work. Phase 2 runs one thread per (key, triplet) over
-// the tile and writes the decoded triplet into the key's shared-memory row;
-// decoded triplets of the positive-level quadrant come from a replicated
-// table and the code's two direction signs flip x and y. Phase 3 runs one
-// warp per key: d/32 coordinates per lane, butterflies, scale, one vector
-// store per lane (fp32 or bf16 rows). The output bytes dominate the
-// traffic (4d or 2d bytes per key against 4W + 4 read).
+// gammas are staged in shared memory by asynchronous copies, one tile ahead
+// (two buffers). A key is handled by d/32 lanes, each owning 32 consecutive
+// coordinates: the lane decodes the 12 triplets that cover them straight
+// into registers (codes from a window of the key's words; decoded triplets
+// of the positive-level quadrant from a replicated table, the code's two
+// direction signs flipping x and y), runs 5 butterfly stages in registers
+// and the remaining log2(d/32) across its lanes, scales and stores its 32
+// outputs (fp32 or bf16). The output bytes dominate the traffic (4d or 2d
+// bytes per key against 4W + 4 read).
 
 #include <cuda_runtime.h>
 
@@ -39,6 +40,7 @@ struct DequantArgs {
   const float* signs;
   void* out;
   int out_bf16;
+  int out_v8;  // out is 32-byte aligned: 32-byte stores (whole sectors per lane)
   int64_t n_heads, n_tokens, cache_cap, token_offset, table_heads;
   int64_t tiles_per_head, n_tiles;
 };
@@ -50,38 +52,64 @@ struct DqCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr int NE = 1 << (3 * B - 1);  // positive quadrant: (m_xi, m_eta, i_rho)
-  static constexpr int REP = NE <= 256 ? 8 : 2;  // replicas: lanes of a quarter-warp in distinct bank groups
-  static constexpr int E = D / 32;               // coordinates per lane in phase 3
-  static constexpr int KT = 64;                  // keys per tile
-  static constexpr int US = (3 * T + 3) / 4 * 4;  // row stride of the decoded directions (floats, 16-byte rows)
-  static constexpr int THREADS = 256;
-  static constexpr int NWARP = THREADS / 32;
+  static constexpr int NE = 1 << (3 * B - 1);      // positive quadrant: (m_xi, m_eta, i_rho)
+  static constexpr int REP = NE <= 256 ? 8 : 2;    // replicas: lanes of a quarter-warp in distinct bank groups
+  static constexpr int LK = D / 32;                // lanes per key, 32 coordinates each
+  static constexpr int LKB = LK == 2 ? 1 : (LK == 4 ? 2 : 3);
+  static constexpr int KW = 32 / LK;               // keys per warp and pass
+  static constexpr int THREADS = 256, NWARP = THREADS / 32;
+  static constexpr int KT = 128;                   // keys per tile
+  static constexpr int PASSES = KT / (NWARP * KW);
+  // A lane decodes the NT triplets from floor(32 j / 3) on: 36 coordinates,
+  // which hold its 32 at any offset 0..2. Their codes lie in a window of NWL
+  // words (one more than the last code's first word, for its upper bits).
+  static constexpr int NT = 12;
+  static constexpr int NWL = ((NT - 1) * C) / 32 + 3;
+  static constexpr int WMAX = ((32 * (LK - 1) / 3) * C) / 32 + NWL;  // end of the last lane's window
+  static constexpr int WP = WMAX > W ? WMAX : W;   // word planes held; planes >= W stay zero
+  static constexpr int CS = KT + 1;                // odd plane stride: a key's planes in distinct banks
   static constexpr size_t TABLE = sizeof(float4) * NE * REP;
-  static constexpr size_t UROWS = sizeof(float) * KT * US;
-  // word planes [W + 1][CS] (+ a zero plane, see phase 2); the odd stride puts
-  // the planes of one key in distinct banks
-  static constexpr int CS = KT + 1;
-  static constexpr size_t CODES = (sizeof(uint32_t) * (W + 1) * CS + 15) / 16 * 16;
-  static constexpr size_t SMEM = TABLE + UROWS + CODES + sizeof(float) * KT;
-  static_assert(TABLE % 16 == 0 && UROWS % 16 == 0 && CODES % 16 == 0, "16-byte aligned parts");
+  static constexpr size_t CBUF = (sizeof(uint32_t) * WP * CS + 15) / 16 * 16;
+  static constexpr size_t SMEM = TABLE + 2 * CBUF + 2 * sizeof(float) * KT;  // two tile buffers
+  static_assert(PASSES * NWARP * KW == KT && NT * 3 >= 32 + 2, "tile and lane coverage");
+  static_assert(TABLE % 16 == 0, "16-byte aligned parts");
 };
 
+// 4-byte asynchronous global -> shared copy; bytes = 0 writes a zero.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(bytes)
+               : "memory");
+}
+// 32-byte global store (sm_100): eight 32-bit words, 32-byte aligned address.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
 template <int D, int B>
-__global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
+__global__ void __launch_bounds__(256, 3) dequant_kernel(DequantArgs a) {
   using Cfg = DqCfg<D, B>;
-  constexpr int T = Cfg::T, C = Cfg::C, W = Cfg::W, E = Cfg::E, KT = Cfg::KT, US = Cfg::US, CS = Cfg::CS;
-  constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, THREADS = Cfg::THREADS;
-  constexpr uint32_t HALF = 1u << B;
+  constexpr int C = Cfg::C, W = Cfg::W, KT = Cfg::KT, CS = Cfg::CS, LK = Cfg::LK, LKB = Cfg::LKB, KW = Cfg::KW;
+  constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, THREADS = Cfg::THREADS, NT = Cfg::NT;
+  constexpr int NWL = Cfg::NWL, WP = Cfg::WP;
+  constexpr uint32_t HALF = 1u << B, CM = (1u << C) - 1u;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float4* table = reinterpret_cast<float4*>(smem_raw);                                  // [NE][REP]
-  float* U = reinterpret_cast<float*>(smem_raw + Cfg::TABLE);                           // [KT][US]
-  uint32_t* cw = reinterpret_cast<uint32_t*>(smem_raw + Cfg::TABLE + Cfg::UROWS);       // [W + 1][CS]
-  float* gs = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + Cfg::UROWS + Cfg::CODES);  // [KT]
+  float4* table = reinterpret_cast<float4*>(smem_raw);  // [NE][REP]
+  uint32_t* cwb = reinterpret_cast<uint32_t*>(smem_raw + Cfg::TABLE);  // [2][WP][CS]
+  float* gsb = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + 2 * Cfg::CBUF);  // [2][KT]
   __shared__ float s_dir_c[32], s_rho_c[8];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = lane & (LK - 1);  // this lane's coordinates: [32 j, 32 j + 32) of its key
+  const int t0 = (32 * j) / 3, roff = 32 * j - 3 * t0;  // first triplet; its offset before 32 j (0..2)
+  const int wa = (t0 * C) >> 5, boff = (t0 * C) & 31;  // code window: first word, bit offset in it
+
   if (tid < Cfg::NDIR) s_dir_c[tid] = a.dir_c[tid];
   if (tid < Cfg::NRHO) s_rho_c[tid] = a.rho_c[tid];
   __syncthreads();
@@ -93,130 +121,140 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
 #pragma unroll
     for (int k = 0; k < REP; ++k) table[e * REP + k] = v;
   }
-  // a zero word plane after the last: the code that ends in word W - 1 reads it as its "next" word
-  for (int k = tid; k < KT; k += THREADS) cw[W * CS + k] = 0u;
+  // word planes past the key's last word read as zeros (both buffers)
+  if constexpr (WP > W) {
+    for (int i = tid; i < 2 * (WP - W) * CS; i += THREADS) {
+      const int bb = i / ((WP - W) * CS), r = i - bb * (WP - W) * CS;
+      cwb[bb * (Cfg::CBUF / 4) + W * CS + r] = 0u;
+    }
+  }
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
   const int rep_off = lane & (REP - 1);
-  __syncthreads();
 
-  // Phase 1 for tile tl: this thread's share of the code words (PW of them,
-  // coalesced along the tokens) and one gamma, into registers; stored to
-  // shared memory once the previous tile no longer needs the buffers, so the
-  // loads overlap the previous tile's phases 2 and 3.
-  constexpr int PW = (W * KT + THREADS - 1) / THREADS;
-  uint32_t nw[PW];
-  float ng = 0.0f;
-  auto fetch = [&](int64_t tl) {
-    const int64_t fh = tl / a.tiles_per_head;
-    const int64_t ft0 = (tl - fh * a.tiles_per_head) * KT;
+  // this block's contiguous range of tiles (a head changes rarely along it)
+  const int64_t per = (a.n_tiles + gridDim.x - 1) / gridDim.x;
+  const int64_t tbeg = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t tend = min(a.n_tiles, tbeg + per);
+
+  // tile tl's code words and gammas into buffer bb (cp.async, zero past the end)
+  auto stage = [&](int64_t tl, int bb) {
+    const int64_t h = tl / a.tiles_per_head;
+    const int64_t ft0 = (tl - h * a.tiles_per_head) * KT;
     const int fnk = static_cast<int>(min(static_cast<int64_t>(KT), a.n_tokens - ft0));
-    const uint32_t* ph = a.packed + fh * W * a.cache_cap + a.token_offset + ft0;
-#pragma unroll
-    for (int j = 0; j < PW; ++j) {
-      const int i = tid + j * THREADS, w = i / KT, k = i - w * KT;
-      nw[j] = (i < W * KT && k < fnk) ? __ldg(ph + static_cast<int64_t>(w) * a.cache_cap + k) : 0u;
+    const int64_t tok0 = a.token_offset + ft0;
+    const uint32_t* ph = a.packed + h * W * a.cache_cap + tok0;
+    uint32_t* cw = cwb + bb * (Cfg::CBUF / 4);
+    for (int i = tid; i < W * KT; i += THREADS) {
+      const int w = i / KT, k = i - w * KT;
+      cp_async4(cw + w * CS + k, ph + static_cast<int64_t>(w) * a.cache_cap + min(k, fnk - 1), k < fnk ? 4u : 0u);
     }
-    ng = tid < fnk ? __ldg(a.gamma + fh * a.cache_cap + a.token_offset + ft0 + tid) : 0.0f;
+    if (tid < KT)
+      cp_async4(gsb + bb * KT + tid, a.gamma + h * a.cache_cap + tok0 + min(tid, fnk - 1), tid < fnk ? 4u : 0u);
   };
-  auto stash_words = [&]() {
-#pragma unroll
-    for (int j = 0; j < PW; ++j) {
-      const int i = tid + j * THREADS;
-      if (i < W * KT) cw[(i / KT) * CS + (i % KT)] = nw[j];
-    }
-  };
-  static_assert(KT <= THREADS, "one gamma per thread");
-  if (static_cast<int64_t>(blockIdx.x) < a.n_tiles) {
-    fetch(blockIdx.x);
-    stash_words();
-    if (tid < KT) gs[tid] = ng;
-  }
+
+  uint32_t smask = 0;  // bit p: s_j < 0 for this lane's coordinate 32 j + p, for head sg_head
+  int64_t sg_head = -1;
+  if (tbeg < tend) stage(tbeg, 0);
+  cp_async_commit_wait();
   __syncthreads();
 
-  for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
+  int bb = 0;
+  for (int64_t tile = tbeg; tile < tend; ++tile, bb ^= 1) {
     const int64_t h = tile / a.tiles_per_head;
-    const int64_t t0 = (tile - h * a.tiles_per_head) * KT;  // first token of the tile, from token_offset
-    const int nk = static_cast<int>(min(static_cast<int64_t>(KT), a.n_tokens - t0));
-    const int64_t next = tile + gridDim.x;
-    if (next < a.n_tiles) fetch(next);
-
-    // phase 2: one thread per (key, triplet); code i of a key sits at stream bit i*C
-    for (int i = tid; i < nk * T; i += THREADS) {
-      const int k = i / T, t = i - k * T;
-      const int bit = t * C, w0 = bit >> 5, sh = bit & 31;
-      const uint32_t code = __funnelshift_r(cw[w0 * CS + k], cw[(w0 + 1) * CS + k], sh) & ((1u << C) - 1u);
-      const uint32_t q = (code & ((1u << (2 * B)) - 1u)) | ((code >> (2 * B + 2)) << (2 * B));
-      float4 v = table[q * REP + rep_off];
-      // the codebook is odd-symmetric and the inverse map odd in x and in y
-      v.x = __uint_as_float(__float_as_uint(v.x) ^ (((code >> (2 * B)) & 1u) << 31));
-      v.y = __uint_as_float(__float_as_uint(v.y) ^ (((code >> (2 * B + 1)) & 1u) << 31));
-      float* u = U + k * US + 3 * t;
-      u[0] = v.x;
-      u[1] = v.y;
-      u[2] = v.z;
+    const int64_t t0tok = (tile - h * a.tiles_per_head) * KT;
+    const int nk = static_cast<int>(min(static_cast<int64_t>(KT), a.n_tokens - t0tok));
+    if (tile + 1 < tend) stage(tile + 1, bb ^ 1);  // overlaps this tile's work
+    if (h != sg_head) {
+      const float* srow = a.signs + (h % a.table_heads) * D + 32 * j;
+      smask = 0;
+#pragma unroll
+      for (int p = 0; p < 32; ++p) smask |= (__ldg(srow + p) < 0.0f ? 1u : 0u) << p;
+      sg_head = h;
     }
-    __syncthreads();
-    if (next < a.n_tiles) stash_words();  // phase 3 does not read the words
-
-    // phase 3: one warp per key: H u_hat, then gamma * s_j / sqrt(d)
-    float sg[E];
-    const float* srow = a.signs + (h % a.table_heads) * D + lane * E;
+    const uint32_t* cw = cwb + bb * (Cfg::CBUF / 4);
+    const float* gs = gsb + bb * KT;
+#pragma unroll 1
+    for (int pass = 0; pass < Cfg::PASSES; ++pass) {
+      const int kk = (pass * NWARP + warp) * KW + (lane >> LKB);  // key of this lane's group in the tile
+      // this lane's code window
+      uint32_t wr[NWL];
 #pragma unroll
-    for (int e = 0; e < E; ++e) sg[e] = __ldg(srow + e) * inv_sqrt_d;
-    auto load_row = [&](int k, float (&v)[E]) {
-      const float* u = U + k * US + lane * E;
-      if constexpr (E == 2) {
-        const float2 x = *reinterpret_cast<const float2*>(u);
-        v[0] = x.x; v[1] = x.y;
-      } else {
+      for (int m = 0; m < NWL; ++m) wr[m] = cw[(wa + m) * CS + kk];
+      // decode triplets t0 .. t0 + NT - 1 into v[3 i + c] (coordinate 32 j - roff + 3 i + c)
+      float v[3 * NT];
 #pragma unroll
-        for (int e = 0; e < E; e += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(u + e);
-          v[e] = x.x; v[e + 1] = x.y; v[e + 2] = x.z; v[e + 3] = x.w;
+      for (int i = 0; i < NT; ++i) {
+        const int qi = (i * C) >> 5;                     // word of the code's first bit, without boff
+        const int o = boff + ((i * C) & 31);             // its bit in word qi (may carry into qi + 1)
+        const bool carry = o >= 32;
+        const uint32_t lo = carry ? wr[qi + 1] : wr[qi];
+        const uint32_t hi = carry ? wr[qi + 2] : wr[qi + 1];
+        const uint32_t code = __funnelshift_r(lo, hi, o & 31) & CM;
+        const uint32_t q = (code & ((1u << (2 * B)) - 1u)) | ((code >> (2 * B + 2)) << (2 * B));
+        const float4 e = table[q * REP + rep_off];
+        // the codebook is odd-symmetric and the inverse map odd in x and in y
+        v[3 * i] = __uint_as_float(__float_as_uint(e.x) ^ ((code << (31 - 2 * B)) & 0x80000000u));
+        v[3 * i + 1] = __uint_as_float(__float_as_uint(e.y) ^ ((code << (30 - 2 * B)) & 0x80000000u));
+        v[3 * i + 2] = e.z;
+      }
+      // shift by roff: x[p] = v[p + roff]
+#pragma unroll
+      for (int p = 0; p < 32; ++p) v[p] = roff == 0 ? v[p] : (roff == 1 ? v[p + 1] : v[p + 2]);
+      // H over the 32 register coordinates, then across the LK lanes of the key
+#pragma unroll
+      for (int hh = 1; hh < 32; hh <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if ((e & hh) == 0) {
+            const float x = v[e], y = v[e + hh];
+            v[e] = x + y;
+            v[e + hh] = x - y;
+          }
         }
       }
-    };
-    auto store_row = [&](int k, float (&v)[E]) {
-      const float g = gs[k];
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] *= g * sg[e];
-      const int64_t off = ((h * a.n_tokens + t0 + k) * D) + lane * E;
-      if (a.out_bf16) {
-        uint32_t p[E / 2];
+      for (int m = 1; m < LK; m <<= 1) {
+        const float sgn = (lane & m) != 0 ? -1.0f : 1.0f;
 #pragma unroll
-        for (int e = 0; e < E; e += 2) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[e], v[e + 1]);
-          p[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.out) + off;
-        if constexpr (E == 2) {
-          *reinterpret_cast<uint32_t*>(o) = p[0];
-        } else if constexpr (E == 4) {
-          *reinterpret_cast<uint2*>(o) = make_uint2(p[0], p[1]);
+        for (int e = 0; e < 32; ++e) v[e] = fmaf(sgn, v[e], __shfl_xor_sync(0xffffffffu, v[e], m));
+      }
+      if (kk < nk) {
+        const float g = gs[kk] * inv_sqrt_d;
+        // k_hat_j = gamma s_j (H u_hat)_j / sqrt(d): scale, then the sign bit of s_j
+        auto outv = [&](int p) {
+          return __uint_as_float(__float_as_uint(v[p] * g) ^ ((smask << (31 - p)) & 0x80000000u));
+        };
+        const int64_t off = (h * a.n_tokens + t0tok + kk) * D + 32 * j;
+        uint32_t w[32];  // the 32 outputs as fp32 bits, or packed bf16 pairs in w[0..15]
+        if (a.out_bf16) {
+#pragma unroll
+          for (int p = 0; p < 32; p += 2) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(outv(p), outv(p + 1));
+            w[p / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < E / 2; e += 4)
-            *reinterpret_cast<uint4*>(o + 2 * e) = make_uint4(p[e], p[e + 1], p[e + 2], p[e + 3]);
+          for (int p = 0; p < 32; ++p) w[p] = __float_as_uint(outv(p));
         }
-      } else {
-        float* o = static_cast<float*>(a.out) + off;
-        if constexpr (E == 2) {
-          *reinterpret_cast<float2*>(o) = make_float2(v[0], v[1]);
+        unsigned char* o = static_cast<unsigned char*>(a.out) + off * (a.out_bf16 ? 2 : 4);
+        const int nw = a.out_bf16 ? 16 : 32;
+        if (a.out_v8) {
+#pragma unroll
+          for (int q = 0; q < 32; q += 8) {
+            if (q < nw) {
+              const uint32_t w8[8] = {w[q], w[q + 1], w[q + 2], w[q + 3], w[q + 4], w[q + 5], w[q + 6], w[q + 7]};
+              st_global_v8(o + 4 * q, w8);
+            }
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < E; e += 4)
-            *reinterpret_cast<float4*>(o + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+          for (int q = 0; q < 32; q += 4)
+            if (q < nw) *reinterpret_cast<uint4*>(o + 4 * q) = make_uint4(w[q], w[q + 1], w[q + 2], w[q + 3]);
         }
       }
-    };
-    for (int k = warp; k < nk; k += NWARP) {
-      float v[E];
-      load_row(k, v);
-      fwht_warp<E>(v, lane);
-      store_row(k, v);
     }
-    __syncthreads();  // the rows and gammas are reused by the next tile
-    if (next < a.n_tiles && tid < KT) gs[tid] = ng;
+    cp_async_commit_wait();  // the next tile's words are in
+    __syncthreads();         // and every warp is done with this tile's buffer
   }
 }
 
@@ -275,6 +313,7 @@ extern "C" int octo_dequant(const octo_layout* L, const octo_tables* tab, int64_
   a.signs = tab->signs;
   a.out = out;
   a.out_bf16 = out_dtype == OCTO_BF16;
+  a.out_v8 = reinterpret_cast<uintptr_t>(out) % 32 == 0;
   a.n_heads = n_heads;
   a.n_tokens = n_tokens;
   a.cache_cap = cache_cap;

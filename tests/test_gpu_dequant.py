@@ -86,6 +86,28 @@ def test_dequant_bf16_output_and_head_subset(cuda_ok):
         _check(got[h], _reference(np.float32(e.gamma), e.i_xi, e.i_eta, e.i_rho, signs[h], tb, d, b), bf16=True)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_dequant_output_only_16_byte_aligned(cuda_ok, dtype):
+    """An output that is 16- but not 32-byte aligned takes the 16-byte store path."""
+    d, b, H, N = 128, 3, 2, 150
+    tb = parity.oracle_tables(d, b)
+    signs = tables.rotation_signs(19, d, H)
+    keys = inputs.to_bf16(inputs.llm_keys(20, H, N, d))
+    encs, cache = _oracle_cache(keys, d, b, list(signs), tb, N)
+    esz = 4 if dtype == torch.float32 else 2
+    buf = torch.empty(H * N * d + 32, dtype=dtype, device="cuda")
+    shift = 16 // esz
+    out = buf[shift:shift + H * N * d].view(H, N, d)
+    assert out.data_ptr() % 32 == 16
+    api.dequant(api.Layout(d, b), api.DeviceTables(*tb, signs), cache, out=out)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    for h in range(H):
+        e = encs[h]
+        _check(got[h], _reference(np.float32(e.gamma), e.i_xi, e.i_eta, e.i_rho, signs[h], tb, d, b),
+               bf16=dtype == torch.bfloat16)
+
+
 def test_dequant_ignores_the_qjl_sketch(cuda_ok):
     """A QJL layout reconstructs from the base codes alone: the result equals
     the plain layout's on the same words, whatever the sketch holds."""
