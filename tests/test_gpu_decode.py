@@ -51,12 +51,16 @@ def _oracle_cache(keys, d, b, signs_rows, tb, qjl_S=None, cap=None):
 
 
 def _run_case(B, Hq, Hkv, Lq, d, b, N, qjl=False, q_dtype=torch.bfloat16, cap=None, seed=0, logits_only=False,
-              kv_len=None, check_logits=True):
+              kv_len=None, check_logits=True, key_ramp=0.0):
     tb = parity.oracle_tables(d, b)
     H = B * Hkv
     signs = tables.rotation_signs(seed, d, Hkv)
     S = tables.qjl_matrix(seed + 7, d, Hkv) if qjl else None
-    keys = inputs.to_bf16(inputs.llm_keys(seed + 1, H, N, d))
+    keys = inputs.llm_keys(seed + 1, H, N, d)
+    if key_ramp:
+        # key norms grow along the sequence, so the running maximum of the logits keeps moving
+        keys = keys * (1.0 + key_ramp * np.arange(N, dtype=np.float32) / N)[None, :, None]
+    keys = inputs.to_bf16(keys)
     rows = [signs[h % Hkv] for h in range(H)]
     Srows = [S[h % Hkv] for h in range(H)] if qjl else None
     encs, cache = _oracle_cache(keys, d, b, rows, tb, Srows, cap)
@@ -135,9 +139,42 @@ def test_logits_single_head_4096(cuda_ok):
     dict(B=1, Hq=4, Hkv=1, Lq=1, d=128, b=3, N=300, cap=1000),             # cache larger than kv_len
     dict(B=1, Hq=4, Hkv=1, Lq=1, d=128, b=3, N=1),                         # a single key
     dict(B=3, Hq=4, Hkv=1, Lq=1, d=128, b=2, N=64, kv_len=0),              # empty context
+    dict(B=1, Hq=8, Hkv=1, Lq=1, d=128, b=3, N=2000),                      # 8 rows at d=128 (three products)
+    dict(B=1, Hq=16, Hkv=2, Lq=1, d=128, b=4, N=1500, qjl=True),           # 8 rows, b=4, QJL
+    dict(B=2, Hq=4, Hkv=2, Lq=1, d=128, b=2, N=900),                       # 2 rows in the 4-row layout
+    dict(B=1, Hq=4, Hkv=1, Lq=1, d=128, b=3, N=40000),                     # one head: > 32 slices to merge
+    dict(B=1, Hq=4, Hkv=1, Lq=1, d=128, b=3, N=6000, key_ramp=20.0),       # logits growing along the cache
 ])
 def test_decode_attention_cases(cuda_ok, case):
     _run_case(**case)
+
+
+def test_decode_rescale_when_the_maximum_jumps(cuda_ok):
+    """Keys along the query direction: the first 400 give scaled logits near 0, the rest near 9 (base 2),
+    so the running maximum jumps past the slack once; the earlier keys keep a share of about
+    400 * 2^-9 / 600 of the weight, which a missed or misapplied rescale would multiply by 2^9."""
+    d, b, N, G = 128, 3, 1000, 4
+    tb = parity.oracle_tables(d, b)
+    signs = tables.rotation_signs(21, d, 1)
+    q = inputs.normal(22, (1, 1, 1, d))
+    q = np.repeat(q, G, axis=1)                                   # 4 equal query rows of one KV head
+    qn = q[0, 0, 0] / np.linalg.norm(q[0, 0, 0])
+    noise = inputs.normal(23, (N, d)) * 0.05
+    target = np.where(np.arange(N) < 400, 0.0, 9.0) / (math.log2(math.e) / math.sqrt(d))  # raw logit per key
+    keys = ((target / np.linalg.norm(q[0, 0, 0]))[:, None] * qn[None, :] + noise)[None].astype(np.float32)
+    encs, cache = _oracle_cache(keys, d, b, list(signs), tb)
+    V = inputs.to_bf16(inputs.normal(24, (1, cache.cap, d)))
+    lay = api.Layout(d, b)
+    out, _ = api.decode_attn(lay, api.DeviceTables(*tb, signs), torch.from_numpy(q).cuda(), cache,
+                             torch.from_numpy(V).to(torch.bfloat16).cuda(), 1)
+    torch.cuda.synchronize()
+    e = encs[0]
+    ref, lg = attention.decode_attention(q[0, :, 0].astype(np.float64), e.gamma, e.i_xi, e.i_eta, e.i_rho,
+                                         V[0, :N].astype(np.float64), signs[0], tb, codec.Layout(d, b))
+    w = np.exp((lg[0] - lg[0].max()) / math.sqrt(d))
+    assert 1e-4 < w[:400].sum() / w.sum() < 0.2               # small, but a missed rescale would weigh it 2^9 times
+    got = out[0, :, 0].cpu().numpy()
+    assert np.all(np.abs(got - ref) <= 2e-3 * np.max(np.abs(ref), axis=1, keepdims=True))
 
 
 def test_decode_llm_shaped_full_size(cuda_ok):
