@@ -217,10 +217,14 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       if (!a.joint) {
         rho_level(rho, ir, rh);
       } else {
-        // centre first, then (dx, dy) row-major; replace only on strictly smaller error
-        const float s = nb.x * x + nb.y * y + nb.z * z;
-        rho_level(s, ir, rh);
-        float best = rh * (rh - 2.0f * s);
+        // For a fixed direction n_hat the best norm level is the centroid
+        // nearest s = n_hat . t, and the error is rho^2 + min_l (c_l^2 -
+        // 2 c_l s). Every norm centroid c_l is positive, so that error falls
+        // strictly as s grows: the candidate of least error is the one with
+        // the largest s, and the norm level is searched once, for it.
+        // Centre first, then (dx, dy) row-major; replace only on a strictly
+        // larger s (a strictly smaller error).
+        float sbest = nb.x * x + nb.y * y + nb.z * z;
         const int cx = ix, cy = iy;
 #pragma unroll
         for (int dx = -1; dx <= 1; ++dx) {
@@ -231,13 +235,10 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
             if (ux < 0 || ux >= NDIR || uy < 0 || uy >= NDIR) continue;
             const float4 n = nhat[(ux * NDIR + uy) * REP + rep_off];
             const float sc = n.x * x + n.y * y + n.z * z;
-            int rci;
-            float rr;
-            rho_level(sc, rci, rr);
-            const float err = rr * (rr - 2.0f * sc);
-            if (err < best) { best = err; ix = ux; iy = uy; ir = rci; rh = rr; nb = n; }
+            if (sc > sbest) { sbest = sc; ix = ux; iy = uy; nb = n; }
           }
         }
+        rho_level(sbest, ir, rh);
       }
       codes[k * T + i] = static_cast<uint16_t>(direction_field<B>(ix, iy) | (ir << (2 * Cfg::BD)));
       if constexpr (QJL) {

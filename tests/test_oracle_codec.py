@@ -253,6 +253,32 @@ def test_bit_allocation_sweep(b):
     assert lo - 10 <= 100 * (m[2] / m[0] - 1) <= hi + 10
 
 
+@pytest.mark.parametrize("d,b", [(64, 2), (128, 3), (256, 4)])
+def test_joint_rounding_picks_the_candidate_of_largest_s(d, b):
+    """With every norm centroid positive, the error rho^2 + min_l (c_l^2 - 2 c_l s) falls strictly
+    as s = n_hat . t grows, so the 3x3 search's least-error candidate is the valid neighbour with the
+    largest s (the encoder kernel searches by s and picks the norm level once)."""
+    lay = codec.Layout(d, b)
+    dc, dt, rc, rt = (np.asarray(x, dtype=np.float64) for x in tables.codebooks(d, b))
+    assert np.all(rc > 0)
+    k = inputs.gaussian_keys(31, 1, 200, d)[0].astype(np.float64)
+    t = codec.triplets(codec.rotate(k / np.linalg.norm(k, axis=1, keepdims=True), tables.rotation_signs(3, d, 1)[0]))
+    xi, eta = codec.oct_forward(t)
+    ix0, iy0 = codec.scalar_index(xi, dt), codec.scalar_index(eta, dt)
+    bx, by, br, _ = codec.joint_round(t, ix0, iy0, dc, rc, rt)
+    L = len(dc)
+    best_s = np.full(ix0.shape, -np.inf)
+    sx, sy = ix0.copy(), iy0.copy()
+    for dx, dy in [(0, 0)] + [(a, c) for a in (-1, 0, 1) for c in (-1, 0, 1) if (a, c) != (0, 0)]:
+        ux, uy = ix0 + dx, iy0 + dy
+        ok = (ux >= 0) & (ux < L) & (uy >= 0) & (uy < L)
+        s = np.sum(codec.oct_inverse(dc[np.clip(ux, 0, L - 1)], dc[np.clip(uy, 0, L - 1)]) * t, axis=-1)
+        take = ok & (s > best_s)
+        sx, sy, best_s = np.where(take, ux, sx), np.where(take, uy, sy), np.where(take, s, best_s)
+    assert np.array_equal(sx, bx) and np.array_equal(sy, by)
+    assert np.array_equal(codec.scalar_index(best_s, rt), br)
+
+
 def test_zero_key():
     d, b = 128, 3
     lay = codec.Layout(d, b)
