@@ -59,7 +59,12 @@ struct EncCfg {
   static constexpr int KT = 8192 / D;              // keys per tile
   static constexpr int US = ((3 * T) % 2 == 0) ? 3 * T + 1 : 3 * T;  // odd row stride (floats)
   static constexpr int THREADS = 256;
-  static constexpr int REP = NDIR * NDIR <= 256 ? 8 : 4;  // n_hat replicas (distinct bank groups per quarter-warp)
+  // n_hat replicas (8: distinct bank groups per quarter-warp); 4 from 16
+  // levels per axis on, so that three blocks still fit on an SM
+  static constexpr int REP = NDIR * NDIR <= 64 ? 8 : 4;
+  // the n_hat table has a border of one cell on every side (NaN vectors), so
+  // that the 3x3 neighbourhood of any cell is inside it
+  static constexpr int NB = NDIR + 2;
 };
 
 // Direction field of a triplet code from the ordered cells (ix, iy): the
@@ -84,8 +89,9 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 
   constexpr int REP = Cfg::REP;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float4* nhat = reinterpret_cast<float4*>(smem_raw);                 // [NDIR*NDIR][REP]
-  float* U = reinterpret_cast<float*>(nhat + NDIR * NDIR * REP);      // [KT][US]
+  constexpr int NB = Cfg::NB;
+  float4* nhat = reinterpret_cast<float4*>(smem_raw);                 // [NB*NB][REP], cell (ix, iy) at (ix+1, iy+1)
+  float* U = reinterpret_cast<float*>(nhat + NB * NB * REP);          // [KT][US]
   uint16_t* codes = reinterpret_cast<uint16_t*>(U + KT * US);         // [KT][T]
   __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[8], s_rho_t[8];
 
@@ -97,9 +103,14 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   if (tid < NRHO) s_rho_c[tid] = a.rho_c[tid];
   if (tid < NRHO - 1) s_rho_t[tid] = a.rho_t[tid];
   __syncthreads();
-  for (int e = tid; e < NDIR * NDIR; e += Cfg::THREADS) {
-    const float3 n = oct_inverse(s_dir_c[e / NDIR], s_dir_c[e % NDIR]);
-    const float4 v = make_float4(n.x, n.y, n.z, 0.0f);
+  // a border cell holds NaN: its s = n . t is NaN, and "s > best" is false
+  for (int e = tid; e < NB * NB; e += Cfg::THREADS) {
+    const int bx = e / NB - 1, by = e % NB - 1;
+    float4 v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000), __int_as_float(0x7fc00000), 0.0f);
+    if (bx >= 0 && bx < NDIR && by >= 0 && by < NDIR) {
+      const float3 n = oct_inverse(s_dir_c[bx], s_dir_c[by]);
+      v = make_float4(n.x, n.y, n.z, 0.0f);
+    }
 #pragma unroll
     for (int k = 0; k < REP; ++k) nhat[e * REP + ((k + lane) & (REP - 1))] = v;
   }
@@ -213,7 +224,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       int iy = dir_index(eta);
       int ir;
       float rh;
-      float4 nb = nhat[(ix * NDIR + iy) * REP + rep_off];
+      const float4* nc = nhat + ((ix + 1) * NB + (iy + 1)) * REP + rep_off;  // the centre cell
+      float4 nb = *nc;
       if (!a.joint) {
         rho_level(rho, ir, rh);
       } else {
@@ -223,21 +235,20 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
         // strictly as s grows: the candidate of least error is the one with
         // the largest s, and the norm level is searched once, for it.
         // Centre first, then (dx, dy) row-major; replace only on a strictly
-        // larger s (a strictly smaller error).
+        // larger s (a strictly smaller error). Neighbours outside the
+        // codebook are border cells whose s is NaN and never wins.
         float sbest = nb.x * x + nb.y * y + nb.z * z;
-        const int cx = ix, cy = iy;
+        int kbest = 4;  // (dx + 1) * 3 + (dy + 1)
 #pragma unroll
-        for (int dx = -1; dx <= 1; ++dx) {
-#pragma unroll
-          for (int dy = -1; dy <= 1; ++dy) {
-            if (dx == 0 && dy == 0) continue;
-            const int ux = cx + dx, uy = cy + dy;
-            if (ux < 0 || ux >= NDIR || uy < 0 || uy >= NDIR) continue;
-            const float4 n = nhat[(ux * NDIR + uy) * REP + rep_off];
-            const float sc = n.x * x + n.y * y + n.z * z;
-            if (sc > sbest) { sbest = sc; ix = ux; iy = uy; nb = n; }
-          }
+        for (int k = 0; k < 9; ++k) {
+          if (k == 4) continue;
+          const float4 n = nc[((k / 3 - 1) * NB + (k % 3 - 1)) * REP];
+          const float sc = n.x * x + n.y * y + n.z * z;
+          if (sc > sbest) { sbest = sc; kbest = k; }
         }
+        ix += kbest / 3 - 1;
+        iy += kbest % 3 - 1;
+        if constexpr (QJL) nb = nc[((kbest / 3 - 1) * NB + (kbest % 3 - 1)) * REP];
         rho_level(sbest, ir, rh);
       }
       codes[k * T + i] = static_cast<uint16_t>(direction_field<B>(ix, iy) | (ir << (2 * Cfg::BD)));
@@ -306,7 +317,7 @@ static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
   EncodeArgs a = a0;
   a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
   a.n_tiles = a.tiles_per_head * a.n_heads;
-  const size_t smem = sizeof(float4) * Cfg::NDIR * Cfg::NDIR * Cfg::REP + sizeof(float) * Cfg::KT * Cfg::US +
+  const size_t smem = sizeof(float4) * Cfg::NB * Cfg::NB * Cfg::REP + sizeof(float) * Cfg::KT * Cfg::US +
                       sizeof(uint16_t) * Cfg::KT * Cfg::T;
   auto kern = encode_kernel<D, B, QJL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
