@@ -56,15 +56,23 @@ struct EncCfg {
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
   static constexpr int E = D / 32;                 // coordinates per lane in phase 1
-  static constexpr int KT = 8192 / D;              // keys per tile
   static constexpr int US = ((3 * T) % 2 == 0) ? 3 * T + 1 : 3 * T;  // odd row stride (floats)
   static constexpr int THREADS = 256;
-  // n_hat replicas (8: distinct bank groups per quarter-warp); 4 from 16
-  // levels per axis on, so that three blocks still fit on an SM
-  static constexpr int REP = NDIR * NDIR <= 64 ? 8 : 4;
   // the n_hat table has a border of one cell on every side (NaN vectors), so
   // that the 3x3 neighbourhood of any cell is inside it
   static constexpr int NB = NDIR + 2;
+  // n_hat replicas: 8 put the lanes of a quarter-warp in distinct bank
+  // groups; the 34 x 34 table of b = 4 keeps 4
+  static constexpr int REP = NB * NB * 8 * 16 <= 48 * 1024 ? 8 : 4;
+  static constexpr size_t TABLE = sizeof(float4) * NB * NB * REP;
+  // keys per tile: as many as leave room for BLOCKS blocks per SM (decoded
+  // rows and codes per key), at most 8192 / D, a multiple of the 8 warps
+  static constexpr int BLOCKS = TABLE <= 48 * 1024 ? 3 : 2;
+  static constexpr size_t PER_KEY = sizeof(float) * US + sizeof(uint16_t) * T;
+  static constexpr int KT_FIT = static_cast<int>((227 * 1024 / BLOCKS - 1024 - TABLE) / PER_KEY) / 8 * 8;
+  static constexpr int KT = KT_FIT < 8192 / D ? KT_FIT : 8192 / D;
+  static constexpr size_t SMEM = TABLE + sizeof(float) * KT * US + sizeof(uint16_t) * KT * T;
+  static_assert(KT >= 8, "tile of keys");
 };
 
 // Direction field of a triplet code from the ordered cells (ix, iy): the
@@ -208,7 +216,6 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       const int k = j / T, i = j - k * T;
       float* tp = U + k * US + 3 * i;
       const float x = tp[0], y = tp[1], z = tp[2];
-      const float rho = sqrtf(x * x + y * y + z * z);
       const float l1 = fabsf(x) + fabsf(y) + fabsf(z);
       float px = 0.0f, py = 0.0f, pz = 1.0f;
       if (l1 > 0.0f) {
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       const float4* nc = nhat + ((ix + 1) * NB + (iy + 1)) * REP + rep_off;  // the centre cell
       float4 nb = *nc;
       if (!a.joint) {
-        rho_level(rho, ir, rh);
+        rho_level(sqrtf(x * x + y * y + z * z), ir, rh);  // rho, only scalar rounding uses it
       } else {
         // For a fixed direction n_hat the best norm level is the centroid
         // nearest s = n_hat . t, and the error is rho^2 + min_l (c_l^2 -
@@ -317,8 +324,7 @@ static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
   EncodeArgs a = a0;
   a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
   a.n_tiles = a.tiles_per_head * a.n_heads;
-  const size_t smem = sizeof(float4) * Cfg::NB * Cfg::NB * Cfg::REP + sizeof(float) * Cfg::KT * Cfg::US +
-                      sizeof(uint16_t) * Cfg::KT * Cfg::T;
+  const size_t smem = Cfg::SMEM;
   auto kern = encode_kernel<D, B, QJL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
