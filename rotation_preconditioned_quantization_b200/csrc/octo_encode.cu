@@ -165,34 +165,53 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     float sgn[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) sgn[e] = __ldg(sg + lane * E + e);
-    for (int k = warp; k < nk; k += NWARP) {
+    // This lane's raw words of key k (E bf16 in E/2 words, or E fp32 words).
+    // The next key's words are fetched while the current key is rotated, so a
+    // warp waits for one global load per tile rather than one per key.
+    auto fetch = [&](int k, uint32_t (&r)[E]) {
       const int64_t base = h * a.head_stride + (n0 + k) * a.token_stride + lane * E;
-      float v[E];
       if (a.key_bf16) {
-        const __nv_bfloat16* p = static_cast<const __nv_bfloat16*>(a.keys) + base;
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(a.keys) + base);
         if constexpr (E == 2) {
-          const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p));
-          v[0] = bf16_lo(w); v[1] = bf16_hi(w);
+          r[0] = __ldg(p);
         } else if constexpr (E == 4) {
           const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
-          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+          r[0] = w.x; r[1] = w.y;
         } else {
           const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
-          v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
-          v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+          r[0] = w.x; r[1] = w.y; r[2] = w.z; r[3] = w.w;
         }
       } else {
         const float* p = static_cast<const float*>(a.keys) + base;
         if constexpr (E == 2) {
-          const float2 w = __ldg(reinterpret_cast<const float2*>(p));
-          v[0] = w.x; v[1] = w.y;
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
+          r[0] = w.x; r[1] = w.y;
         } else {
 #pragma unroll
           for (int e = 0; e < E; e += 4) {
-            const float4 w = __ldg(reinterpret_cast<const float4*>(p + e));
-            v[e] = w.x; v[e + 1] = w.y; v[e + 2] = w.z; v[e + 3] = w.w;
+            const uint4 w = __ldg(reinterpret_cast<const uint4*>(p + e));
+            r[e] = w.x; r[e + 1] = w.y; r[e + 2] = w.z; r[e + 3] = w.w;
           }
         }
+      }
+    };
+    uint32_t rn[E];
+    if (warp < nk) fetch(warp, rn);
+    for (int k = warp; k < nk; k += NWARP) {
+      uint32_t rc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) rc[e] = rn[e];
+      if (k + NWARP < nk) fetch(k + NWARP, rn);
+      float v[E];
+      if (a.key_bf16) {
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          v[e] = bf16_lo(rc[e / 2]);
+          v[e + 1] = bf16_hi(rc[e / 2]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = __uint_as_float(rc[e]);
       }
       float ss = 0.0f;
 #pragma unroll
