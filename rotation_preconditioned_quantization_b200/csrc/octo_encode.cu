@@ -55,7 +55,6 @@ struct EncCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr int E = D / 32;                 // coordinates per lane in phase 1
   static constexpr int US = ((3 * T) % 2 == 0) ? 3 * T + 1 : 3 * T;  // odd row stride (floats)
   static constexpr int THREADS = 256;
   // the n_hat table has a border of one cell on every side (NaN vectors), so
@@ -89,10 +88,24 @@ __device__ __forceinline__ uint32_t direction_field(int ix, int iy) {
   return mx | (my << B) | (sx << (2 * B)) | (sy << (2 * B + 1));
 }
 
+// Read-only load of VB bytes (4, 8 or 16; aligned) as 32-bit words.
+template <int VB>
+__device__ __forceinline__ void ld_words(const unsigned char* p, uint32_t* w) {
+  if constexpr (VB == 4) {
+    w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+  } else if constexpr (VB == 8) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = x.x; w[1] = x.y;
+  } else {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+  }
+}
+
 template <int D, int B, bool QJL>
-__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+__global__ void __launch_bounds__(256, 3) encode_kernel(EncodeArgs a) {
   using Cfg = EncCfg<D, B>;
-  constexpr int T = Cfg::T, KT = Cfg::KT, US = Cfg::US, E = Cfg::E, W = Cfg::W, C = Cfg::C;
+  constexpr int T = Cfg::T, KT = Cfg::KT, US = Cfg::US, W = Cfg::W, C = Cfg::C;
   constexpr int NDIR = Cfg::NDIR, NRHO = Cfg::NRHO;
 
   constexpr int REP = Cfg::REP;
@@ -154,79 +167,102 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
 
-  for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
+  // Phase 1 layout: LK = D/32 lanes per key, lane j owning coordinates
+  // [32 j, 32 j + 32): 5 butterfly stages run in registers and log2(LK)
+  // across the key's lanes; a warp holds 32/LK keys at once.
+  constexpr int LK = D / 32, KWP = 32 / LK;
+  const int jq = lane & (LK - 1), kslot = lane / LK;
+  uint32_t smask = 0;  // bit p: s < 0 at coordinate 32 jq + p of head smask_head
+  int64_t smask_head = -1;
+
+  // each block walks a contiguous range of tiles (the head, hence the sign
+  // vector, changes rarely along it)
+  const int64_t per = (a.n_tiles + gridDim.x - 1) / gridDim.x;
+  const int64_t tbeg = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t tend = a.n_tiles < tbeg + per ? a.n_tiles : tbeg + per;
+  for (int64_t tile = tbeg; tile < tend; ++tile) {
     const int64_t h = tile / a.tiles_per_head;
     const int64_t n0 = (tile % a.tiles_per_head) * KT;
     const int nk = static_cast<int>(a.n_tokens - n0 < KT ? a.n_tokens - n0 : KT);
-    const float* sg = a.signs + (h % a.table_heads) * D;
+    if (h != smask_head) {
+      const float* srow = a.signs + (h % a.table_heads) * D + 32 * jq;
+      smask = 0;
+#pragma unroll
+      for (int p = 0; p < 32; ++p) smask |= (__ldg(srow + p) < 0.0f ? 1u : 0u) << p;
+      smask_head = h;
+    }
     __syncthreads();  // previous tile's shared buffers are free
 
-    // ---------------- phase 1: warp per key
-    float sgn[E];
+    // ---------------- phase 1: LK lanes per key
+    // the key's 32 elements of this lane, in loads of the alignment the API
+    // guarantees (min(16, D/32 x element size) bytes)
+    for (int k0 = warp * KWP; k0 < nk; k0 += NWARP * KWP) {
+      const int k = k0 + kslot;
+      const bool valid = k < nk;
+      float v[32];
+      if (!valid) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) sgn[e] = __ldg(sg + lane * E + e);
-    // This lane's raw words of key k (E bf16 in E/2 words, or E fp32 words).
-    // The next key's words are fetched while the current key is rotated, so a
-    // warp waits for one global load per tile rather than one per key.
-    auto fetch = [&](int k, uint32_t (&r)[E]) {
-      const int64_t base = h * a.head_stride + (n0 + k) * a.token_stride + lane * E;
-      if (a.key_bf16) {
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(a.keys) + base);
-        if constexpr (E == 2) {
-          r[0] = __ldg(p);
-        } else if constexpr (E == 4) {
-          const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
-          r[0] = w.x; r[1] = w.y;
-        } else {
-          const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
-          r[0] = w.x; r[1] = w.y; r[2] = w.z; r[3] = w.w;
+        for (int q = 0; q < 32; ++q) v[q] = 0.0f;
+      } else if (a.key_bf16) {
+        constexpr int VB = (D / 32) * 2 < 16 ? (D / 32) * 2 : 16;
+        const unsigned char* p = reinterpret_cast<const unsigned char*>(
+            static_cast<const __nv_bfloat16*>(a.keys) + h * a.head_stride + (n0 + k) * a.token_stride + 32 * jq);
+        uint32_t w[16];
+#pragma unroll
+        for (int q = 0; q < 64 / VB; ++q) ld_words<VB>(p + q * VB, w + q * (VB / 4));
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          v[2 * q] = bf16_lo(w[q]);
+          v[2 * q + 1] = bf16_hi(w[q]);
         }
       } else {
-        const float* p = static_cast<const float*>(a.keys) + base;
-        if constexpr (E == 2) {
-          const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
-          r[0] = w.x; r[1] = w.y;
-        } else {
+        constexpr int VB = (D / 32) * 4 < 16 ? (D / 32) * 4 : 16;
+        const unsigned char* p = reinterpret_cast<const unsigned char*>(
+            static_cast<const float*>(a.keys) + h * a.head_stride + (n0 + k) * a.token_stride + 32 * jq);
+        uint32_t w[32];
 #pragma unroll
-          for (int e = 0; e < E; e += 4) {
-            const uint4 w = __ldg(reinterpret_cast<const uint4*>(p + e));
-            r[e] = w.x; r[e + 1] = w.y; r[e + 2] = w.z; r[e + 3] = w.w;
-          }
-        }
-      }
-    };
-    uint32_t rn[E];
-    if (warp < nk) fetch(warp, rn);
-    for (int k = warp; k < nk; k += NWARP) {
-      uint32_t rc[E];
+        for (int q = 0; q < 128 / VB; ++q) ld_words<VB>(p + q * VB, w + q * (VB / 4));
 #pragma unroll
-      for (int e = 0; e < E; ++e) rc[e] = rn[e];
-      if (k + NWARP < nk) fetch(k + NWARP, rn);
-      float v[E];
-      if (a.key_bf16) {
-#pragma unroll
-        for (int e = 0; e < E; e += 2) {
-          v[e] = bf16_lo(rc[e / 2]);
-          v[e + 1] = bf16_hi(rc[e / 2]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) v[e] = __uint_as_float(rc[e]);
+        for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(w[q]);
       }
       float ss = 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) ss = fmaf(v[e], v[e], ss);
-      ss = warp_sum(ss);
+      for (int q = 0; q < 32; ++q) ss = fmaf(v[q], v[q], ss);
+#pragma unroll
+      for (int m = 1; m < LK; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
       const float g = sqrtf(ss);
       const float ig = g > 0.0f ? 1.0f / g : 0.0f;
+      // u = k / gamma, then the signs s (exact)
 #pragma unroll
-      for (int e = 0; e < E; ++e) v[e] = v[e] * ig * sgn[e];
-      fwht_warp<E>(v, lane);
-      float* row = U + k * US;
+      for (int q = 0; q < 32; ++q)
+        v[q] = __uint_as_float(__float_as_uint(v[q] * ig) ^ ((smask << (31 - q)) & 0x80000000u));
+      // H: coordinate bits 0-4 in registers, then bits 5.. across the key's lanes
 #pragma unroll
-      for (int e = 0; e < E; ++e) row[lane * E + e] = v[e] * inv_sqrt_d;
-      if (lane < 3 * T - D) row[D + lane] = 0.0f;
-      if (lane == 0) a.gamma[h * a.cache_cap + a.token_offset + n0 + k] = g;
+      for (int hh = 1; hh < 32; hh <<= 1) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          if ((q & hh) == 0) {
+            const float x0 = v[q], x1 = v[q + hh];
+            v[q] = x0 + x1;
+            v[q + hh] = x0 - x1;
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 1; m < LK; m <<= 1) {
+        const float sgn = (lane & m) != 0 ? -1.0f : 1.0f;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = fmaf(sgn, v[q], __shfl_xor_sync(0xffffffffu, v[q], m));
+      }
+      if (valid) {
+        float* row = U + k * US;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) row[32 * jq + q] = v[q] * inv_sqrt_d;
+        if (jq == 0) {
+          for (int q = D; q < 3 * T; ++q) row[q] = 0.0f;  // the zero pad of the last triplet
+          a.gamma[h * a.cache_cap + a.token_offset + n0 + k] = g;
+        }
+      }
     }
     __syncthreads();
 
