@@ -103,7 +103,7 @@ __device__ __forceinline__ void ld_words(const unsigned char* p, uint32_t* w) {
 }
 
 template <int D, int B, bool QJL>
-__global__ void __launch_bounds__(256, 3) encode_kernel(EncodeArgs a) {
+__global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) {
   using Cfg = EncCfg<D, B>;
   constexpr int T = Cfg::T, KT = Cfg::KT, US = Cfg::US, W = Cfg::W, C = Cfg::C;
   constexpr int NDIR = Cfg::NDIR, NRHO = Cfg::NRHO;
@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(EncodeArgs a) {
   float* U = reinterpret_cast<float*>(nhat + NB * NB * REP);          // [KT][US]
   uint16_t* codes = reinterpret_cast<uint16_t*>(U + KT * US);         // [KT][T]
   __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[8], s_rho_t[8];
+  __shared__ uint32_t sketch[QJL ? KT * (D / 32) : 1];  // [KT][D/32] sketch words of the tile (QJL)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NWARP = Cfg::THREADS / 32;
@@ -192,6 +193,8 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(EncodeArgs a) {
       smask_head = h;
     }
     __syncthreads();  // previous tile's shared buffers are free
+    if constexpr (QJL)
+      for (int i = tid; i < KT * (D / 32); i += Cfg::THREADS) sketch[i] = 0u;
 
     // ---------------- phase 1: LK lanes per key
     // the key's 32 elements of this lane, in loads of the alignment the API
@@ -339,35 +342,67 @@ __global__ void __launch_bounds__(256, 3) encode_kernel(EncodeArgs a) {
 
     if constexpr (QJL) {
       // ---------------- phase 4: sketch bits = [ (S e)_r >= 0 ], nu = ||e||
+      // Warp w takes rows [w RW, w RW + RW) of S, lane l the keys l + 32 kk:
+      // one accumulator per (row, key), so each S value loaded feeds KPL
+      // keys and each residual value RW rows. Every sum runs over m in
+      // ascending order, as a plain dot product would.
       constexpr int QW = D / 32;                  // sketch words per key
-      constexpr int KG = (KT + 31) / 32;          // 32-key groups
-      const float* S = a.qjl_S + (h % a.table_heads) * D * D;
-      for (int item = warp; item < QW * KG; item += NWARP) {
-        const int qw = item % QW, kg = item / QW;
-        const int k = kg * 32 + lane;
-        if (k < nk) {
-          const float* e = U + k * US;
-          uint32_t bits = 0;
-          for (int r = 0; r < 32; ++r) {
-            const float4* srow = reinterpret_cast<const float4*>(S + (qw * 32 + r) * D);
-            float acc = 0.0f;
-#pragma unroll 8
-            for (int m4 = 0; m4 < D / 4; ++m4) {
-              const float4 sv = __ldg(srow + m4);
-              acc = fmaf(sv.x, e[4 * m4], acc);
-              acc = fmaf(sv.y, e[4 * m4 + 1], acc);
-              acc = fmaf(sv.z, e[4 * m4 + 2], acc);
-              acc = fmaf(sv.w, e[4 * m4 + 3], acc);
-            }
-            bits |= (acc >= 0.0f ? 1u : 0u) << r;
-          }
-          a.qjl_bits[(h * QW + qw) * a.cache_cap + a.token_offset + n0 + k] = bits;
-          if (qw == 0) {
-            float ss = 0.0f;
-            for (int m = 0; m < D; ++m) ss = fmaf(e[m], e[m], ss);
-            a.qjl_norm[h * a.cache_cap + a.token_offset + n0 + k] = sqrtf(ss);
+      constexpr int RW = D / NWARP;               // rows per warp
+      constexpr int KPL = (KT + 31) / 32;         // keys per lane
+      const float* S = a.qjl_S + (h % a.table_heads) * D * D + warp * RW * D;
+      float acc[RW][KPL];
+#pragma unroll
+      for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int kk = 0; kk < KPL; ++kk) acc[r][kk] = 0.0f;
+      for (int m = 0; m < D; m += 4) {
+        float ev[KPL][4];
+#pragma unroll
+        for (int kk = 0; kk < KPL; ++kk) {
+          const int k = lane + 32 * kk;
+          const float* e = U + (k < nk ? k : 0) * US + m;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ev[kk][i] = e[i];
+        }
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+          const float4 sv = __ldg(reinterpret_cast<const float4*>(S + r * D + m));
+#pragma unroll
+          for (int kk = 0; kk < KPL; ++kk) {
+            float t = acc[r][kk];
+            t = fmaf(sv.x, ev[kk][0], t);
+            t = fmaf(sv.y, ev[kk][1], t);
+            t = fmaf(sv.z, ev[kk][2], t);
+            acc[r][kk] = fmaf(sv.w, ev[kk][3], t);
           }
         }
+      }
+      // this warp's RW bits of each key into the key's sketch words
+      static_assert(32 % RW == 0 || RW % 32 == 0, "rows per warp and sketch words");
+#pragma unroll
+      for (int kk = 0; kk < KPL; ++kk) {
+        const int k = lane + 32 * kk;
+        if (k < nk) {
+#pragma unroll
+          for (int r0 = 0; r0 < RW; r0 += 32) {
+            uint32_t bits = 0;
+#pragma unroll
+            for (int r = r0; r < r0 + 32 && r < RW; ++r) bits |= (acc[r][kk] >= 0.0f ? 1u : 0u) << (r - r0);
+            const int row = warp * RW + r0;  // first sketch row of these bits
+            atomicOr(&sketch[k * QW + row / 32], bits << (row % 32));
+          }
+        }
+      }
+      for (int k = tid; k < nk; k += Cfg::THREADS) {
+        const float* e = U + k * US;
+        float ss = 0.0f;
+        for (int m = 0; m < D; ++m) ss = fmaf(e[m], e[m], ss);
+        a.qjl_norm[h * a.cache_cap + a.token_offset + n0 + k] = sqrtf(ss);
+      }
+      __syncthreads();
+      for (int i = tid; i < nk * QW; i += Cfg::THREADS) {
+        const int qw = i / nk, k = i - qw * nk;
+        a.qjl_bits[(h * QW + qw) * a.cache_cap + a.token_offset + n0 + k] = sketch[k * QW + qw];
       }
     }
   }
