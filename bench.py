@@ -317,6 +317,60 @@ def dequant_workload(dev, peak, iters=6):
     return out
 
 
+def encode_sweep(dev, peak):
+    """Encode throughput sweep: 2^22 fp32 keys ~ N(0,1) (8 heads x 2^19 tokens)
+    streamed into the cache in appends of n ~ U{1..4096} tokens (one encode
+    launch per append, all heads), for d in {64, 128, 256} x b in {2, 3, 4}.
+    Keys are resident on the device; the time is the whole stream (CUDA
+    events), launch gaps included. "Mkeys/s" replays the append stream as
+    one CUDA graph (the GPU-side rate); "Mkeys/s_eager" issues the appends
+    one by one from Python, whose per-call overhead then dominates."""
+    import torch
+    from rotation_preconditioned_quantization_b200 import api, inputs
+
+    H, N = 8, 1 << 19
+    lens = inputs.append_lengths(SEED + 17, N, 1, 4096)
+    out = {}
+    for d in (64, 128, 256):
+        keys = torch.empty((H, N, d), dtype=torch.float32, device=dev)
+        keys.normal_(generator=torch.Generator(device=dev).manual_seed(SEED + d))
+        for b in (2, 3, 4):
+            lay = api.Layout(d, b)
+            tabs = api.DeviceTables.build(lay, SEED, H, device=dev)
+            cache = api.Cache.empty(lay, H, N, dev)
+
+            def stream_appends():
+                cache.length = 0
+                for n in lens:
+                    s = cache.length
+                    api.encode(lay, tabs, keys[:, s:s + n], cache)
+
+            def timed(fn):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize(dev)
+                return e0.elapsed_time(e1)
+
+            timed(stream_appends)  # warm-up (also fills the launch caches)
+            ms_eager = timed(stream_appends)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                stream_appends()
+            graph.replay()
+            torch.cuda.synchronize(dev)
+            ms = timed(graph.replay)
+            nbytes = H * N * (4 * d + 4 * lay.words + 4)
+            out[f"d{d}_b{b}"] = {"Mkeys/s": H * N / (ms * 1e-3) / 1e6, "ms": ms, "appends": len(lens),
+                                 "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peak,
+                                 "Mkeys/s_eager": H * N / (ms_eager * 1e-3) / 1e6}
+            del graph, cache
+        del keys
+    return out
+
+
 def run_gpu(args):
     import torch
     from rotation_preconditioned_quantization_b200 import api, inputs
@@ -430,6 +484,7 @@ def run_gpu(args):
         return 0
     extra = None if args.no_extra else other_workloads(dev, peak)
     dq = None if args.no_extra else dequant_workload(dev, peak)
+    sweep = None if args.no_extra else encode_sweep(dev, peak)
     line = {
         "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -450,6 +505,7 @@ def run_gpu(args):
         "gpu_launches": launches,
         "other_workloads": extra,
         "dequant": dq,
+        "encode_sweep": sweep,
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and ws == 1:
@@ -497,7 +553,8 @@ def main():
     ap.add_argument("--impl", default="octopus", choices=["octopus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode timings of the other workload shapes")
-    ap.add_argument("--only", choices=["dequant"], help="time only this kernel on the bench cache (one GPU; prints its JSON)")
+    ap.add_argument("--only", choices=["dequant", "encode_sweep"],
+                    help="time only this part (one GPU; prints its JSON)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -509,6 +566,13 @@ def main():
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         print(json.dumps({"dequant": dequant_workload(dev, _peaks()[0])}))
+        return 0
+    if args.only == "encode_sweep":
+        import torch
+
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"encode_sweep": encode_sweep(dev, _peaks()[0])}))
         return 0
     return run_gpu(args)
 

@@ -5,11 +5,44 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/octopus.h"
 
 namespace octo {
 
 constexpr int kWarp = 32;
+
+// Launch set-up that does not change between calls of one kernel on one
+// device: the dynamic shared-memory opt-in and the number of blocks that can
+// be resident at once (SMs x blocks per SM). Each launcher keeps one cache per
+// kernel instantiation; the first call on a device fills its entry.
+constexpr int kLaunchCacheDevices = 64;
+struct LaunchCache {
+  std::atomic<int> resident[kLaunchCacheDevices];  // 0: not known yet
+};
+
+template <typename Kern>
+inline cudaError_t launch_setup(Kern kern, LaunchCache& c, int threads, size_t smem, int& resident) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kLaunchCacheDevices;
+  int v = cached ? c.resident[dev].load(std::memory_order_acquire) : 0;
+  if (v == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (e != cudaSuccess) return e;
+    v = sms * (per_sm > 0 ? per_sm : 1);
+    if (cached) c.resident[dev].store(v, std::memory_order_release);
+  }
+  resident = v;
+  return cudaSuccess;
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -17,9 +17,13 @@ namespace octo {
 // host side
 // ---------------------------------------------------------------------------
 static int sm_count() {
+  static std::atomic<int> known[kLaunchCacheDevices];  // 0: not queried yet
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool cached = dev >= 0 && dev < kLaunchCacheDevices;
+  if (cached && (sms = known[dev].load(std::memory_order_relaxed)) > 0) return sms;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  if (cached) known[dev].store(sms, std::memory_order_relaxed);
   return sms;
 }
 

@@ -1458,13 +1458,17 @@ cudaError_t launch_decode_one(const DecodeArgs& a, const TmaDesc& tm, dim3 grid,
   if constexpr (OCTO_DECODE_TC && tc_fits<D, B, G, QJL>()) {
     using Cfg = TcCfg<D, B, G, QJL>;
     auto k = decode_tc_kernel<D, B, G, QJL>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
+    static LaunchCache cache;
+    int resident = 0;
+    const cudaError_t e = launch_setup(k, cache, Cfg::THREADS, Cfg::SMEM, resident);
     if (e != cudaSuccess) return e;
     k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a, tm);  // grid: (splits, heads)
   } else {
     using Cfg = DecCfg<D, B, G, QJL>;
     auto k = decode_kernel<D, B, G, QJL>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
+    static LaunchCache cache;
+    int resident = 0;
+    const cudaError_t e = launch_setup(k, cache, Cfg::THREADS, Cfg::SMEM, resident);
     if (e != cudaSuccess) return e;
     k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a);  // grid: (splits, heads)
   }

@@ -265,14 +265,11 @@ static cudaError_t launch_dequant(const DequantArgs& a0, cudaStream_t st) {
   a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
   a.n_tiles = a.tiles_per_head * a.n_heads;
   auto kern = dequant_kernel<D, B>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(Cfg::SMEM));
+  static LaunchCache cache;
+  int resident = 0;
+  const cudaError_t e = launch_setup(kern, cache, Cfg::THREADS, Cfg::SMEM, resident);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, Cfg::SMEM);
-  if (per_sm < 1) per_sm = 1;
-  const int64_t grid = std::min<int64_t>(a.n_tiles, static_cast<int64_t>(sms) * per_sm);
+  const int64_t grid = std::min<int64_t>(a.n_tiles, resident);
   kern<<<static_cast<unsigned>(grid), Cfg::THREADS, Cfg::SMEM, st>>>(a);
   return cudaGetLastError();
 }

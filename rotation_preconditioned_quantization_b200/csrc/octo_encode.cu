@@ -416,14 +416,11 @@ static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
   a.n_tiles = a.tiles_per_head * a.n_heads;
   const size_t smem = Cfg::SMEM;
   auto kern = encode_kernel<D, B, QJL>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  static LaunchCache cache;
+  int resident = 0;
+  const cudaError_t e = launch_setup(kern, cache, Cfg::THREADS, smem, resident);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::THREADS, smem);
-  if (per_sm < 1) per_sm = 1;
-  const int64_t grid = std::min<int64_t>(a.n_tiles, static_cast<int64_t>(sms) * per_sm);
+  const int64_t grid = std::min<int64_t>(a.n_tiles, resident);
   kern<<<static_cast<unsigned>(grid), Cfg::THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
