@@ -17,7 +17,10 @@
  *  - Return value: OCTO_OK (0) or a negative OCTO_E* status; nothing aborts,
  *    no C++ exception crosses this boundary. octo_status_string() names it.
  *  - The caller owns every buffer. The library allocates and frees no
- *    memory and keeps no state between calls.
+ *    memory and keeps no data between calls. The one exception is
+ *    octo_decode_attn_static's fixed scratch array. Each kernel's launch
+ *    set-up (shared-memory opt-in, blocks resident per SM, SM count) is
+ *    looked up on its first call on a device and reused.
  *  - "device" pointers are CUDA global-memory addresses of the current
  *    device; "host" pointers are ordinary process memory.
  *  - Device entry points are asynchronous on the given stream; they return
