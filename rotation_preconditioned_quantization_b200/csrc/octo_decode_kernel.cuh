@@ -13,8 +13,14 @@
 // Because R is orthogonal, q . k_hat = gamma q_rot . u_rot_hat, so the keys
 // are never inverse-rotated.
 //
-// Structure (one CTA = one KV head x one contiguous slice of the cache,
-// 8 warps, every warp a consumer, thread 0 also the producer):
+// The file holds two kernels. decode_tc_kernel (further below) serves every
+// head dimension up to 128: logits and P.V on tensor cores, whole rounds of
+// keys staged by TMA tensor copies from a producer warp, 8 to 12 consumer
+// warps. decode_kernel, described here, serves d = 256 (where the
+// tensor-core layout does not fit in shared memory):
+//
+// Structure of decode_kernel (one CTA = one KV head x one contiguous slice
+// of the cache, 8 warps, every warp a consumer, thread 0 also the producer):
 //  * The slice is cut into stages of CK = 512 keys. For each stage thread 0
 //    issues TMA bulk copies (cp.async.bulk, completion on an mbarrier) of the
 //    stage's code words and gammas (and sketch words and residual norms)

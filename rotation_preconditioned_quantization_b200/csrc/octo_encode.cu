@@ -11,15 +11,19 @@
 // "optional residual correction") also store sign(S e) and ||e|| for the
 // rotated residual e = u_rot - u_rot_hat.
 //
-// Kernel structure: a persistent grid walks tiles of KT consecutive tokens
-// of one head. Phase 1: one warp per key - coalesced vector loads, norm by
-// warp reduction, sign flip, WHT butterflies in registers + shuffles; the
-// rotated direction goes to shared memory. Phase 2: one thread per triplet
-// over the whole tile (balanced whatever T is) - octahedral map, indexing,
-// joint search against a shared-memory table of decoded unit directions.
-// Phase 3: one thread per (key, word) assembles the packed words and stores
-// them token-contiguously (coalesced). Phase 4 (QJL): one lane per key, one
-// warp per 32 sketch rows.
+// Kernel structure: each block walks a contiguous range of tiles of KT
+// consecutive tokens of one head (KT as large as leaves room for three
+// blocks per SM). Phase 1: d/32 lanes per key, 32 coordinates per lane -
+// vector loads, the norm by a short shuffle reduction, sign flips from a lane
+// bit mask, 5 butterfly stages in registers and the rest across the key's
+// lanes; the rotated direction goes to shared memory. Phase 2: one thread
+// per triplet over the whole tile (balanced whatever T is) - octahedral map,
+// indexing, and the joint search as the largest s = n_hat . t over a
+// bordered shared-memory table of decoded unit directions. Phase 3: one
+// thread per (key, word) assembles the packed words and stores them
+// token-contiguously (coalesced). Phase 4 (QJL): the projection S e
+// register-blocked - each warp d/8 rows of S, each lane a few keys - and the
+// sign bits gathered per key in shared memory.
 
 #include <cuda_runtime.h>
 
