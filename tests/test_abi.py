@@ -136,6 +136,22 @@ def test_encode_and_decode_validate_before_launch():
     assert lib.octo_decode_attn_workspace(L.ref, 1, 4, 1, 1, 0) >= 256
 
 
+def test_decode_size_limits_return_unsupported_before_launch():
+    """B*Hkv is the grid's y extent (at most 65535) and token coordinates of the tensor copies
+    are 32-bit: larger requests are refused before anything touches the GPU."""
+    L = api.Layout(128, 3)
+    lib = _lib.lib()
+    Tf = _lib.OctoTables(16, 16, 16, 16, 16, None, 1)
+
+    def dec(B, Hkv, kv, cap, scale=0.1):
+        return lib.octo_decode_attn(L.ref, ctypes.byref(Tf), 256, 0, B, 4 * Hkv, Hkv, 1, kv, cap, 256, 256, None,
+                                    None, 256, ctypes.c_float(scale), 256, None, 256, 1 << 30, None)
+    assert dec(65536, 1, 8, 8) == _lib.OCTO_EUNSUPPORTED
+    assert dec(4096, 16, 8, 8) == _lib.OCTO_EUNSUPPORTED
+    assert dec(1, 1, 1 << 31, 1 << 31) == _lib.OCTO_EUNSUPPORTED
+    assert dec(1, 1, 8, 8, scale=float("nan")) == _lib.OCTO_EINVAL
+
+
 def test_dequant_validates_before_launch():
     L = api.Layout(128, 3)
     lib = _lib.lib()

@@ -177,6 +177,31 @@ def test_decode_rescale_when_the_maximum_jumps(cuda_ok):
     assert np.all(np.abs(got - ref) <= 2e-3 * np.max(np.abs(ref), axis=1, keepdims=True))
 
 
+def test_decode_identical_keys_give_the_mean_of_v(cuda_ok):
+    """Every key the same: all logits are equal, so the attention output is the plain mean of the
+    V rows (a closed form, checked against numpy's mean as well as the oracle)."""
+    d, b, N = 128, 3, 777
+    tb = parity.oracle_tables(d, b)
+    signs = tables.rotation_signs(25, d, 1)
+    key = inputs.llm_keys(26, 1, 1, d)
+    keys = np.repeat(key, N, axis=1)
+    encs, cache = _oracle_cache(keys, d, b, list(signs), tb)
+    V = inputs.to_bf16(inputs.normal(27, (1, cache.cap, d)))
+    q = inputs.normal(28, (1, 4, 1, d))
+    out, lg = api.decode_attn(api.Layout(d, b), api.DeviceTables(*tb, signs), torch.from_numpy(q).cuda(), cache,
+                              torch.from_numpy(V).to(torch.bfloat16).cuda(), 1, logits=True)
+    torch.cuda.synchronize()
+    mean_v = V[0, :N].astype(np.float64).mean(axis=0)
+    got = out[0, :, 0].cpu().numpy()
+    assert np.all(np.abs(got - mean_v[None, :]) <= 2e-3 * np.max(np.abs(mean_v)))
+    l = lg[0, :, 0].cpu().numpy()
+    assert np.all(l == l[:, :1])  # the same code words give the same logit, bit for bit
+    e = encs[0]
+    ref, _ = attention.decode_attention(q[0, :, 0].astype(np.float64), e.gamma, e.i_xi, e.i_eta, e.i_rho,
+                                        V[0, :N].astype(np.float64), signs[0], tb, codec.Layout(d, b))
+    assert np.allclose(ref, mean_v[None, :], rtol=0, atol=1e-12)
+
+
 def test_decode_llm_shaped_full_size(cuda_ok):
     """B=1, 32 query / 8 KV heads, d=128, 32768 tokens, b=3: every output and logit."""
     _run_case(1, 32, 8, 1, 128, 3, 32768)
