@@ -59,7 +59,12 @@ struct EncCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr int US = ((3 * T) % 2 == 0) ? 3 * T + 1 : 3 * T;  // odd row stride (floats)
+  // row stride of the rotated directions (floats), at least 3T. From d = 128
+  // on it is 4 mod 32, so that 8 rows x 4 consecutive columns (an MMA B
+  // fragment of the sketch projection) hit 32 banks; at d = 64 it is odd, so
+  // that one row per lane (the FMA projection) does.
+  static constexpr int US = D >= 128 ? 3 * T + ((4 - 3 * T) % 32 + 32) % 32
+                                     : ((3 * T) % 2 == 0 ? 3 * T + 1 : 3 * T);
   static constexpr int THREADS = 256;
   // the n_hat table has a border of one cell on every side (NaN vectors), so
   // that the 3x3 neighbourhood of any cell is inside it
@@ -90,6 +95,21 @@ __device__ __forceinline__ uint32_t direction_field(int ix, int iy) {
   const uint32_t mx = (static_cast<uint32_t>(ix) ^ (sx ? ones : 0u)) & (half - 1u);
   const uint32_t my = (static_cast<uint32_t>(iy) ^ (sy ? ones : 0u)) & (half - 1u);
   return mx | (my << B) | (sx << (2 * B)) | (sy << (2 * B + 1));
+}
+
+// x as a tf32 head plus a tf32 remainder (x - head), each in a 32-bit register.
+__device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  const float r = x - __uint_as_float(hi);
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+}
+
+// D += A B for one m16n8k8 tile with tf32 operands and fp32 accumulation.
+__device__ __forceinline__ void mma_tf32_1688(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 // Read-only load of VB bytes (4, 8 or 16; aligned) as 32-bit words.
@@ -346,54 +366,110 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
 
     if constexpr (QJL) {
       // ---------------- phase 4: sketch bits = [ (S e)_r >= 0 ], nu = ||e||
-      // Warp w takes rows [w RW, w RW + RW) of S, lane l the keys l + 32 kk:
-      // one accumulator per (row, key), so each S value loaded feeds KPL
-      // keys and each residual value RW rows. Every sum runs over m in
-      // ascending order, as a plain dot product would.
-      constexpr int QW = D / 32;                  // sketch words per key
-      constexpr int RW = D / NWARP;               // rows per warp
-      constexpr int KPL = (KT + 31) / 32;         // keys per lane
-      const float* S = a.qjl_S + (h % a.table_heads) * D * D + warp * RW * D;
-      float acc[RW][KPL];
-#pragma unroll
-      for (int r = 0; r < RW; ++r)
-#pragma unroll
-        for (int kk = 0; kk < KPL; ++kk) acc[r][kk] = 0.0f;
-      for (int m = 0; m < D; m += 4) {
-        float ev[KPL][4];
-#pragma unroll
-        for (int kk = 0; kk < KPL; ++kk) {
-          const int k = lane + 32 * kk;
-          const float* e = U + (k < nk ? k : 0) * US + m;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ev[kk][i] = e[i];
-        }
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-          const float4 sv = __ldg(reinterpret_cast<const float4*>(S + r * D + m));
-#pragma unroll
-          for (int kk = 0; kk < KPL; ++kk) {
-            float t = acc[r][kk];
-            t = fmaf(sv.x, ev[kk][0], t);
-            t = fmaf(sv.y, ev[kk][1], t);
-            t = fmaf(sv.z, ev[kk][2], t);
-            acc[r][kk] = fmaf(sv.w, ev[kk][3], t);
+      // Tensor cores from d = 128 on; at d = 64 the projection is small and
+      // the register-blocked FMA form is faster.
+      constexpr int QW = D / 32;  // sketch words per key
+      if constexpr (D >= 128) {
+        // P = S E^T for the tile (rows of S x keys) on tensor cores: mma.sync
+        // m16n8k8 with tf32 operands, each operand split into a tf32 head and a
+        // tf32 remainder and three products summed (head.head + head.rem +
+        // rem.head), about 2^-21 of sum |S_rm e_m| from the fp32 result. A warp
+        // takes one 16-row tile of S and a group of up to 4 eight-key tiles; the
+        // S fragments of a k-step serve the whole group.
+        constexpr int MT = D / 16;                  // row tiles of S
+        constexpr int NT = (KT + 7) / 8;            // key tiles
+        constexpr int NGT = 4;                      // key tiles per work item
+        constexpr int NG = (NT + NGT - 1) / NGT;
+        const float* Sh = a.qjl_S + (h % a.table_heads) * D * D;
+        const int g8 = lane >> 2, c4 = lane & 3;
+        for (int item = warp; item < MT * NG; item += NWARP) {
+          const int mt = item % MT, ng = item / MT;
+          float acc[NGT][4];
+  #pragma unroll
+          for (int t = 0; t < NGT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+          const float* s0 = Sh + (16 * mt + g8) * D + c4;  // A rows g8 and g8 + 8, columns c4 and c4 + 4
+  #pragma unroll 2
+          for (int k0 = 0; k0 < D; k0 += 8) {
+            uint32_t ah[4], al[4];
+            tf32_split(__ldg(s0 + k0), ah[0], al[0]);
+            tf32_split(__ldg(s0 + 8 * D + k0), ah[1], al[1]);
+            tf32_split(__ldg(s0 + k0 + 4), ah[2], al[2]);
+            tf32_split(__ldg(s0 + 8 * D + k0 + 4), ah[3], al[3]);
+  #pragma unroll
+            for (int t = 0; t < NGT; ++t) {
+              const int key = (ng * NGT + t) * 8 + g8;   // B column g8: this lane's key of the tile
+              if (ng * NGT + t < NT) {
+                const float* e = U + (key < KT ? key : 0) * US + k0 + c4;
+                uint32_t bh[2], bl[2];
+                tf32_split(e[0], bh[0], bl[0]);
+                tf32_split(e[4], bh[1], bl[1]);
+                mma_tf32_1688(acc[t], al, bh);
+                mma_tf32_1688(acc[t], ah, bl);
+                mma_tf32_1688(acc[t], ah, bh);
+              }
+            }
+          }
+          // rows 16 mt + g8 (+8), keys 8 (ng NGT + t) + 2 c4 (+1)
+  #pragma unroll
+          for (int t = 0; t < NGT; ++t) {
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int row = 16 * mt + g8 + 8 * (i >> 1);
+              const int key = (ng * NGT + t) * 8 + 2 * c4 + (i & 1);
+              if (ng * NGT + t < NT && key < nk && acc[t][i] >= 0.0f)
+                atomicOr(&sketch[key * QW + row / 32], 1u << (row % 32));
+            }
           }
         }
-      }
-      // this warp's RW bits of each key into the key's sketch words
-      static_assert(32 % RW == 0 || RW % 32 == 0, "rows per warp and sketch words");
-#pragma unroll
-      for (int kk = 0; kk < KPL; ++kk) {
-        const int k = lane + 32 * kk;
-        if (k < nk) {
-#pragma unroll
-          for (int r0 = 0; r0 < RW; r0 += 32) {
-            uint32_t bits = 0;
-#pragma unroll
-            for (int r = r0; r < r0 + 32 && r < RW; ++r) bits |= (acc[r][kk] >= 0.0f ? 1u : 0u) << (r - r0);
-            const int row = warp * RW + r0;  // first sketch row of these bits
-            atomicOr(&sketch[k * QW + row / 32], bits << (row % 32));
+      } else {
+        // Warp w takes rows [w RW, w RW + RW) of S, lane l the keys l + 32 kk:
+        // one accumulator per (row, key), so each S value loaded feeds KPL
+        // keys and each residual value RW rows. Every sum runs over m in
+        // ascending order, as a plain dot product would.
+        constexpr int RW = D / NWARP;               // rows per warp
+        constexpr int KPL = (KT + 31) / 32;         // keys per lane
+        const float* S = a.qjl_S + (h % a.table_heads) * D * D + warp * RW * D;
+        float acc[RW][KPL];
+  #pragma unroll
+        for (int r = 0; r < RW; ++r)
+  #pragma unroll
+          for (int kk = 0; kk < KPL; ++kk) acc[r][kk] = 0.0f;
+        for (int m = 0; m < D; m += 4) {
+          float ev[KPL][4];
+  #pragma unroll
+          for (int kk = 0; kk < KPL; ++kk) {
+            const int k = lane + 32 * kk;
+            const float* e = U + (k < nk ? k : 0) * US + m;
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) ev[kk][i] = e[i];
+          }
+  #pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            const float4 sv = __ldg(reinterpret_cast<const float4*>(S + r * D + m));
+  #pragma unroll
+            for (int kk = 0; kk < KPL; ++kk) {
+              float t = acc[r][kk];
+              t = fmaf(sv.x, ev[kk][0], t);
+              t = fmaf(sv.y, ev[kk][1], t);
+              t = fmaf(sv.z, ev[kk][2], t);
+              acc[r][kk] = fmaf(sv.w, ev[kk][3], t);
+            }
+          }
+        }
+        // this warp's RW bits of each key into the key's sketch words
+        static_assert(32 % RW == 0 || RW % 32 == 0, "rows per warp and sketch words");
+  #pragma unroll
+        for (int kk = 0; kk < KPL; ++kk) {
+          const int k = lane + 32 * kk;
+          if (k < nk) {
+  #pragma unroll
+            for (int r0 = 0; r0 < RW; r0 += 32) {
+              uint32_t bits = 0;
+  #pragma unroll
+              for (int r = r0; r < r0 + 32 && r < RW; ++r) bits |= (acc[r][kk] >= 0.0f ? 1u : 0u) << (r - r0);
+              const int row = warp * RW + r0;  // first sketch row of these bits
+              atomicOr(&sketch[k * QW + row / 32], bits << (row % 32));
+            }
           }
         }
       }
