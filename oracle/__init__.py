@@ -24,7 +24,7 @@ cites the passage of the pages it follows, by page and section:
           quantization", arxivlens / chatpaper pages).
 
 Where the pages leave a step open, the reading taken is stated in the
-function's docstring and listed in the design doc.
+function's docstring.
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test in
 ``tests/test_oracle_*.py`` except the QJL sketch for a fixed seed, whose only

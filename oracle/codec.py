@@ -5,7 +5,7 @@ folding" (forward and inverse map), "non-uniform bit allocation" ((b+1, b-1)
 bits) and "joint rounding" (3x3 neighbourhood, rho chosen from s = n_hat . t).
 All arithmetic is float64; indices are int64.
 
-Index layout conventions (readings, listed in the design doc):
+Index layout conventions (readings where the pages leave the layout open):
 * key k (length d) -> gamma = ||k||, u = k / gamma (gamma = 0 gives u = 0);
 * rotated direction u_rot = (1/sqrt(d)) H (s * u), H the Sylvester-ordered
   Walsh-Hadamard matrix, s the per-head sign vector;
