@@ -27,9 +27,11 @@ Where the pages leave a step open, the reading taken is stated in the
 function's docstring.
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test in
-``tests/test_oracle_*.py`` except the QJL sketch for a fixed seed, whose only
-pin is statistical (unbiasedness over seeds): its per-seed values are
-"parity unpinned" beyond that property.
+``tests/test_oracle_*.py``. The QJL sketch is pinned three ways: a worked
+case with a non-symmetric permutation as the projection (orientation of S,
+the sign of a zero projection, the scale), the estimator's unbiasedness over
+seeds, and its closed-form variance over seeds; the projection matrix itself
+is pinned by the generator's published test vector and its moments.
 """
 
 from . import tables, codec, attention, baselines  # noqa: F401

@@ -440,3 +440,54 @@ def test_qjl_pack_round_trip():
     assert w.shape == (5, 4)
     assert np.array_equal(codec.qjl_unpack(w, 128), bits)
     assert int(w[0, 0]) == sum(int(bits[0, j]) << j for j in range(32))
+
+
+def test_qjl_sketch_by_hand_with_a_permutation_projection():
+    """[EXPL] "optional residual correction" / [SUMM] "OCTOPUS-QJL": bit j is
+    the sign of row j of S applied to the residual, a zero projection counts
+    as a 1, and the correction is nu sqrt(pi/2)/m <S q, 2 bits - 1>. S is a
+    permutation that is not symmetric, so S e and S^T e differ."""
+    S = np.zeros((4, 4))
+    for j, t in enumerate((1, 3, 0, 2)):   # row j picks coordinate t
+        S[j, t] = 1.0
+    u_rot = np.array([[0.5, -0.25, 0.0, 0.125]])
+    u_hat = np.array([[0.25, 0.0, 0.0, 0.125]])
+    bits, nu, proj = codec.qjl_encode(u_rot, u_hat, S)
+    # e = (0.25, -0.25, 0, 0); S e = (e1, e3, e0, e2) = (-0.25, 0, 0.25, 0)
+    assert np.array_equal(proj, [[-0.25, 0.0, 0.25, 0.0]])
+    assert np.array_equal(bits, [[0, 1, 1, 1]])
+    assert nu[0] == pytest.approx(math.sqrt(0.125), rel=1e-15)
+    q_rot = np.array([[1.0, 2.0, 3.0, 4.0]])
+    # S q = (2, 4, 1, 3); signs (-1, +1, +1, +1): -2 + 4 + 1 + 3 = 6
+    got = codec.qjl_correction(q_rot, bits, nu, S)
+    assert got.shape == (1, 1)
+    assert got[0, 0] == pytest.approx(6.0 * math.sqrt(0.125) * math.sqrt(math.pi / 2.0) / 4.0, rel=1e-15)
+
+
+def test_qjl_estimator_variance_matches_closed_form():
+    """For one Gaussian row s, Y = nu sqrt(pi/2) (s.q) sign(s.e) has E[Y] = q.e
+    and E[Y^2] = (pi/2) nu^2 |q|^2, so the mean over m independent rows has
+    variance ((pi/2) nu^2 |q|^2 - (q.e)^2) / m. A wrong scale, a dropped nu
+    or a mismatched m moves the sample variance off this value."""
+    d, b = 64, 2
+    lay = codec.Layout(d, b)
+    tb = tables.codebooks(d, b)
+    s = tables.rotation_signs(1, d, 1)[0]
+    k = inputs.gaussian_keys(21, 1, 3, d)[0].astype(np.float64)
+    q = inputs.normal(22, (1, d), np.float64)
+    e = codec.encode(k, s, tb, lay)
+    ur_hat = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, lay)
+    q_rot = codec.rotate(q, s)
+    n_seeds = 3000
+    corr = np.empty((n_seeds, k.shape[0]))
+    for i in range(n_seeds):
+        S = tables.qjl_matrix(50_000 + i, d, 1)[0]
+        bits, nu, _ = codec.qjl_encode(e.u_rot, ur_hat, S)
+        corr[i] = codec.qjl_correction(q_rot, bits, nu, S)[0]
+    res = e.u_rot - ur_hat
+    nu = np.linalg.norm(res, axis=1)
+    qe = (q_rot @ res.T)[0]
+    var = ((math.pi / 2.0) * nu ** 2 * np.sum(q_rot ** 2) - qe ** 2) / d
+    # the sample variance of 3000 draws is within ~3 % (1 sigma) of the true one
+    assert np.all(np.abs(corr.var(axis=0) / var - 1.0) < 0.15)
+    assert np.all(np.abs(corr.mean(axis=0) - qe) < 4.0 * np.sqrt(var / n_seeds))
