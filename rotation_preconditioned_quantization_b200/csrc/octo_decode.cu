@@ -32,7 +32,7 @@ static int sm_count() {
 // 8 us measured on B200) plus its slice's bytes at about 30 GB/s per SM, and
 // CTAs run in waves of the SM count; pick the split count that minimises
 //   waves(s) * (fixed + (kv_len / s) * unit_bytes / per_sm_rate).
-// Slices start at multiples of 64 keys (whole rounds of the kernels).
+// Slices start at multiples of 16 keys (one consumer chunk of the kernels).
 static void choose_splits(int64_t heads, int64_t kv_len, int sms, int64_t unit_bytes, int& n_splits,
                           int64_t& per) {
   constexpr double kFixedUs = 8.0, kBytesPerUs = 30.0e3;
