@@ -237,13 +237,13 @@ OTHER_WORKLOADS = (
 )
 
 
-def other_workloads(dev, peak, iters=6):
+def other_workloads(dev, peak, iters=6, shapes=OTHER_WORKLOADS):
     import torch
     from rotation_preconditioned_quantization_b200 import api
 
     out = {}
     flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)  # > L2 between timed calls
-    for name, B_, HQ_, HKV_, LQ_, D_, BITS_, N_, qjl in OTHER_WORKLOADS:
+    for name, B_, HQ_, HKV_, LQ_, D_, BITS_, N_, qjl in shapes:
         lay = api.Layout(D_, BITS_, qjl=qjl)
         H = B_ * HKV_
         tabs = api.DeviceTables.build(lay, SEED, HKV_, device=dev)
@@ -556,8 +556,12 @@ def main():
     ap.add_argument("--impl", default="octopus", choices=["octopus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the decode timings of the other workload shapes")
-    ap.add_argument("--only", choices=["dequant", "encode_sweep"],
+    ap.add_argument("--only", choices=["dequant", "encode_sweep", "decode_shape"],
                     help="time only this part (one GPU; prints its JSON)")
+    ap.add_argument("--shape", default="llm_decode_large",
+                    help="with --only decode_shape: the other decode workload to time (name prefix)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="with --only decode_shape: replace the workload's batch size (a smaller case to profile)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -569,6 +573,20 @@ def main():
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         print(json.dumps({"dequant": dequant_workload(dev, _peaks()[0])}))
+        return 0
+    if args.only == "decode_shape":
+        import torch
+
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        shapes = [w for w in OTHER_WORKLOADS if w[0].startswith(args.shape)]
+        if len(shapes) != 1:
+            raise SystemExit(f"--shape {args.shape!r} names {len(shapes)} workloads")
+        w = list(shapes[0])
+        if args.batch > 0 and args.batch != w[1]:
+            w[0] = w[0].replace(f"B={w[1]},", f"B={args.batch},")
+            w[1] = args.batch
+        print(json.dumps({"decode_shape": other_workloads(dev, _peaks()[0], shapes=[tuple(w)])}))
         return 0
     if args.only == "encode_sweep":
         import torch
