@@ -181,3 +181,41 @@ def test_status_strings():
         assert _lib.status_string(s).startswith("OCTO_")
     with pytest.raises(_lib.OctoError):
         _lib.check(-1, "x")
+
+
+def _planned_workspace(heads, kv_len, d, words, qjl, G, sms=148):
+    """Workspace bytes for the split count the planner documents: minimise
+    waves(s) * (8 us + keys per slice * unit bytes / 30 GB/s per SM) over
+    s <= min(1024, ceil(kv/64)); slices are rounded up to 16 keys."""
+    unit = 4 * words + 4 + 2 * d + (4 * (d // 32) + 4 if qjl else 0)
+    kv = max(kv_len, 1)
+    best, best_s = None, 1
+    for s in range(1, max(1, min(1024, (kv + 63) // 64)) + 1):
+        waves = (heads * s + sms - 1) // sms
+        cost = waves * (8.0 + ((kv + s - 1) // s) * unit / 30.0e3)
+        if best is None or cost < best * (1.0 - 1e-9):
+            best, best_s = cost, s
+    per = -(-kv // best_s)
+    per = -(-per // 16) * 16
+    n_splits = max(1, -(-kv // per))
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    total = 256 + up(4 * heads) + 2 * up(4 * heads * n_splits * G) + up(4 * heads * n_splits * G * d)
+    return n_splits, total
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,d,b,qjl,kv,G", [
+    (1, 32, 8, 1, 128, 3, False, 32768, 4),    # the LLM decode workload
+    (1, 16, 16, 8, 64, 2, False, 65536, 8),    # video/audio: 8 query tokens per head
+    (8, 32, 8, 1, 128, 4, True, 131072, 4),    # long context with the QJL sketch
+    (8, 32, 8, 1, 128, 3, False, 131072, 4),
+    (1, 4, 1, 1, 256, 2, False, 5, 4),         # fewer keys than one chunk
+    (2, 2, 2, 1, 64, 4, False, 100000, 1),
+])
+def test_split_planner_workspace(B, Hq, Hkv, Lq, d, b, qjl, kv, G):
+    """The host's split plan, seen through the workspace size it asks for
+    (on a machine without a GPU the planner assumes 148 SMs)."""
+    L = api.Layout(d, b, qjl=qjl)
+    n_splits, total = _planned_workspace(B * Hkv, kv, d, L.words, qjl, G)
+    assert _lib.lib().octo_decode_attn_workspace(L.ref, B, Hq, Hkv, Lq, kv) == total
+    if (B, kv) == (1, 32768):
+        assert n_splits == 18  # 8 heads x 18 slices: 144 CTAs, one wave on 148 SMs
