@@ -142,6 +142,38 @@ class Cache:
         return int(self.gamma.shape[0])
 
 
+def _check_cache(layout: Layout, tables: DeviceTables, cache: Cache, heads: int, *others):
+    """The C ABI takes plain pointers, so the shapes and devices it cannot see
+    are checked here: the cache must hold at least ``heads`` heads in the
+    layout's word count (and sketch planes for a QJL layout), contiguous, and
+    the tables and every other tensor must live on the cache's device."""
+    cap = cache.cap
+    if cache.packed.dtype != torch.int32 or cache.gamma.dtype != torch.float32:
+        raise ValueError("cache.packed must be int32 and cache.gamma float32")
+    H = int(cache.gamma.shape[0])
+    if tuple(cache.packed.shape) != (H, layout.words, cap) or not cache.packed.is_contiguous():
+        raise ValueError(f"cache.packed must be a contiguous [{H}][{layout.words}][{cap}] tensor for {layout!r}")
+    if cache.gamma.dim() != 2 or not cache.gamma.is_contiguous():
+        raise ValueError("cache.gamma must be a contiguous [n_heads][cap] tensor")
+    if layout.qjl:
+        qb, qn = cache.qjl_bits, cache.qjl_norm
+        if qb is None or qn is None:
+            raise ValueError("a QJL layout needs a cache with sketch planes (qjl_bits, qjl_norm)")
+        if (qb.dtype != torch.int32 or tuple(qb.shape) != (H, layout.qjl_words, cap) or not qb.is_contiguous()
+                or qn.dtype != torch.float32 or tuple(qn.shape) != (H, cap) or not qn.is_contiguous()):
+            raise ValueError(f"cache sketch planes must be contiguous [{H}][{layout.qjl_words}][{cap}] int32 "
+                             f"and [{H}][{cap}] float32")
+    if heads > H:
+        raise ValueError(f"{heads} heads requested, the cache holds {H}")
+    dev = cache.gamma.device
+    for t in (cache.packed, cache.qjl_bits, cache.qjl_norm, tables.dir_c, tables.rho_c, tables.signs,
+              tables.qjl_S) + others:
+        if t is not None and t.device != dev:
+            raise ValueError(f"a tensor is on device {t.device}, the cache on device {dev}")
+    if layout.qjl and tables.qjl_S is None:
+        raise ValueError("a QJL layout needs tables with the projection matrices (qjl_S)")
+
+
 def encode(layout: Layout, tables: DeviceTables, keys: torch.Tensor, cache: Cache, token_offset: int | None = None,
            stream=None) -> Cache:
     """Encode keys [n_heads][n_tokens][d] (float32 or bfloat16, CUDA) into cache at token_offset.
@@ -158,6 +190,7 @@ def encode(layout: Layout, tables: DeviceTables, keys: torch.Tensor, cache: Cach
         raise ValueError(f"unsupported key dtype {keys.dtype}")
     off = cache.length if token_offset is None else int(token_offset)
     n_heads, n_tok = int(keys.shape[0]), int(keys.shape[1])
+    _check_cache(layout, tables, cache, n_heads, keys)
     st = _lib.lib().octo_encode(layout.ref, tables.ref, _ptr(keys), dt, n_heads, n_tok, keys.stride(0), keys.stride(1),
                                 cache.cap, off, _ptr(cache.packed), _ptr(cache.gamma), _ptr(cache.qjl_bits),
                                 _ptr(cache.qjl_norm), _stream_ptr(stream))
@@ -185,6 +218,7 @@ def dequant(layout: Layout, tables: DeviceTables, cache: Cache, n_tokens: int | 
         out = torch.empty(shape, dtype=dtype, device=cache.gamma.device)
     elif tuple(out.shape) != shape or not out.is_contiguous():
         raise ValueError(f"out must be a contiguous {shape} tensor")
+    _check_cache(layout, tables, cache, h, out)
     st = _lib.lib().octo_dequant(layout.ref, tables.ref, h, n, cache.cap, int(token_offset), _ptr(cache.packed),
                                  _ptr(cache.gamma), _ptr(out), dt, _stream_ptr(stream))
     _lib.check(st, "octo_dequant")
@@ -240,14 +274,22 @@ def decode_attn(layout: Layout, tables: DeviceTables, q: torch.Tensor, cache: Ca
     if scale is None:
         scale = 1.0 / math.sqrt(layout.d)
     if V is not None:
-        if V.dtype != torch.bfloat16 or not V.is_contiguous():
-            raise ValueError("V must be contiguous bfloat16 [B*Hkv][cap][d]")
+        # the kernel steps from head to head by cap rows of V
+        if (V.dtype != torch.bfloat16 or not V.is_contiguous() or V.dim() != 3 or V.shape[0] < B * Hkv
+                or tuple(V.shape[1:]) != (cache.cap, layout.d)):
+            raise ValueError(f"V must be contiguous bfloat16 [B*Hkv][{cache.cap}][{layout.d}] (the cache's capacity)")
         if out is None:
             out = torch.empty((B, Hq, Lq, layout.d), dtype=torch.float32, device=q.device)
+        elif out.dtype != torch.float32 or tuple(out.shape) != (B, Hq, Lq, layout.d) or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous float32 {(B, Hq, Lq, layout.d)} tensor")
     if logits is True:
         logits = torch.empty((B, Hq, Lq, kv), dtype=torch.float32, device=q.device)
     elif logits is False:
         logits = None
+    elif logits is not None and (logits.dtype != torch.float32 or tuple(logits.shape) != (B, Hq, Lq, kv)
+                                 or not logits.is_contiguous()):
+        raise ValueError(f"logits must be a contiguous float32 {(B, Hq, Lq, kv)} tensor")
+    _check_cache(layout, tables, cache, B * Hkv, q, V, out, logits)
     need = decode_attn_workspace_bytes(layout, B, Hq, Hkv, Lq, kv)
     if workspace is None:
         workspace = Workspace(need, q.device)

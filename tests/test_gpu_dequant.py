@@ -45,6 +45,7 @@ def _check(got, ref, bf16=False):
     if bf16:
         tol = tol + 2.0 ** -7 * np.abs(ref)
     err = np.abs(got - ref)
+    tol = np.broadcast_to(tol, err.shape)
     assert np.all(err <= tol), f"max err {err.max():.3e} (tol at argmax {tol.flat[np.argmax(err - tol)]:.3e})"
 
 
