@@ -1,22 +1,32 @@
 """Benchmark of the OCTOPUS codec on B200: encode + fused decode attention.
 
-Workload (one GPU): LLM-shaped decode - batch 1, 32 query heads over 8 KV
-heads (GQA 4), head_dim 128, context 32768, bf16 keys (N(0,1), four outlier
-channels x10, per-token lognormal(0, 0.5) scale), bf16 V and q ~ N(0,1),
-b = 3, joint rounding. One step = encode the prefill cache (8 x 32768 keys)
-+ one fused decode-attention step (32 query heads over the whole cache).
+Headline workload (one GPU, the largest single-GPU decode workload):
+batched long-context decode with OCTOPUS-QJL - batch 8, 32 query heads over
+8 KV heads (GQA 4), head_dim 128, context 131072, bf16 keys (N(0,1), four
+outlier channels x10, per-token lognormal(0, 0.5) scale), bf16 V and q ~
+N(0,1), b = 4 plus the 1-bit residual sign sketch, joint rounding. One step
+= encode the prefill cache (64 x 131072 keys) + one fused decode-attention
+step (256 query heads over the whole cache).
 
 Timing: CUDA events on the launching stream around each kernel; the step
 loop is bracketed by a barrier and a device synchronize; the max over ranks
-is reported. L2 (126 MB): inputs rotate over 3 independent copies of the
-workload (~150 MB each) and each step decodes the cache that the previous
-step encoded, so no decode input was touched within the last ~150 MB of
-traffic. Primary metric: decode-attention achieved HBM GB/s over the
-algorithmic bytes (packed codes + gamma + bf16 V + q + out); encode is
-reported in Mkeys/s.
+is reported. L2 (126 MB): two caches alternate, so each decode reads the
+cache encoded one step earlier (2.95 GB of decode input, far larger than
+L2, with the other cache's encode - 2.15 GB read, 0.8 GB written - in
+between). Primary metric: decode-attention achieved HBM GB/s over the
+algorithmic bytes (packed codes + gamma + sketch words + residual norms +
+bf16 V + q + out); encode is reported in Mkeys/s.
 
-``--impl reference`` times the CPU oracle (the plain float64 restatement of
-the method) on a bounded sample of the same workload instead.
+The other decode workloads (LLM decode at context 32768 with b = 3, the
+video/audio shape with d = 64, b = 2 and 8 query tokens) are timed over
+caches the encoder wrote from keys of their recipe, with L2 flushed (a
+512 MB buffer written) before every timed call.
+
+``--gpus N`` without a launcher starts N ranks itself (one process per GPU,
+each an independent batch, no collective on the data path); under torchrun
+the ranks come from the environment. ``--impl reference`` times the CPU
+oracle (the plain float64 restatement of the method) on a bounded sample of
+the headline workload instead.
 """
 
 from __future__ import annotations
@@ -24,23 +34,37 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import re
+import socket
+import subprocess
 import sys
 import threading
 import time
+from collections import namedtuple
 
 import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-# workload
-B, HQ, HKV, D, N, BITS = 1, 32, 8, 128, 32768, 3
 SEED = 0
 METRIC = "compressed-KV decode-attention HBM GB/s (% of ~8 TB/s); encode Mkeys/s"
-WORKLOAD = "llm-decode: B=1, Hq=32, Hkv=8 (GQA 4), d=128, ctx=32768, bf16 K/V/q, b=3 joint"
+
+Workload = namedtuple("Workload", "name B HQ HKV LQ D BITS N QJL keys")
+QJL_LONG = Workload("qjl_long_context", 8, 32, 8, 1, 128, 4, 131072, True, "llm")
+LLM_DECODE = Workload("llm_decode", 1, 32, 8, 1, 128, 3, 32768, False, "llm")
+VIDEO_AUDIO = Workload("video_audio", 1, 16, 16, 8, 64, 2, 65536, False, "gauss")
+LLM_DECODE_LARGE = Workload("llm_decode_large", 8, 32, 8, 1, 128, 3, 131072, False, "llm")
+HEADLINE = QJL_LONG
+OTHER_WORKLOADS = (LLM_DECODE, VIDEO_AUDIO, LLM_DECODE_LARGE)
+
+
+def describe(w: Workload) -> str:
+    keys = "bf16 keys N(0,1) x 4 outlier channels x10 x per-token lognormal(0,0.5)" if w.keys == "llm" else \
+        "bf16 keys N(0,1)"
+    return (f"{w.name}: B={w.B}, Hq={w.HQ}, Hkv={w.HKV}, Lq={w.LQ}, d={w.D}, ctx={w.N}, b={w.BITS}"
+            f"{' + QJL sketch' if w.QJL else ''}, joint rounding, {keys}, bf16 V/q")
 
 
 def _peaks():
@@ -52,21 +76,33 @@ def _peaks():
     return 6650.0, "fallback"
 
 
-def _bytes_decode(words):
-    units = B * HKV * N
-    per_unit = 4 * words + 4 + 2 * D            # packed words + gamma + bf16 V row
-    return units * per_unit + B * HQ * D * 2 + B * HQ * D * 4   # + q (bf16) + out (fp32)
+def unit_bytes(w: Workload, words: int) -> int:
+    """Decode bytes of one (token, KV head): code words, gamma, bf16 V row (+ sketch words, residual norm)."""
+    return 4 * words + 4 + 2 * w.D + ((4 * (w.D // 32) + 4) if w.QJL else 0)
 
 
-def _bytes_encode(words):
-    return B * HKV * N * (2 * D + 4 * words + 4)
+def decode_bytes(w: Workload, words: int) -> int:
+    units = w.B * w.HKV * w.N
+    return units * unit_bytes(w, words) + w.B * w.HQ * w.LQ * w.D * (2 + 4)   # + q (bf16) + out (fp32)
+
+
+def encode_bytes(w: Workload, words: int) -> int:
+    per = 2 * w.D + 4 * words + 4 + ((4 * (w.D // 32) + 4) if w.QJL else 0)  # bf16 key in; codes, gamma (+ sketch) out
+    return w.B * w.HKV * w.N * per
+
+
+def _cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - non-Linux
+        return os.cpu_count() or 1
 
 
 class ClockSampler:
     """Samples SM clocks and clock-event (throttle) reasons during the timed region.
 
-    Polls NVML every ~1 ms from a thread (the timed region is only tens of
-    milliseconds); falls back to no samples if NVML is unavailable.
+    Polls NVML every ~1 ms from a thread; falls back to no samples if NVML is
+    unavailable.
     """
 
     REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
@@ -136,6 +172,7 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
+# ------------------------------------------------------------------ ranks
 def _dist_init():
     import torch
     import torch.distributed as dist
@@ -165,37 +202,140 @@ def _barrier(ws):
         dist.barrier()
 
 
-def cpu_baseline(kv_heads: int = 1, tokens: int = N):
-    """Time the CPU oracle on a bounded sample: oracle encode + decode attention of
-    ``kv_heads`` KV heads (4 query heads each) over ``tokens`` tokens."""
+def _finish_ranks(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(n: int, argv, timeout_s: float = 1800.0) -> int:
+    """Start ``n`` ranks of this script (one process per GPU, rank r on GPU r)
+    with the rendezvous on 127.0.0.1. Rank 0's output is passed through (it
+    alone prints the JSON line); the others' output is discarded. Returns the
+    largest exit code."""
+    port = _free_port()
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n), LOCAL_WORLD_SIZE=str(n),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        out = None if r == 0 else subprocess.DEVNULL
+        procs.append(subprocess.Popen([sys.executable, os.path.join(ROOT, "bench.py"), *argv], env=env, stdout=out,
+                                      cwd=ROOT))
+    rc = 0
+    deadline = time.time() + timeout_s
+    for p in procs:
+        try:
+            rc = max(rc, p.wait(timeout=max(1.0, deadline - time.time())))
+        except subprocess.TimeoutExpired:
+            p.kill()
+            rc = max(rc, 124)
+    return rc
+
+
+def run_dry(args):
+    """The rank logic without the GPU (a CPU check of the N-rank path): every
+    rank takes its own batch, reports a made-up duration, and rank 0 prints
+    the line with the whole-job units and the max over ranks."""
+    ws, rank, _ = _dist_init()
+    units = HEADLINE.B * HEADLINE.HKV * HEADLINE.N
+    my_ms = 10.0 * (rank + 1)
+    _barrier(ws)
+    worst = _max_over_ranks(my_ms, ws)
+    seeds = [SEED + 1000 * r for r in range(ws)]
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "dry_run": True, "n_gpus": ws, "value": ws * units / worst,
+                          "unit": "units/ms", "max_ms": worst, "scaling": "weak",
+                          "config": {"workload": describe(HEADLINE), "per_rank_seeds": seeds,
+                                     "per_rank": "independent batch per GPU (no collective)"}}))
+    _finish_ranks(ws)
+    return 0
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _oracle_head(job):
+    """Oracle encode + decode attention of one KV head (runs in a worker)."""
+    w, head, tokens, seed, one_thread = job
+    if one_thread:  # a pool worker: one BLAS thread per process
+        try:
+            from threadpoolctl import threadpool_limits
+            threadpool_limits(1)
+        except Exception:
+            pass
     from oracle import attention, codec, tables
     from rotation_preconditioned_quantization_b200 import inputs
+    g = w.HQ // w.HKV
+    tb = tables.as_f32(*tables.codebooks(w.D, w.BITS))
+    lay = codec.Layout(w.D, w.BITS)
+    signs = tables.rotation_signs(SEED, w.D, w.HKV)[head % w.HKV]
+    S = tables.qjl_matrix(SEED + 0x517CC1, w.D, w.HKV)[head % w.HKV] if w.QJL else None
+    if w.keys == "llm":
+        keys = inputs.to_bf16(inputs.llm_keys(seed + 1, 1, tokens, w.D))[0]
+    else:
+        keys = inputs.to_bf16(inputs.gaussian_keys(seed + 1, 1, tokens, w.D))[0]
+    V = inputs.to_bf16(inputs.normal(seed + 3, (tokens, w.D)))
+    q = inputs.to_bf16(inputs.normal(seed + 2, (g * w.LQ, w.D)))
+    t0 = time.perf_counter()
+    e = codec.encode(keys.astype(np.float64), signs, tb, lay)
+    qjl = None
+    if w.QJL:
+        uh = codec.decode_rotated(e.i_xi, e.i_eta, e.i_rho, tb, lay)
+        bits, nu, _ = codec.qjl_encode(e.u_rot, uh, S)
+        qjl = (bits, np.float32(nu).astype(np.float64), S)
+    t1 = time.perf_counter()
+    attention.decode_attention(q.astype(np.float64), e.gamma, e.i_xi, e.i_eta, e.i_rho, V.astype(np.float64), signs,
+                               tb, lay, qjl=qjl)
+    t2 = time.perf_counter()
+    return t0, t1, t2  # CLOCK_MONOTONIC: comparable across the pool's processes
+
+
+def cpu_baseline(w: Workload = HEADLINE, heads: int = 1, tokens: int = 8192, pool: int = 0):
+    """Time the CPU oracle on a bounded sample of workload ``w``: oracle encode
+    (+ sketch) and decode attention of ``heads`` KV heads (their query heads)
+    over ``tokens`` tokens each. With ``pool`` > 0 the heads run in a process
+    pool of that many workers (spawned: the caller may hold a CUDA context)."""
+    from oracle import codec
+
+    lay = codec.Layout(w.D, w.BITS)
+    jobs = [(w, h, tokens, SEED + 101 * h, pool > 0) for h in range(heads)]
+    if pool > 0:
+        import multiprocessing as mp
+        with mp.get_context("spawn").Pool(pool) as p:
+            res = p.map(_oracle_head, jobs)
+    else:
+        res = [_oracle_head(j) for j in jobs]
+    enc_s = float(sum(r[1] - r[0] for r in res))
+    dec_s = float(sum(r[2] - r[1] for r in res))
+    per = unit_bytes(w, lay.words)
+    dec_bytes = heads * tokens * per + heads * (w.HQ // w.HKV) * w.LQ * w.D * 6
+    if pool > 0:
+        # the pool's span from the first encode start to the last decode end
+        # (worker start-up and table set-up excluded), split in the ratio of
+        # the summed encode and decode times
+        span = max(r[2] for r in res) - min(r[0] for r in res)
+        enc_s, dec_s = span * enc_s / (enc_s + dec_s), span * dec_s / (enc_s + dec_s)
     try:
         from threadpoolctl import threadpool_info
-        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+        blas = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
     except Exception:
-        cores = os.cpu_count() or 1
-    tb = tables.as_f32(*tables.codebooks(D, BITS))
-    lay = codec.Layout(D, BITS)
-    signs = tables.rotation_signs(SEED, D, HKV)
-    keys = inputs.to_bf16(inputs.llm_keys(SEED + 1, kv_heads, tokens, D))
-    V = inputs.to_bf16(inputs.normal(SEED + 3, (kv_heads, tokens, D)))
-    q = inputs.to_bf16(inputs.normal(SEED + 2, (kv_heads, HQ // HKV, D)))
-    t0 = time.perf_counter()
-    encs = [codec.encode(keys[h].astype(np.float64), signs[h], tb, lay) for h in range(kv_heads)]
-    t1 = time.perf_counter()
-    for h in range(kv_heads):
-        e = encs[h]
-        attention.decode_attention(q[h].astype(np.float64), e.gamma, e.i_xi, e.i_eta, e.i_rho,
-                                   V[h].astype(np.float64), signs[h], tb, lay)
-    t2 = time.perf_counter()
-    per_unit = 4 * lay.words + 4 + 2 * D
-    dec_bytes = kv_heads * tokens * per_unit + kv_heads * (HQ // HKV) * D * 6
+        blas = 1
+    cores = _cores()
+    used = min(pool, cores) if pool > 0 else min(blas, cores)
     return {
-        "value": dec_bytes / (t2 - t1) / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-        "sample": f"{kv_heads} KV head(s) x {tokens} tokens (of {HKV} x {N}); oracle float64 numpy",
-        "encode_mkeys_per_s": kv_heads * tokens / (t1 - t0) / 1e6,
-        "encode_s": t1 - t0, "decode_s": t2 - t1,
+        "value": dec_bytes / dec_s / 1e9, "unit": "GB/s",
+        "cores": used,
+        "kind": "oracle",
+        "sample": (f"{heads} KV head(s) x {tokens} tokens of {describe(w)}; oracle float64 numpy, "
+                   + (f"{pool}-process pool (one head per task, one BLAS thread each) on {cores} affinity cores"
+                      if pool > 0 else f"one process, {used} BLAS thread(s) on {cores} affinity cores")),
+        "encode_mkeys_per_s": heads * tokens / enc_s / 1e6,
+        "encode_s": enc_s, "decode_s": dec_s,
     }
 
 
@@ -203,10 +343,10 @@ def run_reference(args):
     # the oracle runs on rank 0 alone; it needs no process group
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    tokens = 4096
+    w, tokens = HEADLINE, 4096
     steps = []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(1, tokens)
+        r = cpu_baseline(w, 1, tokens)
         if i >= args.warmup:
             steps.append(r)
     dec_s = float(np.mean([s["decode_s"] for s in steps]))
@@ -217,7 +357,7 @@ def run_reference(args):
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * (dec_s + enc_s), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": f"1 KV head x {tokens} tokens per step"},
+        "config": {"workload": describe(w), "sample": f"1 KV head x {tokens} tokens per step"},
         "encode_mkeys_per_s": float(np.mean([s["encode_mkeys_per_s"] for s in steps])),
         "cpu_baseline": {"value": val, "unit": "GB/s", "cores": steps[0]["cores"], "kind": "oracle",
                          "sample": steps[0]["sample"]},
@@ -227,85 +367,84 @@ def run_reference(args):
     return 0
 
 
-# Decode throughput on the other workload shapes (reported next to the main
-# metric). Codes, gammas, sketches, V and queries are drawn on the device:
-# the decode's work and traffic do not depend on their values.
-OTHER_WORKLOADS = (
-    ("video_audio: B=1, 16/16 heads, d=64, ctx=65536, b=2, 8 query tokens", 1, 16, 16, 8, 64, 2, 65536, False),
-    ("qjl_long_context: B=8, 32/8 heads, d=128, ctx=131072, b=4 + QJL sketch", 8, 32, 8, 1, 128, 4, 131072, True),
-    ("llm_decode_large: B=8, 32/8 heads, d=128, ctx=131072, b=3", 8, 32, 8, 1, 128, 3, 131072, False),
-)
+# ------------------------------------------------------------------ GPU workloads
+def setup(w: Workload, dev, seed: int, n_caches: int = 1, batch: int | None = None):
+    """Device inputs of workload ``w`` (optionally another batch size): tables,
+    keys, V, queries, ``n_caches`` empty caches, an output and a workspace."""
+    import torch
+    from rotation_preconditioned_quantization_b200 import api, inputs
+
+    B = w.B if not batch else batch
+    H = B * w.HKV
+    lay = api.Layout(w.D, w.BITS, qjl=w.QJL)
+    tabs = api.DeviceTables.build(lay, SEED, w.HKV, device=dev)
+    if w.keys == "llm":
+        keys = inputs.device_llm_keys(seed + 1, H, w.N, w.D, dev)
+    else:
+        keys = inputs.device_normal(seed + 1, (H, w.N, w.D), dev)
+    V = inputs.device_normal(seed + 3, (H, w.N, w.D), dev)
+    q = inputs.device_normal(seed + 2, (B, w.HQ, w.LQ, w.D), dev)
+    caches = [api.Cache.empty(lay, H, w.N, dev) for _ in range(n_caches)]
+    out = torch.empty((B, w.HQ, w.LQ, w.D), dtype=torch.float32, device=dev)
+    wsp = api.Workspace(api.decode_attn_workspace_bytes(lay, B, w.HQ, w.HKV, w.LQ, w.N), dev)
+    return dict(lay=lay, tabs=tabs, keys=keys, V=V, q=q, caches=caches, out=out, wsp=wsp, B=B)
 
 
-def other_workloads(dev, peak, iters=6, shapes=OTHER_WORKLOADS):
+def time_decode_flushed(w: Workload, dev, peak, iters: int = 6, batch: int | None = None):
+    """Decode of workload ``w`` over a cache the encoder wrote from keys of its
+    recipe; L2 flushed (512 MB written) before every timed call."""
     import torch
     from rotation_preconditioned_quantization_b200 import api
 
-    out = {}
-    flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)  # > L2 between timed calls
-    for name, B_, HQ_, HKV_, LQ_, D_, BITS_, N_, qjl in shapes:
-        lay = api.Layout(D_, BITS_, qjl=qjl)
-        H = B_ * HKV_
-        tabs = api.DeviceTables.build(lay, SEED, HKV_, device=dev)
-        g = torch.Generator(device=dev).manual_seed(SEED)
-        cache = api.Cache.empty(lay, H, N_, dev)
-        cache.packed.random_(generator=g)
-        cache.gamma.uniform_(0.5, 2.0, generator=g)
-        if qjl:
-            cache.qjl_bits.random_(generator=g)
-            cache.qjl_norm.uniform_(0.0, 0.3, generator=g)
-        cache.length = N_
-        V = torch.randn((H, N_, D_), device=dev, generator=g).to(torch.bfloat16)
-        q = torch.randn((B_, HQ_, LQ_, D_), device=dev, generator=g).to(torch.bfloat16)
-        o = torch.empty((B_, HQ_, LQ_, D_), device=dev)
-        wsp = api.Workspace(api.decode_attn_workspace_bytes(lay, B_, HQ_, HKV_, LQ_, N_), dev)
-        ts = []
-        for i in range(iters + 2):
-            flush.sum()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            api.decode_attn(lay, tabs, q, cache, V, HKV_, out=o, workspace=wsp)
-            e1.record()
-            torch.cuda.synchronize(dev)
-            if i >= 2:
-                ts.append(e0.elapsed_time(e1))
-        unit = 4 * lay.words + 4 + 2 * D_ + (4 * (D_ // 32) + 4 if qjl else 0)
-        nbytes = H * N_ * unit
-        ms = float(np.mean(ts))
-        gbs = nbytes / (ms * 1e-3) / 1e9
-        out[name] = {"GB/s": gbs, "frac": gbs / peak, "ms": ms, "MB": nbytes / 1e6,
-                     "kernel": "tensor-core" if D_ <= 128 else "ffma"}
-        del cache, V
-    return out
+    s = setup(w, dev, SEED + 77, batch=batch)
+    lay, cache = s["lay"], s["caches"][0]
+    api.encode(lay, s["tabs"], s["keys"], cache, 0)
+    del s["keys"]
+    flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)
+    ts = []
+    for i in range(iters + 2):
+        flush.fill_(float(i))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        api.decode_attn(lay, s["tabs"], s["q"], cache, s["V"], w.HKV, out=s["out"], workspace=s["wsp"])
+        e1.record()
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1))
+    assert s["wsp"].status() == 0, "a bounded on-chip wait of the decode kernel expired"
+    wb = w._replace(B=s["B"])
+    nbytes = decode_bytes(wb, lay.words)
+    ms = float(np.mean(ts))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"GB/s": gbs, "frac": gbs / peak, "ms": ms, "ms_min": float(np.min(ts)), "MB": nbytes / 1e6,
+            "cache": "encoded by octo_encode", "l2": "flushed (512 MB written) before each call",
+            "kernel": "tensor-core" if w.D <= 128 else "ffma"}
 
 
 def dequant_workload(dev, peak, iters=6):
-    """octo_dequant (key reconstruction) of the bench workload's cache
-    (8 KV heads x 32768 tokens, d=128, b=3) into fp32 and bf16 rows.
-    Algorithmic bytes per key: 4W + 4 read, 4d or 2d written."""
+    """octo_dequant (key reconstruction) of an LLM decode cache (8 KV heads x
+    32768 tokens, d=128, b=3) into fp32 and bf16 rows. Algorithmic bytes per
+    key: 4W + 4 read, 4d or 2d written."""
     import torch
     from rotation_preconditioned_quantization_b200 import api
 
-    lay = api.Layout(D, BITS)
-    H = B * HKV
-    tabs = api.DeviceTables.build(lay, SEED, HKV, device=dev)
-    g = torch.Generator(device=dev).manual_seed(SEED + 5)
-    cache = api.Cache.empty(lay, H, N, dev)
-    cache.packed.random_(generator=g)
-    cache.gamma.uniform_(0.5, 2.0, generator=g)
-    cache.length = N
+    w = LLM_DECODE
+    s = setup(w, dev, SEED + 5)
+    lay, cache = s["lay"], s["caches"][0]
+    api.encode(lay, s["tabs"], s["keys"], cache, 0)
+    H, N, D = w.B * w.HKV, w.N, w.D
     flush = torch.empty(512 * 1024 * 1024 // 4, device=dev)  # > L2 between timed calls
     out = {}
     for name, dt, esz in (("f32", torch.float32, 4), ("bf16", torch.bfloat16, 2)):
         o = torch.empty((H, N, D), dtype=dt, device=dev)
         ts = []
         for i in range(iters + 2):
-            flush.sum()
+            flush.fill_(float(i))
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
-            api.dequant(lay, tabs, cache, out=o)
+            api.dequant(lay, s["tabs"], cache, out=o)
             e1.record()
             torch.cuda.synchronize(dev)
             if i >= 2:
@@ -373,47 +512,32 @@ def encode_sweep(dev, peak):
 
 def run_gpu(args):
     import torch
-    from rotation_preconditioned_quantization_b200 import api, inputs
+    from rotation_preconditioned_quantization_b200 import api
 
     ws, rank, local = _dist_init()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    lay = api.Layout(D, BITS)
-    tabs = api.DeviceTables.build(lay, SEED, HKV, device=dev)
-    n_copies = 3
-
-    # inputs: distinct per copy and per rank
-    def make(copy):
-        s = SEED + 1000 * rank + 10 * copy
-        keys = torch.from_numpy(inputs.llm_keys(s + 1, B * HKV, N, D)).to(torch.bfloat16)
-        V = torch.from_numpy(inputs.normal(s + 3, (B * HKV, N, D))).to(torch.bfloat16)
-        q = torch.from_numpy(inputs.normal(s + 2, (B, HQ, 1, D))).to(torch.bfloat16)
-        return keys, V, q
-
-    host = [make(c) for c in range(n_copies)]
-    devc = []
-    for keys, V, q in host:
-        devc.append(dict(keys=keys.to(dev), V=V.to(dev), q=q.to(dev), cache=api.Cache.empty(lay, B * HKV, N, dev),
-                         out=torch.empty((B, HQ, 1, D), dtype=torch.float32, device=dev)))
-    wsp = api.Workspace(api.decode_attn_workspace_bytes(lay, B, HQ, HKV, 1, N), dev)
+    w = HEADLINE
+    seed = SEED + 1000 * rank  # an independent batch per rank
+    s = setup(w, dev, seed, n_caches=2)
+    lay, tabs, caches = s["lay"], s["tabs"], s["caches"]
     stream = torch.cuda.current_stream(dev)
 
     def step(i, ev=None):
-        c_enc = devc[i % n_copies]
-        c_dec = devc[(i - 1) % n_copies]
+        c_enc = caches[i % 2]
+        c_dec = caches[(i - 1) % 2]
         if ev is not None:
             ev[0].record(stream)
-        api.encode(lay, tabs, c_enc["keys"], c_enc["cache"], 0)
+        api.encode(lay, tabs, s["keys"], c_enc, 0)
         if ev is not None:
             ev[1].record(stream)
-        api.decode_attn(lay, tabs, c_dec["q"], c_dec["cache"], c_dec["V"], HKV, kv_len=N, out=c_dec["out"],
-                        workspace=wsp)
+        api.decode_attn(lay, tabs, s["q"], c_dec, s["V"], w.HKV, kv_len=w.N, out=s["out"], workspace=s["wsp"])
         if ev is not None:
             ev[2].record(stream)
 
-    # prime: every copy's cache encoded once, then warm-up steps
-    for c in range(n_copies):
-        api.encode(lay, tabs, devc[c]["keys"], devc[c]["cache"], 0)
+    # prime: both caches encoded once, then warm-up steps
+    for c in caches:
+        api.encode(lay, tabs, s["keys"], c, 0)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(dev)
@@ -430,6 +554,8 @@ def run_gpu(args):
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     _barrier(ws)
+    if s["wsp"].status() != 0:
+        raise RuntimeError("a bounded on-chip wait of the decode kernel expired")
     total_ms = t_start.elapsed_time(t_end)
     enc_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
@@ -438,54 +564,58 @@ def run_gpu(args):
     total_ms_max = _max_over_ranks(total_ms, ws)
     dec_sum_max = _max_over_ranks(float(np.sum(dec_ms)), ws)
     enc_sum_max = _max_over_ranks(float(np.sum(enc_ms)), ws)
-    dbytes = _bytes_decode(lay.words)
-    ebytes = _bytes_encode(lay.words)
+    dbytes = decode_bytes(w, lay.words)
+    ebytes = encode_bytes(w, lay.words)
+    units = w.B * w.HKV * w.N
     value = ws * dbytes * args.steps / (dec_sum_max * 1e-3) / 1e9
-    enc_mkeys = ws * B * HKV * N * args.steps / (enc_sum_max * 1e-3) / 1e6
+    enc_mkeys = ws * units * args.steps / (enc_sum_max * 1e-3) / 1e6
 
-    # end to end through the public API from pinned host buffers
-    hk, hV, hq = (t.pin_memory() for t in host[0])
-    hout = torch.empty((B, HQ, 1, D), dtype=torch.float32).pin_memory()
-    e2e_cache = api.Cache.empty(lay, B * HKV, N, dev)
-    dk = torch.empty_like(hk, device=dev)
-    dV = torch.empty_like(hV, device=dev)
-    dq = torch.empty_like(hq, device=dev)
-    dout = torch.empty((B, HQ, 1, D), dtype=torch.float32, device=dev)
+    # end to end through the public API from pinned host buffers: per step the
+    # keys, V and queries go host -> device, then encode + decode, then the
+    # output comes back
+    e2e_cache = caches[0]
+    hk = s["keys"].cpu().pin_memory()
+    hV = s["V"].cpu().pin_memory()
+    hq = s["q"].cpu().pin_memory()
+    hout = torch.empty_like(s["out"], device="cpu").pin_memory()
+    dk, dV, dq = s["keys"], s["V"], s["q"]
 
     def e2e_step():
         dk.copy_(hk, non_blocking=True)
         dV.copy_(hV, non_blocking=True)
         dq.copy_(hq, non_blocking=True)
         api.encode(lay, tabs, dk, e2e_cache, 0)
-        api.decode_attn(lay, tabs, dq, e2e_cache, dV, HKV, kv_len=N, out=dout, workspace=wsp)
-        hout.copy_(dout, non_blocking=True)
+        api.decode_attn(lay, tabs, dq, e2e_cache, dV, w.HKV, kv_len=w.N, out=s["out"], workspace=s["wsp"])
+        hout.copy_(s["out"], non_blocking=True)
 
-    for _ in range(max(1, args.warmup)):
+    e2e_steps = max(1, min(args.steps, 10))
+    for _ in range(max(1, min(args.warmup, 3))):
         e2e_step()
     torch.cuda.synchronize(dev)
     _barrier(ws)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(e2e_steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), ws)
     h2d = hk.numel() * 2 + hV.numel() * 2 + hq.numel() * 2
     d2h = hout.numel() * 4
-    e2e_val = ws * dbytes * args.steps / (e2e_ms * 1e-3) / 1e9
+    e2e_val = ws * dbytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+    del hk, hV
 
     peak, peak_kind = _peaks()
     dec_avg_s = float(np.mean(dec_ms)) * 1e-3
     achieved = dbytes / dec_avg_s / 1e9
     traffic = _ncu_traffic()
     if rank != 0:  # every collective is behind us; rank 0 alone reports
-        if ws > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        _finish_ranks(ws)
         return 0
-    extra = None if args.no_extra else other_workloads(dev, peak)
+    del s
+    torch.cuda.empty_cache()
+    extra = None if args.no_extra else {describe(o): time_decode_flushed(o, dev, peak) for o in OTHER_WORKLOADS}
     dq = None if args.no_extra else dequant_workload(dev, peak)
     sweep = None if args.no_extra else encode_sweep(dev, peak)
     line = {
@@ -493,18 +623,22 @@ def run_gpu(args):
         "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "per_rank": "independent batch per GPU (no collective)",
-                   "l2": "3 rotating input copies (~150 MB each > 126 MB L2); decode reads the cache encoded one step earlier"},
+        "config": {"workload": describe(w), "per_rank": "independent batch per GPU (no collective)",
+                   "l2": "inputs larger than L2: each decode reads 2.95 GB of cache + V, encoded one step earlier "
+                         "into the other of two caches (the other cache's encode in between)"},
         "encode_mkeys_per_s": enc_mkeys,
         "encode_ms": float(np.mean(enc_ms)), "decode_ms": float(np.mean(dec_ms)),
+        "decode_ms_min": float(np.min(dec_ms)),
         "decode_bytes_per_step": dbytes, "encode_bytes_per_step": ebytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "kernel": "octo_decode_attn",
-                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6650 GB/s"},
-        "encode_roofline": {"bound": "hbm", "achieved": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9, "peak": peak,
-                            "unit": "GB/s", "frac": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9 / peak},
+                     "frac": achieved / peak, "traffic": traffic, "kernel": "octo_decode_attn (decode_tc_kernel<128,4,4,QJL>)",
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback 6650 GB/s",
+                     "algorithmic_bytes": "per (token, KV head) 4W + 4 + 2d + 4d/32 + 4 = 352 B (W = 18), x 8.39 M units, + q + out"},
+        "encode_roofline": {"bound": "alu", "hbm_achieved": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9,
+                            "hbm_peak": peak, "unit": "GB/s",
+                            "hbm_frac": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9 / peak},
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms / args.steps},
+                "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps},
         "gpu_launches": launches,
         "other_workloads": extra,
         "dequant": dq,
@@ -512,16 +646,18 @@ def run_gpu(args):
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline and ws == 1:
-        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(1, N).items() if k not in ("encode_s", "decode_s")}
+        one = cpu_baseline(w, 1, 8192)
+        pool_n = min(_cores(), 8)
+        many = cpu_baseline(w, pool_n, 8192, pool=pool_n)
+        line["cpu_baseline"] = {k: v for k, v in many.items() if k not in ("encode_s", "decode_s")}
+        line["cpu_baseline"]["single_process"] = {k: v for k, v in one.items() if k not in ("encode_s", "decode_s")}
     print(json.dumps(line))
-    if ws > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    _finish_ranks(ws)
     return 0
 
 
 DECODE_KERNEL_SOURCES = ("octo_common.cuh", "octo_decode_kernel.cuh", "octo_decode.cu")
-DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_tc_kernel_llm_decode_b1_h32x8_d128_ctx32768_b3.md")
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_tc_kernel_qjl_long_context_h32x8_d128_ctx131072_b4qjl.md")
 
 
 def kernel_sources_digest(names=DECODE_KERNEL_SOURCES) -> str:
@@ -534,8 +670,9 @@ def kernel_sources_digest(names=DECODE_KERNEL_SOURCES) -> str:
 
 
 def _ncu_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, or None when
-    the summary is missing or was taken on other kernel sources."""
+    """DRAM bytes per headline decode launch from the committed ncu summary
+    (captured on a smaller batch and scaled by the units processed), or None
+    when the summary is missing or was taken on other kernel sources."""
     try:
         with open(DECODE_PROFILE) as f:
             text = f.read()
@@ -551,15 +688,16 @@ def _ncu_traffic():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="octopus", choices=["octopus", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-extra", action="store_true", help="skip the decode timings of the other workload shapes")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads, dequant and the encode sweep")
+    ap.add_argument("--dry-run", action="store_true", help="rank logic only, no GPU (a CPU check of --gpus N)")
     ap.add_argument("--only", choices=["dequant", "encode_sweep", "decode_shape"],
                     help="time only this part (one GPU; prints its JSON)")
-    ap.add_argument("--shape", default="llm_decode_large",
-                    help="with --only decode_shape: the other decode workload to time (name prefix)")
+    ap.add_argument("--shape", default=HEADLINE.name,
+                    help="with --only decode_shape: the decode workload to time (name prefix)")
     ap.add_argument("--batch", type=int, default=0,
                     help="with --only decode_shape: replace the workload's batch size (a smaller case to profile)")
     args = ap.parse_args()
@@ -567,33 +705,28 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
-    if args.only == "dequant":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return spawn_ranks(args.gpus, sys.argv[1:])
+    if args.dry_run:
+        return run_dry(args)
+    if args.only:
         import torch
 
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
-        print(json.dumps({"dequant": dequant_workload(dev, _peaks()[0])}))
-        return 0
-    if args.only == "decode_shape":
-        import torch
-
-        dev = torch.device("cuda", 0)
-        torch.cuda.set_device(dev)
-        shapes = [w for w in OTHER_WORKLOADS if w[0].startswith(args.shape)]
-        if len(shapes) != 1:
-            raise SystemExit(f"--shape {args.shape!r} names {len(shapes)} workloads")
-        w = list(shapes[0])
-        if args.batch > 0 and args.batch != w[1]:
-            w[0] = w[0].replace(f"B={w[1]},", f"B={args.batch},")
-            w[1] = args.batch
-        print(json.dumps({"decode_shape": other_workloads(dev, _peaks()[0], shapes=[tuple(w)])}))
-        return 0
-    if args.only == "encode_sweep":
-        import torch
-
-        dev = torch.device("cuda", 0)
-        torch.cuda.set_device(dev)
-        print(json.dumps({"encode_sweep": encode_sweep(dev, _peaks()[0])}))
+        peak = _peaks()[0]
+        if args.only == "dequant":
+            print(json.dumps({"dequant": dequant_workload(dev, peak)}))
+        elif args.only == "encode_sweep":
+            print(json.dumps({"encode_sweep": encode_sweep(dev, peak)}))
+        else:
+            shapes = [w for w in (HEADLINE, *OTHER_WORKLOADS) if w.name.startswith(args.shape)]
+            if len(shapes) != 1:
+                raise SystemExit(f"--shape {args.shape!r} names {len(shapes)} workloads")
+            w = shapes[0]
+            b = args.batch if args.batch > 0 else None
+            print(json.dumps({"decode_shape": {describe(w._replace(B=b or w.B)): time_decode_flushed(w, dev, peak,
+                                                                                                        batch=b)}}))
         return 0
     return run_gpu(args)
 

@@ -221,11 +221,17 @@ OCTO_API int octo_decode_attn(const octo_layout* L, const octo_tables* tables,
  *   - The first call on a device (with that device current) looks up the
  *     array's device address; make that first call outside any stream
  *     capture.
- *   - Each call zeroes the array's status word and arrival counters on
- *     `stream` before the decode kernel. All calls on a device share the
- *     array, which keeps the last call's contents: calls that overlap on
- *     the GPU (other streams, or other threads) race on it and must not be
- *     issued. */
+ *   - Arguments are checked exactly as octo_decode_attn checks them (same
+ *     status codes, same order) before anything touches the GPU; a
+ *     rejected call launches nothing and leaves the array alone.
+ *   - Each accepted call zeroes the array's status word and arrival
+ *     counters on `stream` before the decode kernel. All calls on a device
+ *     share the array, which keeps the last call's contents: calls that
+ *     overlap on the GPU (other streams, or other threads) race on it and
+ *     must not be issued.
+ *   - The kernel's timeout flag (bit 0 of the status word, see
+ *     octo_decode_attn) lives in the array; read it with
+ *     octo_decode_attn_static_status. */
 #define OCTO_STATIC_SCRATCH_BYTES (8u << 20)
 OCTO_API int octo_decode_attn_static(const octo_layout* L, const octo_tables* tables,
                                      const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
@@ -234,6 +240,24 @@ OCTO_API int octo_decode_attn_static(const octo_layout* L, const octo_tables* ta
                                      const uint32_t* qjl_bits, const float* qjl_norm,
                                      const void* V, float scale, float* out, float* logits,
                                      octo_stream_t stream);
+
+/* Host. The status word that the last octo_decode_attn_static call on the
+ * current device left in the library's scratch array (bit 0 set: one of
+ * the kernel's bounded on-chip waits expired, and that call's outputs are
+ * invalid). Waits for the work queued on `stream` (the stream of that
+ * call) to finish, then copies the word into *status. Not part of the
+ * method; it serves octo_decode_attn_static's callers, who have no
+ * workspace to read the word from. Errors: OCTO_EINVAL (status NULL),
+ * OCTO_ECUDA. */
+OCTO_API int octo_decode_attn_static_status(int* status, octo_stream_t stream);
+
+/* Device. Fills the whole scratch array of octo_decode_attn_static on the
+ * current device with the byte value `byte` & 0xff, on `stream`. A
+ * diagnostic: it lets a test leave nonzero status and counter bytes behind,
+ * as an interrupted call would, and check that the next call still clears
+ * what must start at zero. Normal use never needs it. Same race rules as
+ * octo_decode_attn_static. */
+OCTO_API int octo_decode_attn_static_fill(int byte, octo_stream_t stream);
 
 /* Device. Reconstructs keys from the cache: k_hat = gamma * R^T u_hat
  * (explainer, "triplet decomposition" steps 1-4 undone, for the codec's

@@ -10,8 +10,7 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# OCTO_LIBRARY selects another build of the same library (e.g. a tuning variant)
-LIB_PATH = os.environ.get("OCTO_LIBRARY") or os.path.join(_HERE, "liboctopus_b200.so")
+LIB_PATH = os.path.join(_HERE, "liboctopus_b200.so")
 
 OCTO_OK, OCTO_EINVAL, OCTO_EUNSUPPORTED, OCTO_ECUDA, OCTO_EWORKSPACE = 0, -1, -2, -3, -4
 ROUND_SCALAR, ROUND_JOINT = 0, 1
@@ -63,6 +62,8 @@ _SIGS = {
                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_void_p]),
+    "octo_decode_attn_static_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
+    "octo_decode_attn_static_fill": (ctypes.c_int, [ctypes.c_int, ctypes.c_void_p]),
     "octo_dequant": (ctypes.c_int, [ctypes.POINTER(OctoLayout), ctypes.POINTER(OctoTables), ctypes.c_int64, ctypes.c_int64,
                                     ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_int, ctypes.c_void_p]),

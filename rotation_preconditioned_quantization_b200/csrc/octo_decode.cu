@@ -9,6 +9,7 @@
 #include <climits>
 #include <cstring>
 
+#include "octo_decode_check.h"
 #include "octo_decode_kernel.cuh"
 
 namespace octo {
@@ -170,11 +171,10 @@ extern "C" size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq
   return ws_layout(static_cast<int64_t>(B) * Hkv, n_splits, G, L->d).total;
 }
 
-extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, const void* q, int q_dtype, int B,
-                                int Hq, int Hkv, int Lq, int64_t kv_len, int64_t cache_cap,
-                                const uint32_t* packed, const float* gamma, const uint32_t* qjl_bits,
-                                const float* qjl_norm, const void* V, float scale, float* out, float* logits,
-                                void* workspace, size_t ws_bytes, octo_stream_t stream) {
+int octo::decode_validate(const octo_layout* L, const octo_tables* tab, const void* q, int q_dtype, int B, int Hq,
+                          int Hkv, int Lq, int64_t kv_len, int64_t cache_cap, const uint32_t* packed,
+                          const float* gamma, const uint32_t* qjl_bits, const float* qjl_norm, const void* V,
+                          float scale, const float* out, const float* logits, size_t* ws_need) {
   const int lc = check_layout(L);
   if (lc != OCTO_OK) return lc;
   if (!tab || !q || !packed || !gamma || !tab->dir_c || !tab->rho_c || !tab->signs || tab->n_heads < 1)
@@ -190,12 +190,25 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   // code rows are staged by 16-byte bulk copies
   if (cache_cap % 4 != 0 || misaligned(packed) || misaligned(gamma)) return OCTO_EINVAL;
   if (L->qjl && (misaligned(qjl_bits) || misaligned(qjl_norm))) return OCTO_EINVAL;
-  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return OCTO_EINVAL;
   if (!(scale == scale)) return OCTO_EINVAL;
-  const int g = Hq / Hkv, Gq = g * Lq;
-  if (Gq > 8) return OCTO_EUNSUPPORTED;
+  if ((Hq / Hkv) * Lq > 8) return OCTO_EUNSUPPORTED;
   if (static_cast<int64_t>(B) * Hkv > 65535) return OCTO_EUNSUPPORTED;  // grid.y limit
   if (kv_len > INT_MAX) return OCTO_EUNSUPPORTED;                         // 32-bit token coordinates
+  if (ws_need) *ws_need = octo_decode_attn_workspace(L, B, Hq, Hkv, Lq, kv_len);
+  return OCTO_OK;
+}
+
+extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, const void* q, int q_dtype, int B,
+                                int Hq, int Hkv, int Lq, int64_t kv_len, int64_t cache_cap,
+                                const uint32_t* packed, const float* gamma, const uint32_t* qjl_bits,
+                                const float* qjl_norm, const void* V, float scale, float* out, float* logits,
+                                void* workspace, size_t ws_bytes, octo_stream_t stream) {
+  size_t need = 0;
+  const int vc = octo::decode_validate(L, tab, q, q_dtype, B, Hq, Hkv, Lq, kv_len, cache_cap, packed, gamma,
+                                       qjl_bits, qjl_norm, V, scale, out, logits, &need);
+  if (vc != OCTO_OK) return vc;
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return OCTO_EINVAL;
+  const int g = Hq / Hkv, Gq = g * Lq;
   const int D = L->d;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t heads = static_cast<int64_t>(B) * Hkv;

@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/octopus.h"
+#include "octo_decode_check.h"
 
 namespace {
 
@@ -42,11 +43,12 @@ extern "C" int octo_decode_attn_static(const octo_layout* L, const octo_tables* 
                                        const uint32_t* packed, const float* gamma, const uint32_t* qjl_bits,
                                        const float* qjl_norm, const void* V, float scale, float* out, float* logits,
                                        octo_stream_t stream) {
-  const size_t need = octo_decode_attn_workspace(L, B, Hq, Hkv, Lq, kv_len);
-  if (need == 0) {  // sizes the decode step rejects: too many query rows per KV head, or invalid
-    const bool shaped = L && B >= 1 && Hkv >= 1 && Hq >= Hkv && Hq % Hkv == 0 && Lq >= 1;
-    return shaped && (Hq / Hkv) * Lq > 8 ? OCTO_EUNSUPPORTED : OCTO_EINVAL;
-  }
+  // octo_decode_attn's own checks first (same codes, same order): a rejected
+  // call touches neither the GPU nor the shared array
+  size_t need = 0;
+  const int vc = octo::decode_validate(L, tables, q, q_dtype, B, Hq, Hkv, Lq, kv_len, cache_cap, packed, gamma,
+                                       qjl_bits, qjl_norm, V, scale, out, logits, &need);
+  if (vc != OCTO_OK) return vc;
   if (need > OCTO_STATIC_SCRATCH_BYTES) return OCTO_EWORKSPACE;
   void* scratch = nullptr;
   const int rc = scratch_address(&scratch);
@@ -59,4 +61,25 @@ extern "C" int octo_decode_attn_static(const octo_layout* L, const octo_tables* 
   if (cudaMemsetAsync(scratch, 0, zero, st) != cudaSuccess) return OCTO_ECUDA;
   return octo_decode_attn(L, tables, q, q_dtype, B, Hq, Hkv, Lq, kv_len, cache_cap, packed, gamma, qjl_bits,
                           qjl_norm, V, scale, out, logits, scratch, OCTO_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int octo_decode_attn_static_status(int* status, octo_stream_t stream) {
+  if (!status) return OCTO_EINVAL;
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != OCTO_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, scratch, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return OCTO_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return OCTO_ECUDA;
+  *status = word;
+  return OCTO_OK;
+}
+
+extern "C" int octo_decode_attn_static_fill(int byte, octo_stream_t stream) {
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != OCTO_OK) return rc;
+  const cudaError_t e = cudaMemsetAsync(scratch, byte & 0xff, OCTO_STATIC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? OCTO_OK : OCTO_ECUDA;
 }

@@ -235,4 +235,4 @@ extern "C" const char* octo_status_string(int status) {
   }
 }
 
-extern "C" int octo_abi_version(void) { return 101; }
+extern "C" int octo_abi_version(void) { return 102; }

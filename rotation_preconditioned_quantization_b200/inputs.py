@@ -15,6 +15,11 @@ pages evaluate on; the pages' own models and datasets are not available):
   by a per-token factor drawn from lognormal(0, 0.5).
 * ``normal``: plain N(0, 1) draws for queries and values.
 
+``device_normal`` and ``device_llm_keys`` draw the same distributions with
+torch's seeded generator directly in device memory, for workloads too large
+to draw on the host (the benchmark's long-context cache); they follow the
+same recipes but not the same numbers as their numpy counterparts.
+
 ``to_bf16`` rounds float32 to bfloat16 (round to nearest even) and returns
 float32 arrays holding the bf16 values, so that numpy code sees exactly the
 numbers a bf16 device buffer holds.
@@ -25,7 +30,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["rng", "normal", "gaussian_keys", "llm_keys", "to_bf16", "bf16_bits",
-           "random_codes", "append_lengths"]
+           "random_codes", "append_lengths", "device_normal", "device_llm_keys"]
 
 
 def rng(seed: int) -> np.random.Generator:
@@ -85,4 +90,36 @@ def append_lengths(seed: int, total: int, lo: int = 1, hi: int = 4096) -> list[i
         n = min(n, total - acc)
         out.append(n)
         acc += n
+    return out
+
+
+def device_normal(seed: int, shape, device, dtype=None):
+    """iid N(0, 1) draws of ``shape`` made on ``device`` (torch generator seeded
+    with ``seed``), cast to ``dtype`` (default bfloat16) by torch's rounding."""
+    import torch
+
+    g = torch.Generator(device=device).manual_seed(seed)
+    x = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    return x.to(torch.bfloat16 if dtype is None else dtype)
+
+
+def device_llm_keys(seed: int, n_heads: int, n_tokens: int, d: int, device, dtype=None,
+                    n_outlier: int = 4, outlier_scale: float = 10.0, lognormal_sigma: float = 0.5):
+    """[n_heads][n_tokens][d] LLM-shaped keys drawn on ``device`` (recipe of
+    ``llm_keys``: N(0, 1) entries, ``n_outlier`` channels chosen once without
+    replacement and scaled by ``outlier_scale``, every key scaled by a
+    per-token lognormal(0, ``lognormal_sigma``) factor), cast to ``dtype``
+    (default bfloat16). Drawn one head at a time, so the float32 temporary
+    is a single head."""
+    import torch
+
+    dt = torch.bfloat16 if dtype is None else dtype
+    g = torch.Generator(device=device).manual_seed(seed)
+    ch = torch.from_numpy(rng(seed).choice(d, size=n_outlier, replace=False)).to(device)
+    out = torch.empty((n_heads, n_tokens, d), dtype=dt, device=device)
+    for h in range(n_heads):
+        k = torch.randn((n_tokens, d), generator=g, device=device, dtype=torch.float32)
+        k[:, ch] *= outlier_scale
+        f = torch.empty((n_tokens, 1), device=device, dtype=torch.float32).log_normal_(0.0, lognormal_sigma, generator=g)
+        out[h] = (k * f).to(dt)
     return out

@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_lib.exported_symbols())
-    assert L.octo_abi_version() == 101
+    assert L.octo_abi_version() == 102
 
 
 @pytest.mark.parametrize("d,b", [(64, 2), (64, 4), (128, 3), (128, 4), (256, 2), (256, 4)])

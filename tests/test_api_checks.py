@@ -99,3 +99,39 @@ def test_dequant_refuses_a_non_contiguous_cache():
     with pytest.raises(ValueError, match="packed"):
         api.dequant(lay, _tabs(lay, 2), view)
     assert np.all(big.gamma.numpy() == 0)
+
+
+def test_static_entry_point_refuses_like_the_workspace_one():
+    """octo_decode_attn_static runs octo_decode_attn's own checks first: for every
+    rejected argument set both return the same status, and the static one does so
+    before it looks up or clears its scratch array (nothing here reaches CUDA)."""
+    import ctypes
+
+    from rotation_preconditioned_quantization_b200 import _lib
+
+    lib = _lib.lib()
+    good = api.Layout(128, 3)
+    d96 = _lib.OctoLayout()
+    ctypes.memmove(ctypes.byref(d96), good.ref, ctypes.sizeof(d96))
+    d96.d = 96
+    T = _lib.OctoTables(256, 256, 256, 256, 256, None, 8)
+    nan = float("nan")
+    cases = {  # name: (layout, q, B, Hq, Hkv, Lq, kv, cap, scale)
+        "d=96": (ctypes.byref(d96), 256, 1, 4, 1, 1, 8, 8, 0.1),
+        "B*Hkv > 65535": (good.ref, 256, 65536, 4, 1, 1, 8, 8, 0.1),
+        "B*Hkv > 65535, many tokens": (good.ref, 256, 8192, 64, 8, 1, 131072, 131072, 0.1),
+        "9 query rows": (good.ref, 256, 1, 9, 1, 1, 8, 8, 0.1),
+        "q NULL": (good.ref, None, 1, 4, 1, 1, 8, 8, 0.1),
+        "kv_len > cap": (good.ref, 256, 1, 4, 1, 1, 12, 8, 0.1),
+        "NaN scale": (good.ref, 256, 1, 4, 1, 1, 8, 8, nan),
+    }
+    want = {"d=96": _lib.OCTO_EUNSUPPORTED, "B*Hkv > 65535": _lib.OCTO_EUNSUPPORTED,
+            "B*Hkv > 65535, many tokens": _lib.OCTO_EUNSUPPORTED, "9 query rows": _lib.OCTO_EUNSUPPORTED,
+            "q NULL": _lib.OCTO_EINVAL, "kv_len > cap": _lib.OCTO_EINVAL, "NaN scale": _lib.OCTO_EINVAL}
+    for name, (L, q, B, Hq, Hkv, Lq, kv, cap, sc) in cases.items():
+        ws = lib.octo_decode_attn(L, ctypes.byref(T), q, _lib.BF16, B, Hq, Hkv, Lq, kv, cap, 256, 256, None, None,
+                                  256, ctypes.c_float(sc), 256, None, 256, 1 << 40, None)
+        st = lib.octo_decode_attn_static(L, ctypes.byref(T), q, _lib.BF16, B, Hq, Hkv, Lq, kv, cap, 256, 256, None,
+                                         None, 256, ctypes.c_float(sc), 256, None, None)
+        assert ws == st == want[name], (name, ws, st)
+    assert lib.octo_decode_attn_static_status(None, None) == _lib.OCTO_EINVAL

@@ -64,3 +64,23 @@ def test_reference_arm_prints_one_json_line():
     assert j["impl"] == "reference" and j["unit"] == "GB/s" and j["value"] > 0
     assert j["cpu_baseline"]["kind"] == "oracle" and j["e2e"]["h2d_bytes_per_step"] == 0
     assert j["warmup"] >= 3
+
+
+def test_bench_gpus_two_spawns_two_ranks_and_one_line():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself (gloo here,
+    NCCL on GPUs): each takes its own batch seed, the duration is the max over
+    ranks, the whole-job value counts both ranks' units, and rank 0 alone
+    prints the one JSON line."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env["PYTHONPATH"] = ROOT
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1, r.stdout
+    j = json.loads(lines[0])
+    assert j["n_gpus"] == 2 and j["scaling"] == "weak"
+    assert j["max_ms"] == 20.0                           # rank 1 reports 20 ms, rank 0 10 ms
+    units = 8 * 8 * 131072                               # B x Hkv x context of the headline workload
+    assert j["value"] == 2 * units / 20.0
+    assert len(set(j["config"]["per_rank_seeds"])) == 2  # an independent batch per rank

@@ -45,8 +45,10 @@ def test_octahedral_special_points():
     want = np.array([[0, 0], [1, 1], [1, 0], [-1, 0], [0, 1], [0, -1], [0, 0], [0, 0]], float)
     got = np.stack([xi, eta], axis=1)
     assert np.allclose(got[:6], want[:6], atol=0)
-    # a point just below the equator on the x=y diagonal folds to the square's centre
-    assert np.allclose(got[6], [0.5 * 0 + 0.0, 0.0], atol=1e-12) or np.allclose(got[6], [0.5, 0.5], atol=1e-12)
+    # a point just below the equator on the x=y diagonal: p = (1/2, 1/2, -tiny) takes the
+    # lower branch, ((1 - 1/2) sgn p_x, (1 - 1/2) sgn p_y) = (1/2, 1/2), the same point
+    # the upper branch gives on the equator (the fold is continuous there)
+    assert np.array_equal(got[6], [0.5, 0.5])
     assert np.array_equal(got[7], [0.0, 0.0])
     # corners of the square are the south pole, centre the north pole
     assert np.allclose(codec.oct_inverse(np.array([1.0, -1, 1, -1]), np.array([1.0, 1, -1, -1])),

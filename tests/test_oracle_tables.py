@@ -38,8 +38,14 @@ def test_signs_are_pm1_and_seeded():
     assert set(np.unique(s)) == {-1.0, 1.0}
     assert np.array_equal(s, tables.rotation_signs(7, 128, 4))
     assert not np.array_equal(s, tables.rotation_signs(8, 128, 4))
-    # heads draw disjoint stretches of one stream
-    assert np.array_equal(tables.rotation_signs(7, 128, 4)[1:], tables.rotation_signs(7, 128, 4)[1:])
+    # heads draw consecutive, disjoint stretches of one SplitMix64 stream:
+    # row h is outputs h*d + 1 .. h*d + d, so a table of fewer heads is a
+    # prefix of a table of more, and row h is not row 0 again
+    assert np.array_equal(s[:2], tables.rotation_signs(7, 128, 2))
+    for h in range(4):
+        top = tables.splitmix64(7, np.arange(h * 128 + 1, h * 128 + 129)) >> np.uint64(63)
+        assert np.array_equal(s[h] == -1.0, top == 1)
+    assert not any(np.array_equal(s[0], s[h]) for h in range(1, 4))
     assert abs(np.mean(tables.rotation_signs(1, 256, 64))) < 0.02
 
 

@@ -52,8 +52,51 @@ def test_static_scratch_matches_workspace_entry_point(cuda_ok, B, Hq, Hkv, N):
         lg = torch.full((B, Hq, 1, N), float("nan"), device="cuda")
         assert _static_call(lay, dev, q, cache, V, Hkv, out, lg) == _lib.OCTO_OK
         torch.cuda.synchronize()
+        assert _status() == 0  # no bounded on-chip wait expired
         got = out.cpu().numpy()
         assert np.all(np.abs(got - ref) <= tol), f"call {call}: max err {np.max(np.abs(got - ref))}"
+        assert torch.allclose(lg, ref_lg, rtol=0, atol=1e-4 * float(ref_lg.abs().max()))
+
+
+def _status():
+    st = ctypes.c_int(-1)
+    assert _lib.lib().octo_decode_attn_static_status(ctypes.byref(st), torch.cuda.current_stream().cuda_stream) == 0
+    return st.value
+
+
+def test_static_scratch_cleared_after_garbage_and_a_wider_call(cuda_ok):
+    """Each call must clear the status word and arrival counters itself: the
+    array is filled with 0xff bytes (what an interrupted call could leave:
+    a set status bit, counters far from zero) before the first call, and a
+    call over more cache heads precedes one over fewer, so the narrower
+    call's counters sit where the wider call's were. Without the clearing
+    the ticket never reaches the last split and the outputs stay NaN, or the
+    status word reads nonzero."""
+    d, b = 128, 3
+    lay = api.Layout(d, b)
+    shapes = [(2, 32, 8, 24000), (1, 8, 2, 9000)]  # wider first, then narrower
+    Hkv_max = 8
+    dev = api.DeviceTables(*parity.oracle_tables(d, b), tables.rotation_signs(0, d, Hkv_max))
+    assert _lib.lib().octo_decode_attn_static_fill(0xFF, torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert _status() == -1  # every byte 0xff
+    for B, Hq, Hkv, N in shapes:
+        keys = torch.from_numpy(inputs.to_bf16(inputs.llm_keys(5, B * Hkv, N, d))).to(torch.bfloat16).cuda()
+        V = torch.from_numpy(inputs.to_bf16(inputs.normal(6, (B * Hkv, N, d)))).to(torch.bfloat16).cuda()
+        q = torch.from_numpy(inputs.to_bf16(inputs.normal(7, (B, Hq, 1, d)))).to(torch.bfloat16).cuda()
+        cache = api.Cache.empty(lay, B * Hkv, N)
+        api.encode(lay, dev, keys, cache)
+        ref, ref_lg = api.decode_attn(lay, dev, q, cache, V, Hkv, logits=True)
+        torch.cuda.synchronize()
+        ref = ref.cpu().numpy()
+        out = torch.full((B, Hq, 1, d), float("nan"), device="cuda")
+        lg = torch.full((B, Hq, 1, N), float("nan"), device="cuda")
+        assert _static_call(lay, dev, q, cache, V, Hkv, out, lg) == _lib.OCTO_OK
+        torch.cuda.synchronize()
+        assert _status() == 0
+        got = out.cpu().numpy()
+        tol = 2e-3 * np.max(np.abs(ref), axis=-1, keepdims=True)
+        assert np.all(np.abs(got - ref) <= tol), f"{(B, Hq, Hkv, N)}: max err {np.nanmax(np.abs(got - ref))}"
         assert torch.allclose(lg, ref_lg, rtol=0, atol=1e-4 * float(ref_lg.abs().max()))
 
 
