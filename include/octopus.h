@@ -106,7 +106,7 @@ typedef struct octo_tables {
   const float* rho_c;  /* [n_rho]     norm centroids, increasing */
   const float* rho_t;  /* [n_rho-1]   norm thresholds */
   const float* signs;  /* [n_heads][d] +1/-1 diagonal of the sign-flipped WHT */
-  const float* qjl_S;  /* [n_heads][d][d] row-major Gaussian projection; NULL unless layout.qjl */
+  const float* qjl_S;  /* [n_heads][d][d] row-major Gaussian projection, 16-byte aligned; NULL unless layout.qjl */
   int64_t n_heads;     /* rows in signs / qjl_S, >= 1 */
 } octo_tables;
 

@@ -189,7 +189,7 @@ int octo::decode_validate(const octo_layout* L, const octo_tables* tab, const vo
   if (V && misaligned(V)) return OCTO_EINVAL;
   // code rows are staged by 16-byte bulk copies
   if (cache_cap % 4 != 0 || misaligned(packed) || misaligned(gamma)) return OCTO_EINVAL;
-  if (L->qjl && (misaligned(qjl_bits) || misaligned(qjl_norm))) return OCTO_EINVAL;
+  if (L->qjl && (misaligned(qjl_bits) || misaligned(qjl_norm) || misaligned(tab->qjl_S))) return OCTO_EINVAL;
   if (!(scale == scale)) return OCTO_EINVAL;
   if ((Hq / Hkv) * Lq > 8) return OCTO_EUNSUPPORTED;
   if (static_cast<int64_t>(B) * Hkv > 65535) return OCTO_EUNSUPPORTED;  // grid.y limit

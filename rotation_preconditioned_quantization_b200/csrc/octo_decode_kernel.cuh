@@ -170,6 +170,12 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = pack_bf16x2(r0, r1);
 }
 
+// bf16 hi + lo of (z, 0): the zero half needs no arithmetic.
+__device__ __forceinline__ void split_bf16_z0(float z, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(z, 0.0f);
+  lo = pack_bf16x2(z - bf16_lo(hi), 0.0f);
+}
+
 // 2^x with the hardware approximation (PTX ex2.approx: relative error about
 // 2^-22, 2^-inf = 0); softmax weights need far less.
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -741,6 +747,9 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // warps release a stage on its empty barrier. The load/store unit then only
 // serves shared-memory reads, and no consumer ever waits on a copy issue.
 // ---------------------------------------------------------------------------
+#ifndef OCTO_DECODE_SR_MIN_B
+#define OCTO_DECODE_SR_MIN_B 4  // bit budgets from which the norm is looked up apart from the direction
+#endif
 #ifndef OCTO_DECODE_TC_STAGES
 #define OCTO_DECODE_TC_STAGES 4  // rounds in flight at most (shared-memory stages; fewer when they do not fit)
 #endif
@@ -793,11 +802,21 @@ struct TcCfg {
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  // table over the positive-level quadrant: (m_xi, m_eta, i_rho)
-  static constexpr int NE = 1 << (3 * B - 1);
+  // Decoded-triplet table. For b <= 3 it covers the positive-level quadrant
+  // (m_xi, m_eta, i_rho) with rho_hat * n_hat pre-split into bf16 hi + lo.
+  // For b >= OCTO_DECODE_SR_MIN_B ("split rho") that table would have 2048
+  // entries, too many to replicate in shared memory, so the direction and
+  // the norm are looked up apart: n_hat of the quadrant (m_xi, m_eta) as
+  // fp32, and a small table of signed norm pairs (s_x rho_hat, s_y rho_hat)
+  // indexed by (s_xi, s_eta, i_rho); the product and the hi + lo split are
+  // formed in registers (the same fp32 product, so the same fragments).
+  static constexpr bool SR = B >= OCTO_DECODE_SR_MIN_B;
+  static constexpr int NE = SR ? (1 << (2 * B)) : (1 << (3 * B - 1));
   // replicas: 8 give every lane of a quarter-warp its own bank group (no
-  // conflicts); the 2048-entry b = 4 table keeps 2 to stay in shared memory
+  // conflicts); a full 2048-entry b = 4 table keeps 2 to stay in shared memory
   static constexpr int REP = NE <= 256 ? 8 : 2;
+  static constexpr int NSR = SR ? (1 << (B + 1)) : 0;  // signed norm pairs (s_x, s_y, i_rho)
+  static constexpr int REP_SR = 16;                    // one 8-byte slot per lane of a half-warp
   static constexpr int NKS = (T + 3) / 4;    // logit k-steps (4 triplets each)
   static constexpr bool HL = G <= 4;         // hi and lo halves side by side in the MMA columns
   static constexpr int NB = HL ? 2 : 4;      // query B-fragment registers per k-step
@@ -821,7 +840,7 @@ struct TcCfg {
   static constexpr int ST_END = ST_N + (QJL ? (4 * RK + 127) / 128 * 128 : 0);
   static constexpr int STAGE = (ST_END + 1023) / 1024 * 1024;
   static constexpr int PS = KW + 8;          // P row stride (floats)
-  static constexpr size_t TABLE = sizeof(uint4) * NE * REP;
+  static constexpr size_t TABLE = sizeof(uint4) * NE * REP + sizeof(float2) * NSR * REP_SR;
   static constexpr size_t QROW = (12 * NKS > D + 4 ? 12 * NKS : D + 4);  // padded rotated query row
   static constexpr size_t SCRATCH = (sizeof(float) * G * (QROW + (QJL ? D : 0)) + 15) / 16 * 16;
   static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per consumer warp
@@ -873,10 +892,9 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t& r0, uint32_t& r1, uint32
                : "r"(smem_u32(p)));
 }
 
-__device__ __forceinline__ uint32_t pm1_bf16x2(uint32_t bit_lo, uint32_t bit_hi) {
-  // +1 / -1 in bf16 (0x3F80 / 0xBF80) for sketch bits 1 / 0
-  return 0xBF80BF80u ^ ((bit_lo & 1u) << 15) ^ ((bit_hi & 1u) << 31);
-}
+// +1 / -1 in bf16 (0x3F80 / 0xBF80) for the bits at positions 15 and 31 of x
+// being 1 / 0 (low and high half of the pair).
+__device__ __forceinline__ uint32_t pm1_signs(uint32_t x) { return (x & 0x80008000u) ^ 0xBF80BF80u; }
 
 template <int D, int B, int G, bool QJL>
 __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
@@ -983,14 +1001,28 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   for (int e = tid; e < NE; e += Cfg::THREADS) {
     const int ix = static_cast<int>(HALF + (e & (HALF - 1))), iy = static_cast<int>(HALF + ((e >> B) & (HALF - 1)));
     float3 n = oct_inverse(s_dir_c[ix], s_dir_c[iy]);
-    const float r = s_rho_c[e >> (2 * B)];
-    n.x *= r; n.y *= r; n.z *= r;
-    uint32_t xyh, xyl, zh, zl;
-    split_bf16x2(n.x, n.y, xyh, xyl);
-    split_bf16x2(n.z, 0.0f, zh, zl);
-    const uint4 v = make_uint4(xyh, zh, xyl, zl);
+    uint4 v;
+    if constexpr (Cfg::SR) {
+      v = make_uint4(__float_as_uint(n.x), __float_as_uint(n.y), __float_as_uint(n.z), 0u);
+    } else {
+      const float r = s_rho_c[e >> (2 * B)];
+      n.x *= r; n.y *= r; n.z *= r;
+      uint32_t xyh, xyl, zh, zl;
+      split_bf16x2(n.x, n.y, xyh, xyl);
+      split_bf16x2(n.z, 0.0f, zh, zl);
+      v = make_uint4(xyh, zh, xyl, zl);
+    }
 #pragma unroll
     for (int k = 0; k < REP; ++k) table[e * REP + ((k + lane) & (REP - 1))] = v;
+  }
+  if constexpr (Cfg::SR) {
+    // signed norm pairs: entry s_x | s_y << 1 | i_rho << 2 holds (s_x ? -rho : rho, s_y ? -rho : rho)
+    float2* srt = reinterpret_cast<float2*>(table + NE * REP);
+    for (int e = tid; e < Cfg::NSR * Cfg::REP_SR; e += Cfg::THREADS) {
+      const int idx = e / Cfg::REP_SR;
+      const float r = s_rho_c[idx >> 2];
+      srt[e] = make_float2((idx & 1) ? -r : r, (idx & 2) ? -r : r);
+    }
   }
   // rotate the query rows: warp r handles row r
   if (warp < G) {
@@ -1003,15 +1035,39 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   }
   __syncthreads();
   if constexpr (QJL) {
-    float* p = scratch + G * QROW;  // [G][D]: p_r = S q_rot_r
+    // p_r = S q_rot_r. Four lanes share a row m of S, each taking a quarter
+    // of it with 16-byte loads (a warp reads 8 rows, 2 KB contiguous), and
+    // their partial dot products for every query row meet by two shuffles.
+    float* p = scratch + G * QROW;  // [G][D]
     const float* S = a.qjl_S + trow * D * D;
-    for (int j = tid; j < G * D; j += Cfg::THREADS) {
-      const int r = j / D, m = j - r * D;
-      const float* qrow = scratch + r * QROW;
-      const float* srow = S + static_cast<int64_t>(m) * D;
-      float acc = 0.0f;
-      for (int t = 0; t < D; ++t) acc = fmaf(__ldg(srow + t), qrow[t], acc);
-      p[j] = acc;
+    constexpr int NWT = Cfg::THREADS / 32, TPL = D / 4;
+    const int part = lane & 3;
+    for (int m0 = warp * 8; m0 < D; m0 += NWT * 8) {
+      const int m = m0 + (lane >> 2);
+      const float4* srow = reinterpret_cast<const float4*>(S + static_cast<int64_t>(m) * D + part * TPL);
+      float4 sv[TPL / 4];
+#pragma unroll
+      for (int i = 0; i < TPL / 4; ++i) sv[i] = __ldg(srow + i);
+      float acc[G];
+#pragma unroll
+      for (int r = 0; r < G; ++r) {
+        const float4* qv = reinterpret_cast<const float4*>(scratch + r * QROW + part * TPL);
+        float s0 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < TPL / 4; ++i) {
+          const float4 q4 = qv[i];
+          s0 = fmaf(sv[i].x, q4.x, s0);
+          s0 = fmaf(sv[i].y, q4.y, s0);
+          s0 = fmaf(sv[i].z, q4.z, s0);
+          s0 = fmaf(sv[i].w, q4.w, s0);
+        }
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        acc[r] = s0 + __shfl_xor_sync(0xffffffffu, s0, 2);
+      }
+      if (part == 0) {
+#pragma unroll
+        for (int r = 0; r < G; ++r) p[r * D + m] = acc[r];
+      }
     }
     __syncthreads();
   }
@@ -1040,15 +1096,19 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
       bq[s][0] = xyh; bq[s][1] = zh; bq[s][NB - 2] = xyl; bq[s][NB - 1] = zl;
     }
   }
-  // sketch B fragments: p row, sketch coordinates 16 ks + {2c4, 2c4+1 | 2c4+8, 2c4+9}
+  // Sketch B fragments. The sketch contraction's k order is a relabelling of
+  // the coordinates chosen so that a lane's A fragments are its sketch word
+  // shifted: in k-step ks, lane c4 takes word ks / 2 and bit j0 = 8 (ks & 1) +
+  // 2 c4; k = 2c4, 2c4+1 are the word's bits j0, j0 + 16 and k = 2c4+8, 2c4+9
+  // its bits j0 + 1, j0 + 17 (over the four lanes and two k-steps: all 32 bits).
   uint32_t bp[QJL ? QKS : 1][NB];
   if constexpr (QJL) {
 #pragma unroll
     for (int ks = 0; ks < QKS; ++ks) {
       float p0 = 0.0f, p1 = 0.0f, p8 = 0.0f, p9 = 0.0f;
       if (brow < G) {
-        const float* prow = scratch + G * QROW + brow * D + 16 * ks + 2 * c4;
-        p0 = prow[0]; p1 = prow[1]; p8 = prow[8]; p9 = prow[9];
+        const float* prow = scratch + G * QROW + brow * D + 32 * (ks >> 1) + 8 * (ks & 1) + 2 * c4;
+        p0 = prow[0]; p1 = prow[16]; p8 = prow[1]; p9 = prow[17];
       }
       uint32_t h01, l01, h89, l89;
       split_bf16x2(p0, p1, h01, l01);
@@ -1064,13 +1124,22 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   // where this lane's triplet code of each k-step sits in a key's bit stream
   // (word << 8 | shift). A padding triplet (t >= T) reads code 0's position:
   // its query coordinates are zero, so whatever entry it finds adds nothing.
+  // With split norm tables the code is taken from bit p - 7 of the stream, so
+  // that it arrives shifted left by 7 (the byte offset of a 128-byte table
+  // row); rows are then counted from -1 (+1 in cpos) and the first code of
+  // the stream comes from the pair (row -1, row 0) shifted by 25 - the seven
+  // low bits read from row -1 (other shared data) fall below the masks.
+  constexpr int PRE = Cfg::SR ? 7 : 0;
   uint32_t cpos[NKS];
 #pragma unroll
   for (int s = 0; s < NKS; ++s) {
     const int t = 4 * s + c4;
-    cpos[s] = t < T ? (static_cast<uint32_t>((t * C) >> 5) << 8) | static_cast<uint32_t>((t * C) & 31) : 0u;
+    const int p = (t < T ? t * C : 0) - PRE + (Cfg::SR ? 32 : 0);
+    cpos[s] = (static_cast<uint32_t>(p >> 5) << 8) | static_cast<uint32_t>(p & 31);
   }
   const int rep_off = lane & (REP - 1);
+  const uint32_t rep16 = static_cast<uint32_t>(rep_off) * 16u;                      // byte offset of this lane's replica
+  const uint32_t sr8 = static_cast<uint32_t>(lane & (Cfg::REP_SR - 1)) * 8u;       // ... in the signed norm table
 
   // ------------------------------------------------ main loop
   // This lane's query columns: HL lanes c4 and c4 ^ 2 hold the same two rows
@@ -1121,7 +1190,8 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         float acc[NC][4];
   #pragma unroll
         for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
-        const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + warp * Cfg::CW) + 2 * g8;
+        const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + warp * Cfg::CW) + 2 * g8 -
+                             (Cfg::SR ? KW : 0);
   #pragma unroll
         for (int s = 0; s < NKS; ++s) {
           // the code may straddle words wi and wi + 1; for the last word the
@@ -1130,13 +1200,40 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
           const uint2 lo = *reinterpret_cast<const uint2*>(bk + wi * KW);
           const uint2 hi = *reinterpret_cast<const uint2*>(bk + (wi + 1) * KW);
           const uint32_t cm = (1u << C) - 1u;
-          const uint32_t cA = __funnelshift_r(lo.x, hi.x, sh) & cm, cB = __funnelshift_r(lo.y, hi.y, sh) & cm;
-          uint4 eA = table[quadrant_index<B>(cA) * REP + rep_off];
-          uint4 eB = table[quadrant_index<B>(cB) * REP + rep_off];
-          // the direction signs flip x and y of the hi and lo halves
-          const uint32_t sA = quadrant_signs<B>(cA), sB = quadrant_signs<B>(cB);
-          eA.x ^= sA; eA.z ^= sA;
-          eB.x ^= sB; eB.z ^= sB;
+          uint4 eA, eB;
+          if constexpr (Cfg::SR) {
+            // n_hat of the quadrant (fp32) times the signed norm pair, split into
+            // bf16 hi + lo. Byte offsets straight from the unmasked code:
+            // direction (m_xi, m_eta) = bits [0, 2B) at 16 REP bytes an entry;
+            // (s_x, s_y, i_rho) = bits [2B, 3B + 1) at 8 REP_SR bytes.
+            static_assert(REP * 16 == 128 && Cfg::REP_SR * 8 == 128, "entry strides of the split tables");
+            // c7 = code << 7 (low seven bits: neighbouring data)
+            const uint32_t c7A = __funnelshift_r(lo.x, hi.x, sh), c7B = __funnelshift_r(lo.y, hi.y, sh);
+            constexpr uint32_t DMB = ((1u << (2 * B)) - 1u) << 7, SMB = ((1u << (B + 1)) - 1u) << 7;
+            const unsigned char* tb = reinterpret_cast<const unsigned char*>(table);
+            const unsigned char* sb = tb + 16 * NE * REP;
+            const uint4 nA = *reinterpret_cast<const uint4*>(tb + ((c7A & DMB) | rep16));
+            const uint4 nB = *reinterpret_cast<const uint4*>(tb + ((c7B & DMB) | rep16));
+            const float2 rA = *reinterpret_cast<const float2*>(sb + (((c7A >> (2 * B)) & SMB) | sr8));
+            const float2 rB = *reinterpret_cast<const float2*>(sb + (((c7B >> (2 * B)) & SMB) | sr8));
+            // x, y take the signed norms, z takes |rho|
+            const float xA = __uint_as_float(nA.x) * rA.x, yA = __uint_as_float(nA.y) * rA.y;
+            const float zA = __uint_as_float(nA.z) * fabsf(rA.x);
+            const float xB = __uint_as_float(nB.x) * rB.x, yB = __uint_as_float(nB.y) * rB.y;
+            const float zB = __uint_as_float(nB.z) * fabsf(rB.x);
+            split_bf16x2(xA, yA, eA.x, eA.z);
+            split_bf16_z0(zA, eA.y, eA.w);
+            split_bf16x2(xB, yB, eB.x, eB.z);
+            split_bf16_z0(zB, eB.y, eB.w);
+          } else {
+            const uint32_t cA = __funnelshift_r(lo.x, hi.x, sh) & cm, cB = __funnelshift_r(lo.y, hi.y, sh) & cm;
+            eA = table[quadrant_index<B>(cA) * REP + rep_off];
+            eB = table[quadrant_index<B>(cB) * REP + rep_off];
+            // the direction signs flip x and y of the hi and lo halves
+            const uint32_t sA = quadrant_signs<B>(cA), sB = quadrant_signs<B>(cB);
+            eA.x ^= sA; eA.z ^= sA;
+            eB.x ^= sB; eB.z ^= sB;
+          }
           if constexpr (HL) {
             mma_bf16_16816(acc[0], eA.x, eB.x, eA.y, eB.y, bq[s][0], bq[s][1]);
             mma_bf16_16816(acc[1], eA.z, eB.z, eA.w, eB.w, bq[s][0], bq[s][1]);
@@ -1157,11 +1254,12 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
           float accq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   #pragma unroll
           for (int ks = 0; ks < QKS; ++ks) {
+            // bits j0 and j0 + 16 of the word move to the sign bits 15 and 31
+            // (bit 1: +1, bit 0: -1); a2, a3 take bits j0 + 1, j0 + 17
             const uint2 w2 = *reinterpret_cast<const uint2*>(qk + (ks >> 1) * RK);
-            const int shq = 16 * (ks & 1) + 2 * c4;
-            const uint32_t wA = w2.x >> shq, wB = w2.y >> shq;
-            const uint32_t a0 = pm1_bf16x2(wA, wA >> 1), a1 = pm1_bf16x2(wB, wB >> 1);
-            const uint32_t a2 = pm1_bf16x2(wA >> 8, wA >> 9), a3 = pm1_bf16x2(wB >> 8, wB >> 9);
+            const int shl = 15 - 8 * (ks & 1) - 2 * c4;
+            const uint32_t a0 = pm1_signs(w2.x << shl), a1 = pm1_signs(w2.y << shl);
+            const uint32_t a2 = pm1_signs(w2.x << (shl - 1)), a3 = pm1_signs(w2.y << (shl - 1));
             mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
             if constexpr (!HL) mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
           }

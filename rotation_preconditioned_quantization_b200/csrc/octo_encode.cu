@@ -541,6 +541,7 @@ extern "C" int octo_encode(const octo_layout* L, const octo_tables* tab, const v
     return OCTO_EINVAL;
   if (L->n_rho > 1 && !tab->rho_t) return OCTO_EINVAL;
   if (L->qjl && (!qjl_bits || !qjl_norm || !tab->qjl_S)) return OCTO_EINVAL;
+  if (L->qjl && reinterpret_cast<uintptr_t>(tab->qjl_S) % 16 != 0) return OCTO_EINVAL;
   if (head_stride < 0 || token_stride < 0) return OCTO_EINVAL;
   const int esz = key_dtype == OCTO_F32 ? 4 : 2;
   // each lane loads D/32 contiguous elements with one vector load
