@@ -720,7 +720,8 @@ def main():
         elif args.only == "encode_sweep":
             print(json.dumps({"encode_sweep": encode_sweep(dev, peak)}))
         else:
-            shapes = [w for w in (HEADLINE, *OTHER_WORKLOADS) if w.name.startswith(args.shape)]
+            known = (HEADLINE, *OTHER_WORKLOADS)
+            shapes = [w for w in known if w.name == args.shape] or [w for w in known if w.name.startswith(args.shape)]
             if len(shapes) != 1:
                 raise SystemExit(f"--shape {args.shape!r} names {len(shapes)} workloads")
             w = shapes[0]

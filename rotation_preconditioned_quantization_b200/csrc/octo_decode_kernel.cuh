@@ -170,6 +170,32 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = pack_bf16x2(r0, r1);
 }
 
+// Packed fp32 pairs (sm_100: one instruction for two lanes' worth of work):
+// (a.x b.x, a.y b.y), and x minus the bf16 hi halves of hi (x.x - lo half,
+// x.y - hi half), each rounded to nearest as the scalar operations would be.
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 sub_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " sub.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// split_bf16x2 of a pair with the two subtractions as one packed operation
+__device__ __forceinline__ void split_bf16x2_v(float2 v, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(v.x, v.y);
+  const float2 r = sub_f32x2(v, make_float2(bf16_lo(hi), bf16_hi(hi)));
+  lo = pack_bf16x2(r.x, r.y);
+}
+
 // bf16 hi + lo of (z, 0): the zero half needs no arithmetic.
 __device__ __forceinline__ void split_bf16_z0(float z, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16x2(z, 0.0f);
@@ -747,6 +773,9 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // warps release a stage on its empty barrier. The load/store unit then only
 // serves shared-memory reads, and no consumer ever waits on a copy issue.
 // ---------------------------------------------------------------------------
+#ifndef OCTO_DECODE_F32X2
+#define OCTO_DECODE_F32X2 1  // packed fp32 pairs for the split-norm products and residuals
+#endif
 #ifndef OCTO_DECODE_SR_MIN_B
 #define OCTO_DECODE_SR_MIN_B 4  // bit budgets from which the norm is looked up apart from the direction
 #endif
@@ -811,7 +840,11 @@ struct TcCfg {
   // indexed by (s_xi, s_eta, i_rho); the product and the hi + lo split are
   // formed in registers (the same fp32 product, so the same fragments).
   static constexpr bool SR = B >= OCTO_DECODE_SR_MIN_B;
-  static constexpr int NE = SR ? (1 << (2 * B)) : (1 << (3 * B - 1));
+  // A code of at most 8 bits (b = 2) indexes a full table of every signed
+  // code directly (128 entries, 16 KB with 8 replicas): no quadrant index,
+  // no sign masks.
+  static constexpr bool FULL = !SR && C <= 8;
+  static constexpr int NE = SR ? (1 << (2 * B)) : (FULL ? (1 << C) : (1 << (3 * B - 1)));
   // replicas: 8 give every lane of a quarter-warp its own bank group (no
   // conflicts); a full 2048-entry b = 4 table keeps 2 to stay in shared memory
   static constexpr int REP = NE <= 256 ? 8 : 2;
@@ -1005,7 +1038,14 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
     if constexpr (Cfg::SR) {
       v = make_uint4(__float_as_uint(n.x), __float_as_uint(n.y), __float_as_uint(n.z), 0u);
     } else {
-      const float r = s_rho_c[e >> (2 * B)];
+      // quadrant entries: the norm index sits above the magnitudes; full
+      // entries: above the two direction signs, which flip x and y (the
+      // codebook and the inverse map are odd in each coordinate)
+      const float r = s_rho_c[Cfg::FULL ? (e >> (2 * B + 2)) : (e >> (2 * B))];
+      if constexpr (Cfg::FULL) {
+        if ((e >> (2 * B)) & 1) n.x = -n.x;
+        if ((e >> (2 * B + 1)) & 1) n.y = -n.y;
+      }
       n.x *= r; n.y *= r; n.z *= r;
       uint32_t xyh, xyl, zh, zl;
       split_bf16x2(n.x, n.y, xyh, xyl);
@@ -1129,12 +1169,13 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   // row); rows are then counted from -1 (+1 in cpos) and the first code of
   // the stream comes from the pair (row -1, row 0) shifted by 25 - the seven
   // low bits read from row -1 (other shared data) fall below the masks.
-  constexpr int PRE = Cfg::SR ? 7 : 0;
+  constexpr bool PRESHIFT = Cfg::SR || Cfg::FULL;
+  constexpr int PRE = PRESHIFT ? 7 : 0;
   uint32_t cpos[NKS];
 #pragma unroll
   for (int s = 0; s < NKS; ++s) {
     const int t = 4 * s + c4;
-    const int p = (t < T ? t * C : 0) - PRE + (Cfg::SR ? 32 : 0);
+    const int p = (t < T ? t * C : 0) - PRE + (PRESHIFT ? 32 : 0);
     cpos[s] = (static_cast<uint32_t>(p >> 5) << 8) | static_cast<uint32_t>(p & 31);
   }
   const int rep_off = lane & (REP - 1);
@@ -1191,7 +1232,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   #pragma unroll
         for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
         const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + warp * Cfg::CW) + 2 * g8 -
-                             (Cfg::SR ? KW : 0);
+                             (PRESHIFT ? KW : 0);
   #pragma unroll
         for (int s = 0; s < NKS; ++s) {
           // the code may straddle words wi and wi + 1; for the last word the
@@ -1217,14 +1258,29 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
             const float2 rA = *reinterpret_cast<const float2*>(sb + (((c7A >> (2 * B)) & SMB) | sr8));
             const float2 rB = *reinterpret_cast<const float2*>(sb + (((c7B >> (2 * B)) & SMB) | sr8));
             // x, y take the signed norms, z takes |rho|
+#if OCTO_DECODE_F32X2
+            const float2 xyA = mul_f32x2(make_float2(__uint_as_float(nA.x), __uint_as_float(nA.y)), rA);
+            const float2 xyB = mul_f32x2(make_float2(__uint_as_float(nB.x), __uint_as_float(nB.y)), rB);
+            split_bf16x2_v(xyA, eA.x, eA.z);
+            split_bf16x2_v(xyB, eB.x, eB.z);
+#else
             const float xA = __uint_as_float(nA.x) * rA.x, yA = __uint_as_float(nA.y) * rA.y;
-            const float zA = __uint_as_float(nA.z) * fabsf(rA.x);
             const float xB = __uint_as_float(nB.x) * rB.x, yB = __uint_as_float(nB.y) * rB.y;
-            const float zB = __uint_as_float(nB.z) * fabsf(rB.x);
             split_bf16x2(xA, yA, eA.x, eA.z);
-            split_bf16_z0(zA, eA.y, eA.w);
             split_bf16x2(xB, yB, eB.x, eB.z);
+#endif
+            const float zA = __uint_as_float(nA.z) * fabsf(rA.x);
+            const float zB = __uint_as_float(nB.z) * fabsf(rB.x);
+            split_bf16_z0(zA, eA.y, eA.w);
             split_bf16_z0(zB, eB.y, eB.w);
+          } else if constexpr (Cfg::FULL) {
+            // the pre-shifted code is the entry's byte offset (128 bytes an entry)
+            static_assert(REP * 16 == 128, "entry stride of the full table");
+            constexpr uint32_t FMB = ((1u << C) - 1u) << 7;
+            const uint32_t c7A = __funnelshift_r(lo.x, hi.x, sh), c7B = __funnelshift_r(lo.y, hi.y, sh);
+            const unsigned char* tb = reinterpret_cast<const unsigned char*>(table);
+            eA = *reinterpret_cast<const uint4*>(tb + ((c7A & FMB) | rep16));
+            eB = *reinterpret_cast<const uint4*>(tb + ((c7B & FMB) | rep16));
           } else {
             const uint32_t cA = __funnelshift_r(lo.x, hi.x, sh) & cm, cB = __funnelshift_r(lo.y, hi.y, sh) & cm;
             eA = table[quadrant_index<B>(cA) * REP + rep_off];
