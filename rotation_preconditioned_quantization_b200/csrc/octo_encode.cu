@@ -83,20 +83,6 @@ struct EncCfg {
   static_assert(KT >= 8, "tile of keys");
 };
 
-// Direction field of a triplet code from the ordered cells (ix, iy): the
-// symmetric codebook's cell i is stored as a sign s (1 for the lower half,
-// i < 2^B) and the rank m of |level| among the positive levels, as
-// m_x | m_y << B | s_x << 2B | s_y << (2B + 1); XOR with all ones maps a
-// lower-half cell onto its mirror.
-template <int B>
-__device__ __forceinline__ uint32_t direction_field(int ix, int iy) {
-  constexpr uint32_t half = 1u << B, ones = (2u << B) - 1u;
-  const uint32_t sx = static_cast<uint32_t>(ix) < half, sy = static_cast<uint32_t>(iy) < half;
-  const uint32_t mx = (static_cast<uint32_t>(ix) ^ (sx ? ones : 0u)) & (half - 1u);
-  const uint32_t my = (static_cast<uint32_t>(iy) ^ (sy ? ones : 0u)) & (half - 1u);
-  return mx | (my << B) | (sx << (2 * B)) | (sy << (2 * B + 1));
-}
-
 // x as a tf32 head plus a tf32 remainder (x - head), each in a 32-bit register.
 __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
@@ -139,6 +125,15 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
   float* U = reinterpret_cast<float*>(nhat + NB * NB * REP);          // [KT][US]
   uint16_t* codes = reinterpret_cast<uint16_t*>(U + KT * US);         // [KT][T]
   __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[8], s_rho_t[8];
+  // Cell search tables: s_tpad[i] = threshold i - 1 (-inf, +inf at the ends),
+  // so cell i is s_tpad[i] <= x < s_tpad[i + 1]; s_bin[k] = the cell of the
+  // left edge of bin k of 128 equal bins over [-1, 1]. With at most one
+  // threshold per bin, the bin's cell is within one of x's cell.
+  __shared__ float s_tpad[34];
+  __shared__ uint8_t s_bin[128];
+  // code-field parts of a direction cell: x's (m | s << 2B) and y's (m << B | s << 2B + 1)
+  __shared__ uint16_t s_fx[32], s_fy[32];
+  __shared__ int s_bins_ok;
   __shared__ uint32_t sketch[QJL ? KT * (D / 32) : 1];  // [KT][D/32] sketch words of the tile (QJL)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -148,6 +143,27 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
   if (tid < NDIR - 1) s_dir_t[tid] = a.dir_t[tid];
   if (tid < NRHO) s_rho_c[tid] = a.rho_c[tid];
   if (tid < NRHO - 1) s_rho_t[tid] = a.rho_t[tid];
+  if (tid == 0) s_bins_ok = 1;
+  __syncthreads();
+  if (tid <= NDIR) s_tpad[tid] = tid == 0 ? -INFINITY : (tid == NDIR ? INFINITY : s_dir_t[tid - 1]);
+  if (tid < 128) {
+    const float left = -1.0f + static_cast<float>(tid) * (1.0f / 64.0f);
+    int c = 0;
+    for (int k = 0; k < NDIR - 1; ++k) c += s_dir_t[k] <= left;
+    s_bin[tid] = static_cast<uint8_t>(c);
+  }
+  if (tid < NDIR - 2) {  // two thresholds in one bin: the bin search would be off by two
+    const int b0 = static_cast<int>(floorf((s_dir_t[tid] + 1.0f) * 64.0f));
+    const int b1 = static_cast<int>(floorf((s_dir_t[tid + 1] + 1.0f) * 64.0f));
+    if (b0 == b1) atomicAnd(&s_bins_ok, 0);
+  }
+  if (tid < NDIR) {
+    constexpr uint32_t half = 1u << B, ones = (2u << B) - 1u;
+    const uint32_t sg = static_cast<uint32_t>(tid) < half;
+    const uint32_t m = (static_cast<uint32_t>(tid) ^ (sg ? ones : 0u)) & (half - 1u);
+    s_fx[tid] = static_cast<uint16_t>(m | (sg << (2 * B)));
+    s_fy[tid] = static_cast<uint16_t>((m << B) | (sg << (2 * B + 1)));
+  }
   __syncthreads();
   // a border cell holds NaN: its s = n . t is NaN, and "s > best" is false
   for (int e = tid; e < NB * NB; e += Cfg::THREADS) {
@@ -171,7 +187,17 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
   // Cell of x in the direction codebook: start from the uniform-grid cell
   // and step to the exact one (cell i has t[i-1] <= x < t[i]; the Lloyd-Max
   // thresholds are close to uniform, so this takes 0-1 steps).
+  const bool bins_ok = s_bins_ok != 0;
   auto dir_index = [&](float x) -> int {
+    if (bins_ok) {
+      // bin of x by rounding (x + 1) * 64 to an integer in the mantissa of
+      // 1.5 * 2^23 + (x + 1) * 64; the bin's cell, then one step either way
+      const int bi = min(__float_as_int(fmaf(x, 64.0f, 12582912.0f + 64.0f)) - 0x4B400000, 127);
+      int i = s_bin[bi];
+      i += x >= s_tpad[i + 1];
+      i -= x < s_tpad[i];
+      return i;
+    }
     int i = __float2int_rd((x + 1.0f) * (0.5f * NDIR));
     i = i < 0 ? 0 : (i > NDIR - 1 ? NDIR - 1 : i);
     while (i > 0 && x < s_dir_t[i - 1]) --i;
@@ -298,17 +324,16 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
       const int k = j / T, i = j - k * T;
       float* tp = U + k * US + 3 * i;
       const float x = tp[0], y = tp[1], z = tp[2];
-      const float l1 = fabsf(x) + fabsf(y) + fabsf(z);
-      float px = 0.0f, py = 0.0f, pz = 1.0f;
-      if (l1 > 0.0f) {
-        const float il = 1.0f / l1;
-        px = x * il; py = y * il; pz = z * il;
-      }
-      float xi = px, eta = py;
-      if (!(pz >= 0.0f)) {
-        xi = (1.0f - fabsf(py)) * (px >= 0.0f ? 1.0f : -1.0f);
-        eta = (1.0f - fabsf(px)) * (py >= 0.0f ? 1.0f : -1.0f);
-      }
+      const float ax = fabsf(x), ay = fabsf(y);
+      const float l1 = ax + ay + fabsf(z);
+      // p = t / ||t||_1 (a zero triplet maps to the north pole); the lower
+      // hemisphere (p_z < 0) folds to ((1 - |p_y|) sgn p_x, (1 - |p_x|) sgn p_y)
+      const float il = l1 > 0.0f ? __fdividef(1.0f, l1) : 0.0f;
+      const bool lower = z < 0.0f;
+      const float fx = lower ? fmaf(-ay, il, 1.0f) : ax * il;
+      const float fy = lower ? fmaf(-ax, il, 1.0f) : ay * il;
+      const float xi = x >= 0.0f ? fx : -fx;
+      const float eta = y >= 0.0f ? fy : -fy;
       int ix = dir_index(xi);
       int iy = dir_index(eta);
       int ir;
@@ -340,7 +365,7 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
         if constexpr (QJL) nb = nc[((kbest / 3 - 1) * NB + (kbest % 3 - 1)) * REP];
         rho_level(sbest, ir, rh);
       }
-      codes[k * T + i] = static_cast<uint16_t>(direction_field<B>(ix, iy) | (ir << (2 * Cfg::BD)));
+      codes[k * T + i] = static_cast<uint16_t>(s_fx[ix] | s_fy[iy] | (ir << (2 * Cfg::BD)));
       if constexpr (QJL) {
         // residual e = t - rho_hat n_hat, in place (the pad coordinate is dropped later)
         tp[0] = x - rh * nb.x;
