@@ -83,11 +83,14 @@ struct EncCfg {
   static_assert(KT >= 8, "tile of keys");
 };
 
-// x as a tf32 head plus a tf32 remainder (x - head), each in a 32-bit register.
+// x as a tf32 head (rounded to nearest) plus the exact fp32 remainder x -
+// head. The remainder is passed to the MMA as it is: the tensor core reads
+// the tf32 part of the register (truncating it), which is within 2^-10 of
+// the remainder, itself at most 2^-11 |x| - so head + remainder carries x to
+// about 2^-21.
 __device__ __forceinline__ void tf32_split(float x, uint32_t& hi, uint32_t& lo) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-  const float r = x - __uint_as_float(hi);
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+  lo = __float_as_uint(x - __uint_as_float(hi));
 }
 
 // D += A B for one m16n8k8 tile with tf32 operands and fp32 accumulation.
@@ -403,7 +406,9 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
         // S fragments of a k-step serve the whole group.
         constexpr int MT = D / 16;                  // row tiles of S
         constexpr int NT = (KT + 7) / 8;            // key tiles
-        constexpr int NGT = 4;                      // key tiles per work item
+        // key tiles per work item: all of the tile's when that gives one item per
+        // warp (the S fragments of a k-step are split once for every key)
+        constexpr int NGT = (MT == NWARP && NT <= 8) ? NT : 4;
         constexpr int NG = (NT + NGT - 1) / NGT;
         const float* Sh = a.qjl_S + (h % a.table_heads) * D * D;
         const int g8 = lane >> 2, c4 = lane & 3;
