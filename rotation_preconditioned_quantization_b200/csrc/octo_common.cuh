@@ -87,6 +87,71 @@ __device__ __forceinline__ void fwht_warp(float (&v)[E], int lane) {
   }
 }
 
+// Packed fp32 pairs (sm_100 add/sub/mul/fma .f32x2): one instruction does
+// the two lanes' IEEE round-to-nearest operations, so results are the same
+// as with scalar operations.
+#define OCTO_F32X2_OP(name, op)                                                                         \
+  __device__ __forceinline__ float2 name(float2 a, float2 b) {                                         \
+    float2 d;                                                                                           \
+    asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n " op           \
+        ".rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"                                            \
+        : "=f"(d.x), "=f"(d.y)                                                                          \
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));                                                      \
+    return d;                                                                                           \
+  }
+OCTO_F32X2_OP(add_f32x2, "add")
+OCTO_F32X2_OP(sub_f32x2, "sub")
+OCTO_F32X2_OP(mul_f32x2, "mul")
+#undef OCTO_F32X2_OP
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// Walsh-Hadamard butterflies over the 32 register coordinates of a lane
+// (coordinate bits 0-4, Sylvester order): the stage over bit 0 pairs
+// neighbouring registers and runs scalar; the stages over bits 1-4 pair
+// register pairs (2i, 2i+1), two butterflies per packed add and sub.
+__device__ __forceinline__ void fwht32_regs(float (&v)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float a = v[e], b = v[e + 1];
+    v[e] = a + b;
+    v[e + 1] = a - b;
+  }
+#pragma unroll
+  for (int hh = 2; hh < 32; hh <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      if ((e & hh) == 0) {
+        const float2 a = make_float2(v[e], v[e + 1]), b = make_float2(v[e + hh], v[e + hh + 1]);
+        const float2 s = add_f32x2(a, b), d = sub_f32x2(a, b);
+        v[e] = s.x; v[e + 1] = s.y; v[e + hh] = d.x; v[e + hh + 1] = d.y;
+      }
+    }
+  }
+}
+
+// The butterfly stages across the LK lanes of a key (lane bits 0..log2(LK)-1):
+// lower lane v + o, upper lane o - v, as fma(+-1, v, o) on register pairs.
+template <int LK>
+__device__ __forceinline__ void fwht32_lanes(float (&v)[32], int lane) {
+#pragma unroll
+  for (int m = 1; m < LK; m <<= 1) {
+    const float sg = (lane & m) != 0 ? -1.0f : 1.0f;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const float2 o = make_float2(__shfl_xor_sync(0xffffffffu, v[e], m), __shfl_xor_sync(0xffffffffu, v[e + 1], m));
+      const float2 r = fma_f32x2(make_float2(sg, sg), make_float2(v[e], v[e + 1]), o);
+      v[e] = r.x; v[e + 1] = r.y;
+    }
+  }
+}
+
 // Inverse octahedral map of (a, b) = (xi, eta), normalised (explainer,
 // "octahedral folding": r = 1 - |xi| - |eta|; unfold when r < 0; normalise).
 __device__ __forceinline__ float3 oct_inverse(float a, float b) {

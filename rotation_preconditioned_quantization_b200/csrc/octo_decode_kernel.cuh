@@ -170,25 +170,6 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   lo = pack_bf16x2(r0, r1);
 }
 
-// Packed fp32 pairs (sm_100: one instruction for two lanes' worth of work):
-// (a.x b.x, a.y b.y), and x minus the bf16 hi halves of hi (x.x - lo half,
-// x.y - hi half), each rounded to nearest as the scalar operations would be.
-__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " mul.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-__device__ __forceinline__ float2 sub_f32x2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " sub.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
 // split_bf16x2 of a pair with the two subtractions as one packed operation
 __device__ __forceinline__ void split_bf16x2_v(float2 v, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16x2(v.x, v.y);

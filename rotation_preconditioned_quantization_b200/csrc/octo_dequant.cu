@@ -41,6 +41,7 @@ struct DequantArgs {
   void* out;
   int out_bf16;
   int out_v8;  // out is 32-byte aligned: 32-byte stores (whole sectors per lane)
+  int in_v4;   // token offset, capacity and cache pointers allow 16-byte staging copies
   int64_t n_heads, n_tokens, cache_cap, token_offset, table_heads;
   int64_t tiles_per_head, n_tiles;
 };
@@ -67,7 +68,10 @@ struct DqCfg {
   static constexpr int NWL = ((NT - 1) * C) / 32 + 3;
   static constexpr int WMAX = ((32 * (LK - 1) / 3) * C) / 32 + NWL;  // end of the last lane's window
   static constexpr int WP = WMAX > W ? WMAX : W;   // word planes held; planes >= W stay zero
-  static constexpr int CS = KT + 1;                // odd plane stride: a key's planes in distinct banks
+  // plane stride: 16-byte rows for the 16-byte staging copies; 4 mod 32
+  // words, so the lanes of a key (different planes, same column) mostly
+  // fall in different banks
+  static constexpr int CS = KT + 4;
   static constexpr size_t TABLE = sizeof(float4) * NE * REP;
   static constexpr size_t CBUF = (sizeof(uint32_t) * WP * CS + 15) / 16 * 16;
   static constexpr size_t SMEM = TABLE + 2 * CBUF + 2 * sizeof(float) * KT;  // two tile buffers
@@ -78,6 +82,13 @@ struct DqCfg {
 // 4-byte asynchronous global -> shared copy; bytes = 0 writes a zero.
 __device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(bytes)
+               : "memory");
+}
+// 16-byte asynchronous global -> shared copy (both addresses 16-byte
+// aligned); only the first `bytes` come from global memory, the rest are zeros.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src), "r"(bytes)
                : "memory");
 }
@@ -144,12 +155,26 @@ __global__ void __launch_bounds__(256, 3) dequant_kernel(DequantArgs a) {
     const int64_t tok0 = a.token_offset + ft0;
     const uint32_t* ph = a.packed + h * W * a.cache_cap + tok0;
     uint32_t* cw = cwb + bb * (Cfg::CBUF / 4);
-    for (int i = tid; i < W * KT; i += THREADS) {
-      const int w = i / KT, k = i - w * KT;
-      cp_async4(cw + w * CS + k, ph + static_cast<int64_t>(w) * a.cache_cap + min(k, fnk - 1), k < fnk ? 4u : 0u);
+    if (a.in_v4) {
+      // four tokens a copy; past the last token the copies read less (zeros)
+      constexpr int K4 = KT / 4;
+      for (int i = tid; i < W * K4; i += THREADS) {
+        const int w = i / K4, k = 4 * (i - w * K4);
+        const int n = max(0, min(4, fnk - k));
+        cp_async16(cw + w * CS + k, ph + static_cast<int64_t>(w) * a.cache_cap + (n > 0 ? k : 0), 4u * n);
+      }
+      if (tid < K4) {
+        const int k = 4 * tid, n = max(0, min(4, fnk - k));
+        cp_async16(gsb + bb * KT + k, a.gamma + h * a.cache_cap + tok0 + (n > 0 ? k : 0), 4u * n);
+      }
+    } else {
+      for (int i = tid; i < W * KT; i += THREADS) {
+        const int w = i / KT, k = i - w * KT;
+        cp_async4(cw + w * CS + k, ph + static_cast<int64_t>(w) * a.cache_cap + min(k, fnk - 1), k < fnk ? 4u : 0u);
+      }
+      if (tid < KT)
+        cp_async4(gsb + bb * KT + tid, a.gamma + h * a.cache_cap + tok0 + min(tid, fnk - 1), tid < fnk ? 4u : 0u);
     }
-    if (tid < KT)
-      cp_async4(gsb + bb * KT + tid, a.gamma + h * a.cache_cap + tok0 + min(tid, fnk - 1), tid < fnk ? 4u : 0u);
   };
 
   uint32_t smask = 0;  // bit p: s_j < 0 for this lane's coordinate 32 j + p, for head sg_head
@@ -311,6 +336,8 @@ extern "C" int octo_dequant(const octo_layout* L, const octo_tables* tab, int64_
   a.out = out;
   a.out_bf16 = out_dtype == OCTO_BF16;
   a.out_v8 = reinterpret_cast<uintptr_t>(out) % 32 == 0;
+  a.in_v4 = token_offset % 4 == 0 && cache_cap % 4 == 0 && reinterpret_cast<uintptr_t>(packed) % 16 == 0 &&
+            reinterpret_cast<uintptr_t>(gamma) % 16 == 0;
   a.n_heads = n_heads;
   a.n_tokens = n_tokens;
   a.cache_cap = cache_cap;

@@ -287,33 +287,18 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
 #pragma unroll
       for (int m = 1; m < LK; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
       const float g = sqrtf(ss);
-      const float ig = g > 0.0f ? 1.0f / g : 0.0f;
-      // u = k / gamma, then the signs s (exact)
+      // u_rot = H (s * k) / (gamma sqrt(d)): the signs s (exact) on the raw
+      // key, the butterflies, then one scale (0 for a zero key)
+      const float scale = g > 0.0f ? inv_sqrt_d / g : 0.0f;
 #pragma unroll
-      for (int q = 0; q < 32; ++q)
-        v[q] = __uint_as_float(__float_as_uint(v[q] * ig) ^ ((smask << (31 - q)) & 0x80000000u));
+      for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(__float_as_uint(v[q]) ^ ((smask << (31 - q)) & 0x80000000u));
       // H: coordinate bits 0-4 in registers, then bits 5.. across the key's lanes
-#pragma unroll
-      for (int hh = 1; hh < 32; hh <<= 1) {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          if ((q & hh) == 0) {
-            const float x0 = v[q], x1 = v[q + hh];
-            v[q] = x0 + x1;
-            v[q + hh] = x0 - x1;
-          }
-        }
-      }
-#pragma unroll
-      for (int m = 1; m < LK; m <<= 1) {
-        const float sgn = (lane & m) != 0 ? -1.0f : 1.0f;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = fmaf(sgn, v[q], __shfl_xor_sync(0xffffffffu, v[q], m));
-      }
+      fwht32_regs(v);
+      fwht32_lanes<LK>(v, lane);
       if (valid) {
         float* row = U + k * US;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) row[32 * jq + q] = v[q] * inv_sqrt_d;
+        for (int q = 0; q < 32; ++q) row[32 * jq + q] = v[q] * scale;
         if (jq == 0) {
           for (int q = D; q < 3 * T; ++q) row[q] = 0.0f;  // the zero pad of the last triplet
           a.gamma[h * a.cache_cap + a.token_offset + n0 + k] = g;
