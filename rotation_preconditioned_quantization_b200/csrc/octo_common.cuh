@@ -136,12 +136,13 @@ __device__ __forceinline__ void fwht32_regs(float (&v)[32]) {
   }
 }
 
-// The butterfly stages across the LK lanes of a key (lane bits 0..log2(LK)-1):
-// lower lane v + o, upper lane o - v, as fma(+-1, v, o) on register pairs.
-template <int LK>
+// The butterfly stages across the LK lanes of a key, lane j of the key
+// being lane j * STRIDE of the warp (lane bits log2(STRIDE) and up): lower
+// lane v + o, upper lane o - v, as fma(+-1, v, o) on register pairs.
+template <int LK, int STRIDE>
 __device__ __forceinline__ void fwht32_lanes(float (&v)[32], int lane) {
 #pragma unroll
-  for (int m = 1; m < LK; m <<= 1) {
+  for (int m = STRIDE; m < LK * STRIDE; m <<= 1) {
     const float sg = (lane & m) != 0 ? -1.0f : 1.0f;
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {

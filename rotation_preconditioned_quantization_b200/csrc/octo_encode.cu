@@ -221,11 +221,14 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
 
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
 
-  // Phase 1 layout: LK = D/32 lanes per key, lane j owning coordinates
-  // [32 j, 32 j + 32): 5 butterfly stages run in registers and log2(LK)
+  // Phase 1 layout: LK = D/32 lanes per key, lane jq owning coordinates
+  // [32 jq, 32 jq + 32): 5 butterfly stages run in registers and log2(LK)
   // across the key's lanes; a warp holds 32/LK keys at once.
   constexpr int LK = D / 32, KWP = 32 / LK;
-  const int jq = lane & (LK - 1), kslot = lane / LK;
+  // lane = jq * KWP + kslot: a quarter-warp holds 8 keys (or all of them) at
+  // one coordinate block, so its stores of the rotated rows (rows 4 mod 32
+  // words apart) fall in distinct bank groups
+  const int jq = lane / KWP, kslot = lane % KWP;
   uint32_t smask = 0;  // bit p: s < 0 at coordinate 32 jq + p of head smask_head
   int64_t smask_head = -1;
 
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
 #pragma unroll
       for (int q = 0; q < 32; ++q) ss = fmaf(v[q], v[q], ss);
 #pragma unroll
-      for (int m = 1; m < LK; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      for (int m = KWP; m < LK * KWP; m <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
       const float g = sqrtf(ss);
       // u_rot = H (s * k) / (gamma sqrt(d)): the signs s (exact) on the raw
       // key, the butterflies, then one scale (0 for a zero key)
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
       for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(__float_as_uint(v[q]) ^ ((smask << (31 - q)) & 0x80000000u));
       // H: coordinate bits 0-4 in registers, then bits 5.. across the key's lanes
       fwht32_regs(v);
-      fwht32_lanes<LK>(v, lane);
+      fwht32_lanes<LK, KWP>(v, lane);
       if (valid) {
         float* row = U + k * US;
 #pragma unroll
