@@ -116,6 +116,19 @@ typedef struct octo_tables {
  * b outside the supported set, OCTO_EINVAL for a NULL L or a bad flag. */
 OCTO_API int octo_layout_init(octo_layout* L, int d, int b, int qjl, int rounding);
 
+/* Fills *L for another split of the bit budget (explainer, "non-uniform bit
+ * allocation": each direction coordinate gets b + delta bits and the triplet
+ * norm b - delta; the OCTOPUS allocation is delta = +1, which
+ * octo_layout_init uses). code_bits = 3b + delta. Supported: b in {2, 3, 4}
+ * with 2 <= b + delta <= 5 and 1 <= b - delta <= 5 for octo_codebook_build;
+ * octo_encode and octo_dequant run delta = +1 for every d and, at d = 128
+ * without the sketch, also b = 3 with delta in {-1, 0, +2} and b = 4 with
+ * delta in {-1, 0} (the sweep the explainer reports); octo_decode_attn runs
+ * delta = +1 only. Other combinations return OCTO_EUNSUPPORTED from the call
+ * that cannot run them; qjl with delta != +1 returns OCTO_EUNSUPPORTED here.
+ * Errors as octo_layout_init. */
+OCTO_API int octo_layout_init_delta(octo_layout* L, int d, int b, int delta, int qjl, int rounding);
+
 /* Host. Lloyd-Max codebooks for layout L (explainer, "triplet
  * decomposition": Lloyd-Max quantisers designed for the marginal law; the
  * abstract: "implementation-matched marginals", data-oblivious). The

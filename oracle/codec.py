@@ -30,9 +30,12 @@ JOINT = 1
 
 @dataclass(frozen=True)
 class Layout:
-    """Sizes that follow from (d, b) ([EXPL] "non-uniform bit allocation")."""
+    """Sizes that follow from (d, b, delta) ([EXPL] "non-uniform bit allocation":
+    each direction coordinate gets b + delta bits, the triplet norm b - delta;
+    OCTOPUS uses delta = +1)."""
     d: int
     b: int
+    delta: int = 1
 
     @property
     def T(self) -> int:
@@ -40,11 +43,11 @@ class Layout:
 
     @property
     def b_dir(self) -> int:
-        return self.b + 1
+        return self.b + self.delta
 
     @property
     def b_rho(self) -> int:
-        return self.b - 1
+        return self.b - self.delta
 
     @property
     def code_bits(self) -> int:
@@ -245,13 +248,14 @@ def direction_cells(field, b: int):
 def pack(i_xi, i_eta, i_rho, lay: Layout) -> np.ndarray:
     """[..., T] ordered cell indices -> [..., W] uint32 words (LSB-first stream).
 
-    Triplet code (3b+1 bits) = direction field (2(b+1) bits, see
-    direction_field) | i_rho << 2(b+1). The code of triplet i occupies
-    stream bits [i c, i c + c), c = 3b+1; stream bit p is bit p mod 32 of
+    Triplet code (c = 2 b_dir + b_rho bits; 3b+1 for the OCTOPUS split) =
+    direction field (2 b_dir bits, see direction_field with b_dir - 1
+    magnitude bits) | i_rho << 2 b_dir. The code of triplet i occupies
+    stream bits [i c, i c + c); stream bit p is bit p mod 32 of
     word p // 32, so a code that crosses a word boundary puts its low bits
     at the top of one word and its high bits at the bottom of the next.
     """
-    code = direction_field(i_xi, i_eta, lay.b) | (np.asarray(i_rho, dtype=np.uint64) << np.uint64(2 * lay.b_dir))
+    code = direction_field(i_xi, i_eta, lay.b_dir - 1) | (np.asarray(i_rho, dtype=np.uint64) << np.uint64(2 * lay.b_dir))
     lead = code.shape[:-1]
     words = np.zeros(lead + (lay.words,), dtype=np.uint64)
     c = lay.code_bits
@@ -280,7 +284,7 @@ def unpack(words: np.ndarray, lay: Layout):
         code[..., i] = v & mask
     m_field = np.uint64((1 << (2 * lay.b_dir)) - 1)
     m_rho = np.uint64((1 << lay.b_rho) - 1)
-    i_xi, i_eta = direction_cells(code & m_field, lay.b)
+    i_xi, i_eta = direction_cells(code & m_field, lay.b_dir - 1)
     i_rho = ((code >> np.uint64(2 * lay.b_dir)) & m_rho).astype(np.int64)
     return i_xi, i_eta, i_rho
 

@@ -40,6 +40,8 @@ _lib = None
 # name -> (restype, argtypes)
 _SIGS = {
     "octo_layout_init": (ctypes.c_int, [ctypes.POINTER(OctoLayout), ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "octo_layout_init_delta": (ctypes.c_int, [ctypes.POINTER(OctoLayout), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int]),
     "octo_codebook_build": (ctypes.c_int, [ctypes.POINTER(OctoLayout)] + [ctypes.c_void_p] * 4),
     "octo_rotation_build": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p]),
     "octo_qjl_build": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p]),

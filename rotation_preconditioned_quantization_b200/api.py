@@ -41,10 +41,12 @@ def _ptr(t) -> int | None:
 class Layout:
     """Sizes of the code for head dimension d and bit budget b (``octo_layout``)."""
 
-    def __init__(self, d: int, b: int, qjl: bool = False, rounding: int = ROUND_JOINT):
+    def __init__(self, d: int, b: int, qjl: bool = False, rounding: int = ROUND_JOINT, delta: int = 1):
+        """delta: the split of the bit budget, b + delta bits per direction coordinate and
+        b - delta for the norm (``octo_layout_init_delta``); +1 is the OCTOPUS allocation."""
         self.c = _lib.OctoLayout()
-        _lib.check(_lib.lib().octo_layout_init(ctypes.byref(self.c), int(d), int(b), int(bool(qjl)), int(rounding)),
-                   "octo_layout_init")
+        _lib.check(_lib.lib().octo_layout_init_delta(ctypes.byref(self.c), int(d), int(b), int(delta), int(bool(qjl)),
+                                                     int(rounding)), "octo_layout_init_delta")
 
     def __getattr__(self, name):
         return getattr(self.__dict__["c"], name)

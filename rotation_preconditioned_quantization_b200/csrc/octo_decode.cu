@@ -85,6 +85,7 @@ int check_layout(const octo_layout* L) {
   if (!L) return OCTO_EINVAL;
   if (L->d != 64 && L->d != 128 && L->d != 256) return OCTO_EUNSUPPORTED;
   if (L->b < 2 || L->b > 4) return OCTO_EUNSUPPORTED;
+  if (L->b_dir != L->b + 1 || L->b_rho != L->b - 1) return OCTO_EUNSUPPORTED;  // fused decode: the OCTOPUS split
   octo_layout chk;
   if (octo_layout_init(&chk, L->d, L->b, L->qjl, L->rounding) != OCTO_OK) return OCTO_EINVAL;
   if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits) return OCTO_EINVAL;

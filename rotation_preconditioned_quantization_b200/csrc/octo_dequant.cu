@@ -46,14 +46,17 @@ struct DequantArgs {
   int64_t tiles_per_head, n_tiles;
 };
 
-template <int D, int B>
+// BD_ bits for each of xi and eta, BR_ for rho (the OCTOPUS allocation is
+// (b + 1, b - 1); other splits serve the bit-allocation sweep).
+template <int D, int BD_, int BR_>
 struct DqCfg {
   static constexpr int T = (D + 2) / 3;
-  static constexpr int BD = B + 1, BR = B - 1;
+  static constexpr int BD = BD_, BR = BR_;
+  static constexpr int B = BD - 1;  // magnitude bits of a direction cell
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
-  static constexpr int NE = 1 << (3 * B - 1);      // positive quadrant: (m_xi, m_eta, i_rho)
+  static constexpr int NE = 1 << (2 * B + BR);     // positive quadrant: (m_xi, m_eta, i_rho)
   static constexpr int REP = NE <= 256 ? 8 : 2;    // replicas: lanes of a quarter-warp in distinct bank groups
   static constexpr int LK = D / 32;                // lanes per key, 32 coordinates each
   static constexpr int LKB = LK == 2 ? 1 : (LK == 4 ? 2 : 3);
@@ -102,9 +105,10 @@ __device__ __forceinline__ void cp_async_commit_wait() {
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
-template <int D, int B>
+template <int D, int BD_, int BR_>
 __global__ void __launch_bounds__(256, 3) dequant_kernel(DequantArgs a) {
-  using Cfg = DqCfg<D, B>;
+  using Cfg = DqCfg<D, BD_, BR_>;
+  constexpr int B = Cfg::B;
   constexpr int C = Cfg::C, W = Cfg::W, KT = Cfg::KT, CS = Cfg::CS, LK = Cfg::LK, LKB = Cfg::LKB, KW = Cfg::KW;
   constexpr int NE = Cfg::NE, REP = Cfg::REP, NWARP = Cfg::NWARP, THREADS = Cfg::THREADS, NT = Cfg::NT;
   constexpr int NWL = Cfg::NWL, WP = Cfg::WP;
@@ -114,7 +118,7 @@ __global__ void __launch_bounds__(256, 3) dequant_kernel(DequantArgs a) {
   float4* table = reinterpret_cast<float4*>(smem_raw);  // [NE][REP]
   uint32_t* cwb = reinterpret_cast<uint32_t*>(smem_raw + Cfg::TABLE);  // [2][WP][CS]
   float* gsb = reinterpret_cast<float*>(smem_raw + Cfg::TABLE + 2 * Cfg::CBUF);  // [2][KT]
-  __shared__ float s_dir_c[32], s_rho_c[8];
+  __shared__ float s_dir_c[32], s_rho_c[32];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j = lane & (LK - 1);  // this lane's coordinates: [32 j, 32 j + 32) of its key
@@ -283,13 +287,13 @@ __global__ void __launch_bounds__(256, 3) dequant_kernel(DequantArgs a) {
   }
 }
 
-template <int D, int B>
+template <int D, int BD, int BR>
 static cudaError_t launch_dequant(const DequantArgs& a0, cudaStream_t st) {
-  using Cfg = DqCfg<D, B>;
+  using Cfg = DqCfg<D, BD, BR>;
   DequantArgs a = a0;
   a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
   a.n_tiles = a.tiles_per_head * a.n_heads;
-  auto kern = dequant_kernel<D, B>;
+  auto kern = dequant_kernel<D, BD, BR>;
   static LaunchCache cache;
   int resident = 0;
   const cudaError_t e = launch_setup(kern, cache, Cfg::THREADS, Cfg::SMEM, resident);
@@ -299,13 +303,21 @@ static cudaError_t launch_dequant(const DequantArgs& a0, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// The OCTOPUS split for every d; at d = 128 also the bit-allocation sweep's
+// other splits (the encoder's set).
 template <int D>
-static cudaError_t dequant_dispatch_b(const DequantArgs& a, int b, cudaStream_t st) {
-  switch (b) {
-    case 2: return launch_dequant<D, 2>(a, st);
-    case 3: return launch_dequant<D, 3>(a, st);
-    default: return launch_dequant<D, 4>(a, st);
+static cudaError_t dequant_dispatch_split(const DequantArgs& a, int b_dir, int b_rho, cudaStream_t st) {
+  if (b_dir == 3 && b_rho == 1) return launch_dequant<D, 3, 1>(a, st);
+  if (b_dir == 4 && b_rho == 2) return launch_dequant<D, 4, 2>(a, st);
+  if (b_dir == 5 && b_rho == 3) return launch_dequant<D, 5, 3>(a, st);
+  if constexpr (D == 128) {
+    if (b_dir == 2 && b_rho == 4) return launch_dequant<D, 2, 4>(a, st);
+    if (b_dir == 3 && b_rho == 3) return launch_dequant<D, 3, 3>(a, st);
+    if (b_dir == 5 && b_rho == 1) return launch_dequant<D, 5, 1>(a, st);
+    if (b_dir == 3 && b_rho == 5) return launch_dequant<D, 3, 5>(a, st);
+    if (b_dir == 4 && b_rho == 4) return launch_dequant<D, 4, 4>(a, st);
   }
+  return cudaErrorNotSupported;
 }
 
 }  // namespace octo
@@ -318,8 +330,13 @@ extern "C" int octo_dequant(const octo_layout* L, const octo_tables* tab, int64_
   if (L->d != 64 && L->d != 128 && L->d != 256) return OCTO_EUNSUPPORTED;
   if (L->b < 2 || L->b > 4) return OCTO_EUNSUPPORTED;
   octo_layout chk;
-  if (octo_layout_init(&chk, L->d, L->b, L->qjl, L->rounding) != OCTO_OK) return OCTO_EINVAL;
-  if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits) return OCTO_EINVAL;
+  const int lc = octo_layout_init_delta(&chk, L->d, L->b, L->b_dir - L->b, L->qjl, L->rounding);
+  if (lc != OCTO_OK) return lc;
+  // the OCTOPUS split for every d; the bit-allocation sweep's splits at d = 128 without the sketch
+  const bool octopus_split = L->b_dir == L->b + 1;
+  if (!octopus_split && (L->d != 128 || L->qjl)) return OCTO_EUNSUPPORTED;
+  if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits || chk.b_rho != L->b_rho)
+    return OCTO_EINVAL;
   if (out_dtype != OCTO_F32 && out_dtype != OCTO_BF16) return OCTO_EINVAL;
   if (n_heads < 0 || n_tokens < 0 || token_offset < 0 || cache_cap < 0) return OCTO_EINVAL;
   if (token_offset + n_tokens > cache_cap) return OCTO_EINVAL;
@@ -346,9 +363,10 @@ extern "C" int octo_dequant(const octo_layout* L, const octo_tables* tab, int64_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   switch (L->d) {
-    case 64: e = dequant_dispatch_b<64>(a, L->b, st); break;
-    case 128: e = dequant_dispatch_b<128>(a, L->b, st); break;
-    default: e = dequant_dispatch_b<256>(a, L->b, st); break;
+    case 64: e = dequant_dispatch_split<64>(a, L->b_dir, L->b_rho, st); break;
+    case 128: e = dequant_dispatch_split<128>(a, L->b_dir, L->b_rho, st); break;
+    default: e = dequant_dispatch_split<256>(a, L->b_dir, L->b_rho, st); break;
   }
+  if (e == cudaErrorNotSupported) return OCTO_EUNSUPPORTED;  // a split without a built kernel (nothing launched)
   return e == cudaSuccess ? OCTO_OK : OCTO_ECUDA;
 }

@@ -52,10 +52,13 @@ struct EncodeArgs {
   int64_t n_tiles, tiles_per_head;
 };
 
-template <int D, int B>
+// BD_ bits for each of xi and eta, BR_ for rho (the OCTOPUS allocation is
+// (b + 1, b - 1); other splits serve the bit-allocation sweep).
+template <int D, int BD_, int BR_>
 struct EncCfg {
   static constexpr int T = (D + 2) / 3;
-  static constexpr int BD = B + 1, BR = B - 1;
+  static constexpr int BD = BD_, BR = BR_;
+  static constexpr int MB = BD - 1;  // magnitude bits of a direction cell
   static constexpr int C = 2 * BD + BR;
   static constexpr int W = (T * C + 31) / 32;
   static constexpr int NDIR = 1 << BD, NRHO = 1 << BR;
@@ -115,9 +118,10 @@ __device__ __forceinline__ void ld_words(const unsigned char* p, uint32_t* w) {
   }
 }
 
-template <int D, int B, bool QJL>
+template <int D, int BD_, int BR_, bool QJL>
 __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) {
-  using Cfg = EncCfg<D, B>;
+  using Cfg = EncCfg<D, BD_, BR_>;
+  constexpr int B = Cfg::MB;  // magnitude bits of a direction cell (b for the OCTOPUS split)
   constexpr int T = Cfg::T, KT = Cfg::KT, US = Cfg::US, W = Cfg::W, C = Cfg::C;
   constexpr int NDIR = Cfg::NDIR, NRHO = Cfg::NRHO;
 
@@ -127,7 +131,7 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
   float4* nhat = reinterpret_cast<float4*>(smem_raw);                 // [NB*NB][REP], cell (ix, iy) at (ix+1, iy+1)
   float* U = reinterpret_cast<float*>(nhat + NB * NB * REP);          // [KT][US]
   uint16_t* codes = reinterpret_cast<uint16_t*>(U + KT * US);         // [KT][T]
-  __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[8], s_rho_t[8];
+  __shared__ float s_dir_c[32], s_dir_t[32], s_rho_c[32], s_rho_t[32];
   // Cell search tables: s_tpad[i] = threshold i - 1 (-inf, +inf at the ends),
   // so cell i is s_tpad[i] <= x < s_tpad[i + 1]; s_bin[k] = the cell of the
   // left edge of bin k of 128 equal bins over [-1, 1]. With at most one
@@ -506,14 +510,14 @@ __global__ void __launch_bounds__(256, QJL ? 2 : 3) encode_kernel(EncodeArgs a) 
   }
 }
 
-template <int D, int B, bool QJL>
+template <int D, int BD, int BR, bool QJL>
 static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
-  using Cfg = EncCfg<D, B>;
+  using Cfg = EncCfg<D, BD, BR>;
   EncodeArgs a = a0;
   a.tiles_per_head = (a.n_tokens + Cfg::KT - 1) / Cfg::KT;
   a.n_tiles = a.tiles_per_head * a.n_heads;
   const size_t smem = Cfg::SMEM;
-  auto kern = encode_kernel<D, B, QJL>;
+  auto kern = encode_kernel<D, BD, BR, QJL>;
   static LaunchCache cache;
   int resident = 0;
   const cudaError_t e = launch_setup(kern, cache, Cfg::THREADS, smem, resident);
@@ -523,18 +527,29 @@ static cudaError_t launch_encode(const EncodeArgs& a0, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int D, int B>
-static cudaError_t dispatch_qjl(const EncodeArgs& a, bool qjl, cudaStream_t st) {
-  return qjl ? launch_encode<D, B, true>(a, st) : launch_encode<D, B, false>(a, st);
-}
-
+// The OCTOPUS split (b + 1, b - 1) for every d, with or without the sketch;
+// at d = 128 also the other splits of the bit-allocation sweep (direction
+// b + delta, norm b - delta for b = 3 with delta in {-1, 0, 2} and b = 4 with
+// delta in {-1, 0}), without the sketch.
 template <int D>
-static cudaError_t dispatch_b(const EncodeArgs& a, int b, bool qjl, cudaStream_t st) {
-  switch (b) {
-    case 2: return dispatch_qjl<D, 2>(a, qjl, st);
-    case 3: return dispatch_qjl<D, 3>(a, qjl, st);
-    default: return dispatch_qjl<D, 4>(a, qjl, st);
+static cudaError_t dispatch_split(const EncodeArgs& a, int b_dir, int b_rho, bool qjl, cudaStream_t st) {
+#define OCTO_ENC(BD, BR)                                                                                 \
+  if (b_dir == BD && b_rho == BR)                                                                      \
+    return qjl ? launch_encode<D, BD, BR, true>(a, st) : launch_encode<D, BD, BR, false>(a, st);
+  OCTO_ENC(3, 1)
+  OCTO_ENC(4, 2)
+  OCTO_ENC(5, 3)
+#undef OCTO_ENC
+  if constexpr (D == 128) {
+    if (!qjl) {
+      if (b_dir == 2 && b_rho == 4) return launch_encode<D, 2, 4, false>(a, st);
+      if (b_dir == 3 && b_rho == 3) return launch_encode<D, 3, 3, false>(a, st);
+      if (b_dir == 5 && b_rho == 1) return launch_encode<D, 5, 1, false>(a, st);
+      if (b_dir == 3 && b_rho == 5) return launch_encode<D, 3, 5, false>(a, st);
+      if (b_dir == 4 && b_rho == 4) return launch_encode<D, 4, 4, false>(a, st);
+    }
   }
+  return cudaErrorNotSupported;
 }
 
 }  // namespace octo
@@ -548,8 +563,13 @@ extern "C" int octo_encode(const octo_layout* L, const octo_tables* tab, const v
   if (L->d != 64 && L->d != 128 && L->d != 256) return OCTO_EUNSUPPORTED;
   if (L->b < 2 || L->b > 4) return OCTO_EUNSUPPORTED;
   octo_layout chk;
-  if (octo_layout_init(&chk, L->d, L->b, L->qjl, L->rounding) != OCTO_OK) return OCTO_EINVAL;
-  if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits) return OCTO_EINVAL;
+  const int lc = octo_layout_init_delta(&chk, L->d, L->b, L->b_dir - L->b, L->qjl, L->rounding);
+  if (lc != OCTO_OK) return lc;
+  // the OCTOPUS split for every d; the bit-allocation sweep's splits at d = 128 without the sketch
+  const bool octopus_split = L->b_dir == L->b + 1;
+  if (!octopus_split && (L->d != 128 || L->qjl)) return OCTO_EUNSUPPORTED;
+  if (chk.words != L->words || chk.T != L->T || chk.code_bits != L->code_bits || chk.b_rho != L->b_rho)
+    return OCTO_EINVAL;
   if (key_dtype != OCTO_F32 && key_dtype != OCTO_BF16) return OCTO_EINVAL;
   if (n_heads < 0 || n_tokens < 0 || token_offset < 0 || cache_cap < 0) return OCTO_EINVAL;
   if (token_offset + n_tokens > cache_cap) return OCTO_EINVAL;
@@ -591,9 +611,10 @@ extern "C" int octo_encode(const octo_layout* L, const octo_tables* tab, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   switch (L->d) {
-    case 64: e = dispatch_b<64>(a, L->b, L->qjl != 0, st); break;
-    case 128: e = dispatch_b<128>(a, L->b, L->qjl != 0, st); break;
-    default: e = dispatch_b<256>(a, L->b, L->qjl != 0, st); break;
+    case 64: e = dispatch_split<64>(a, L->b_dir, L->b_rho, L->qjl != 0, st); break;
+    case 128: e = dispatch_split<128>(a, L->b_dir, L->b_rho, L->qjl != 0, st); break;
+    default: e = dispatch_split<256>(a, L->b_dir, L->b_rho, L->qjl != 0, st); break;
   }
+  if (e == cudaErrorNotSupported) return OCTO_EUNSUPPORTED;  // a split without a built kernel (nothing launched)
   return e == cudaSuccess ? OCTO_OK : OCTO_ECUDA;
 }

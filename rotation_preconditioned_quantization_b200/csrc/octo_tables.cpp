@@ -158,18 +158,21 @@ bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
 
 }  // namespace
 
-extern "C" int octo_layout_init(octo_layout* L, int d, int b, int qjl, int rounding) {
+extern "C" int octo_layout_init_delta(octo_layout* L, int d, int b, int delta, int qjl, int rounding) {
   if (!L) return OCTO_EINVAL;
   if ((qjl != 0 && qjl != 1) || (rounding != OCTO_ROUND_SCALAR && rounding != OCTO_ROUND_JOINT))
     return OCTO_EINVAL;
   if (!supported_d(d) || b < 2 || b > 4) return OCTO_EUNSUPPORTED;
+  const int b_dir = b + delta, b_rho = b - delta;
+  if (b_dir < 2 || b_dir > 5 || b_rho < 1 || b_rho > 5) return OCTO_EUNSUPPORTED;
+  if (qjl && delta != 1) return OCTO_EUNSUPPORTED;  // the sketch is kept for the OCTOPUS split only
   std::memset(L, 0, sizeof(*L));
   L->d = d;
   L->b = b;
   L->T = (d + 2) / 3;
-  L->b_dir = b + 1;
-  L->b_rho = b - 1;
-  L->code_bits = 3 * b + 1;
+  L->b_dir = b_dir;
+  L->b_rho = b_rho;
+  L->code_bits = 2 * b_dir + b_rho;
   L->words = (L->T * L->code_bits + 31) / 32;
   L->n_dir = 1 << L->b_dir;
   L->n_rho = 1 << L->b_rho;
@@ -179,10 +182,18 @@ extern "C" int octo_layout_init(octo_layout* L, int d, int b, int qjl, int round
   return OCTO_OK;
 }
 
+extern "C" int octo_layout_init(octo_layout* L, int d, int b, int qjl, int rounding) {
+  return octo_layout_init_delta(L, d, b, 1, qjl, rounding);
+}
+
 extern "C" int octo_codebook_build(const octo_layout* L, float* dir_c, float* dir_t, float* rho_c,
                                    float* rho_t) {
   if (!L || !dir_c || !dir_t || !rho_c || !rho_t) return OCTO_EINVAL;
   if (!supported_d(L->d) || L->b < 2 || L->b > 4) return OCTO_EUNSUPPORTED;
+  octo_layout chk;
+  const int lc = octo_layout_init_delta(&chk, L->d, L->b, L->b_dir - L->b, L->qjl, L->rounding);
+  if (lc != OCTO_OK) return lc;
+  if (chk.b_rho != L->b_rho || chk.n_dir != L->n_dir || chk.n_rho != L->n_rho) return OCTO_EINVAL;
   try {
     std::vector<double> c, t;
     lloyd_max(xi_marginal, -1.0, 1.0, 0.0, L->n_dir, 1e-14, c, t);

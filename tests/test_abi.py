@@ -219,3 +219,40 @@ def test_split_planner_workspace(B, Hq, Hkv, Lq, d, b, qjl, kv, G):
     assert _lib.lib().octo_decode_attn_workspace(L.ref, B, Hq, Hkv, Lq, kv) == total
     if (B, kv) == (1, 32768):
         assert n_splits == 18  # 8 heads x 18 slices: 144 CTAs, one wave on 148 SMs
+
+
+@pytest.mark.parametrize("b,delta", [(3, -1), (3, 0), (3, 1), (3, 2), (4, -1), (4, 0), (4, 1), (2, 0), (2, 1)])
+def test_layout_init_delta_matches_the_oracle_layout(b, delta):
+    """The split of the bit budget ([EXPL] "non-uniform bit allocation": b + delta bits per direction
+    coordinate, b - delta for the norm) gives the oracle's sizes; delta = +1 is octo_layout_init."""
+    from oracle import codec
+    lay = api.Layout(128, b, delta=delta)
+    ol = codec.Layout(128, b, delta)
+    assert (lay.b_dir, lay.b_rho, lay.code_bits, lay.words, lay.n_dir, lay.n_rho, lay.T) == (
+        ol.b_dir, ol.b_rho, ol.code_bits, ol.words, ol.n_dir, ol.n_rho, ol.T)
+    assert lay.code_bits == 3 * b + delta
+    if delta == 1:
+        ref = api.Layout(128, b)
+        assert bytes(lay.c) == bytes(ref.c)
+
+
+def test_layout_init_delta_refusals_and_decode_split():
+    L = _lib.OctoLayout()
+    f = _lib.lib().octo_layout_init_delta
+    assert f(ctypes.byref(L), 128, 4, 2, 0, 1) == _lib.OCTO_EUNSUPPORTED   # 6 direction bits
+    assert f(ctypes.byref(L), 128, 2, 1, 0, 1) == _lib.OCTO_OK
+    assert f(ctypes.byref(L), 128, 2, 2, 0, 1) == _lib.OCTO_EUNSUPPORTED   # no norm bits
+    assert f(ctypes.byref(L), 128, 3, 0, 1, 1) == _lib.OCTO_EUNSUPPORTED   # the sketch: OCTOPUS split only
+    assert f(None, 128, 3, 0, 0, 1) == _lib.OCTO_EINVAL
+    lib = _lib.lib()
+    T = _lib.OctoTables(256, 256, 256, 256, 256, None, 1)
+    sweep = api.Layout(128, 3, delta=0)
+    # the fused decode runs the OCTOPUS split only; refused before anything is launched
+    assert lib.octo_decode_attn(sweep.ref, ctypes.byref(T), 256, 0, 1, 4, 1, 1, 8, 8, 256, 256, None, None, 256,
+                                ctypes.c_float(0.1), 256, None, 256, 1 << 20, None) == _lib.OCTO_EUNSUPPORTED
+    assert lib.octo_decode_attn_workspace(sweep.ref, 1, 4, 1, 1, 8) == 0
+    # encode / reconstruction of a sweep split exist at d = 128 only
+    off = api.Layout(64, 3, delta=0)
+    assert lib.octo_encode(off.ref, ctypes.byref(T), 256, 0, 1, 4, 64, 64, 4, 0, 256, 256, None, None,
+                           None) == _lib.OCTO_EUNSUPPORTED
+    assert lib.octo_dequant(off.ref, ctypes.byref(T), 1, 4, 4, 0, 256, 256, 256, 0, None) == _lib.OCTO_EUNSUPPORTED

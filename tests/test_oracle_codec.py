@@ -493,3 +493,34 @@ def test_qjl_estimator_variance_matches_closed_form():
     # the sample variance of 3000 draws is within ~3 % (1 sigma) of the true one
     assert np.all(np.abs(corr.var(axis=0) / var - 1.0) < 0.15)
     assert np.all(np.abs(corr.mean(axis=0) - qe) < 4.0 * np.sqrt(var / n_seeds))
+
+
+@pytest.mark.parametrize("b,delta", [(3, -1), (3, 0), (3, 2), (4, -1), (4, 0)])
+def test_pack_round_trip_for_the_sweep_splits(b, delta):
+    """Codes of another split of the bit budget (b + delta direction bits, b - delta norm bits)
+    pack into c = 3b + delta bits a triplet and unpack to the same cells."""
+    lay = codec.Layout(128, b, delta)
+    g = inputs.rng(100 + 10 * b + delta)
+    ix = g.integers(0, lay.n_dir, size=(50, lay.T))
+    iy = g.integers(0, lay.n_dir, size=(50, lay.T))
+    ir = g.integers(0, lay.n_rho, size=(50, lay.T))
+    w = codec.pack(ix, iy, ir, lay)
+    assert w.shape == (50, lay.words) and lay.code_bits == 3 * b + delta
+    bx, by, br = codec.unpack(w, lay)
+    assert np.array_equal(bx, ix) and np.array_equal(by, iy) and np.array_equal(br, ir)
+
+
+def test_pack_by_hand_for_an_even_split():
+    """b = 3, delta = 0: 3 bits per direction coordinate (magnitude 2 bits + sign), 3 for the norm,
+    9 bits a triplet. Triplet 0: xi cell 5 (upper half, m = 1), eta cell 2 (lower, m = 4-1-2 = 1),
+    rho 6 -> 1 | 1 << 2 | 0 << 4 | 1 << 5 | 6 << 6 = 0b110_100_101 = 421.
+    Triplet 1 (cells 0, 7, rho 1): m = 3, s = 1; m = 3, s = 0 -> 3 | 3 << 2 | 1 << 4 | 0 << 5 | 1 << 6 = 95,
+    at bit 9: word 0 = 421 | 95 << 9."""
+    lay = codec.Layout(128, 3, 0)
+    ix = np.zeros((1, lay.T), np.int64); iy = np.zeros((1, lay.T), np.int64); ir = np.zeros((1, lay.T), np.int64)
+    ix[0, :2], iy[0, :2], ir[0, :2] = [5, 0], [2, 7], [6, 1]
+    # the remaining triplets: cells (4, 4), rho 0 -> m = 0, s = 0: code 0
+    ix[0, 2:], iy[0, 2:] = 4, 4
+    w = codec.pack(ix, iy, ir, lay)
+    assert int(w[0, 0]) == 421 | (95 << 9)
+    assert int(w[0].astype(np.int64).sum()) == 421 | (95 << 9)
