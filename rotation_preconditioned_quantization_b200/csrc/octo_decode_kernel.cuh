@@ -836,7 +836,7 @@ struct TcCfg {
   static constexpr int NB = HL ? 2 : 4;      // query B-fragment registers per k-step
   static constexpr int KW = 16;              // keys per consumer chunk (one m-tile)
   static constexpr int QW = D / 32;          // sketch words per key
-  static constexpr int QKS = D / 16;         // sketch k-steps
+  static constexpr int QKS = D / 32;         // sketch k-steps (32 coordinates each, 8-bit operands)
   static constexpr int NWARP = tc_warps(D, B);         // consumer warps
   static constexpr int THREADS = 32 * (NWARP + 1);     // + the producer warp
   static constexpr int NS_MAX = OCTO_DECODE_TC_STAGES;
@@ -906,9 +906,19 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t& r0, uint32_t& r1, uint32
                : "r"(smem_u32(p)));
 }
 
-// +1 / -1 in bf16 (0x3F80 / 0xBF80) for the bits at positions 15 and 31 of x
-// being 1 / 0 (low and high half of the pair).
-__device__ __forceinline__ uint32_t pm1_signs(uint32_t x) { return (x & 0x80008000u) ^ 0xBF80BF80u; }
+// D += A B for one m16n8k32 tile of signed 8-bit operands, 32-bit integer
+// accumulation (exact).
+__device__ __forceinline__ void mma_s8_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four signed bytes +1 / -1 for the bits at positions 2, 6, 10, 14 of x
+// being 1 / 0: a byte permute of (all -1, all +1) with those bits as the
+// selectors (0 picks -1, 4 picks +1).
+__device__ __forceinline__ uint32_t pm1_bytes(uint32_t x) { return __byte_perm(0xFFFFFFFFu, 0x01010101u, x & 0x4444u); }
 
 template <int D, int B, int G, bool QJL>
 __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
@@ -933,6 +943,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   __shared__ float s_dir_c[32];
   __shared__ int s_last;
   __shared__ int s_abort;
+  __shared__ float s_qscale[8];  // OCTOPUS-QJL: per query row scale of the integer sketch projections
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool producer = warp == NWARP;
@@ -1117,28 +1128,48 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
       bq[s][0] = xyh; bq[s][1] = zh; bq[s][NB - 2] = xyl; bq[s][NB - 1] = zl;
     }
   }
-  // Sketch B fragments. The sketch contraction's k order is a relabelling of
-  // the coordinates chosen so that a lane's A fragments are its sketch word
-  // shifted: in k-step ks, lane c4 takes word ks / 2 and bit j0 = 8 (ks & 1) +
-  // 2 c4; k = 2c4, 2c4+1 are the word's bits j0, j0 + 16 and k = 2c4+8, 2c4+9
-  // its bits j0 + 1, j0 + 17 (over the four lanes and two k-steps: all 32 bits).
+  // Sketch B fragments: p_r = S q_rot_r as 16-bit integers v = round(p /
+  // scale_r), scale_r = max_m |p_rm| / 32639, held as signed bytes hi = floor((v
+  // + 128) / 256) and lo = v - 256 hi (so v = 256 hi + lo, |hi| <= 127); the
+  // sketch contraction is exact integer arithmetic on them. Its k order is a
+  // relabelling of the coordinates chosen so that a lane's A fragment is a
+  // byte permute of its sketch word: in k-step ks (word ks), lane c4 takes
+  // bits c4 + 4i (k = 4c4 + i) and 16 + c4 + 4i (k = 4c4 + 16 + i), i < 4;
+  // over the four lanes: all 32 bits.
   uint32_t bp[QJL ? QKS : 1][NB];
+  float qscale0 = 0.0f, qscale1 = 0.0f;  // scales of this lane's query columns q0, q1 (below)
   if constexpr (QJL) {
+    const float* pq = scratch + G * QROW;  // [G][D]
+    if (warp < G) {  // row warp: max |p| -> scale
+      float mx = 0.0f;
+      for (int m = lane; m < D; m += 32) mx = fmaxf(mx, fabsf(pq[warp * D + m]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) s_qscale[warp] = mx / 32639.0f;
+    }
+    __syncthreads();
+    auto qbytes = [&](int r, int m0, bool lo_bytes) -> uint32_t {  // 4 bytes of coordinates m0 + 4i
+      uint32_t w = 0;
+      if (r < G) {
+        const float sc = s_qscale[r], inv = sc > 0.0f ? 1.0f / sc : 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int v = max(-32639, min(32639, __float2int_rn(pq[r * D + m0 + 4 * i] * inv)));
+          const int hi = (v + 128) >> 8, lo = v - 256 * hi;
+          w |= (static_cast<uint32_t>(lo_bytes ? lo : hi) & 0xFFu) << (8 * i);
+        }
+      }
+      return w;
+    };
 #pragma unroll
     for (int ks = 0; ks < QKS; ++ks) {
-      float p0 = 0.0f, p1 = 0.0f, p8 = 0.0f, p9 = 0.0f;
-      if (brow < G) {
-        const float* prow = scratch + G * QROW + brow * D + 32 * (ks >> 1) + 8 * (ks & 1) + 2 * c4;
-        p0 = prow[0]; p1 = prow[16]; p8 = prow[1]; p9 = prow[17];
-      }
-      uint32_t h01, l01, h89, l89;
-      split_bf16x2(p0, p1, h01, l01);
-      split_bf16x2(p8, p9, h89, l89);
+      const int m0 = 32 * ks + c4;
       if constexpr (HL) {
-        bp[ks][0] = blo ? l01 : h01;
-        bp[ks][1] = blo ? l89 : h89;
+        bp[ks][0] = qbytes(brow, m0, blo);
+        bp[ks][1] = qbytes(brow, m0 + 16, blo);
       } else {
-        bp[ks][0] = h01; bp[ks][1] = h89; bp[ks][NB - 2] = l01; bp[ks][NB - 1] = l89;
+        bp[ks][0] = qbytes(brow, m0, false); bp[ks][1] = qbytes(brow, m0 + 16, false);
+        bp[ks][NB - 2] = qbytes(brow, m0, true); bp[ks][NB - 1] = qbytes(brow, m0 + 16, true);
       }
     }
   }
@@ -1167,6 +1198,10 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   // This lane's query columns: HL lanes c4 and c4 ^ 2 hold the same two rows
   // (hi and lo columns before the pairwise add), 8-row lanes rows 2c4, 2c4+1.
   const int q0 = HL ? 2 * (c4 & 1) : 2 * c4, q1 = q0 + 1;
+  if constexpr (QJL) {
+    qscale0 = q0 < G ? s_qscale[q0] : 0.0f;
+    qscale1 = q1 < G ? s_qscale[q1] : 0.0f;
+  }
   const bool owner = !HL || c4 < 2;  // writes this lane's columns (the HL mirror lanes do not)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
   float acc_o[MT][4];
@@ -1214,8 +1249,27 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
         const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + warp * Cfg::CW) + 2 * g8 -
                              (PRESHIFT ? KW : 0);
+        // OCTOPUS-QJL: the sketch contraction runs interleaved with the logit
+        // k-steps (independent work between dependent MMAs), in two
+        // accumulator chains (even and odd sketch k-steps)
+        // integer accumulators: the hi-byte and lo-byte products (the HL
+        // layout keeps both in one, as separate columns)
+        int accq[HL ? 1 : 2][4] = {};
+        const uint32_t* qk = QJL ? reinterpret_cast<const uint32_t*>(st + Cfg::ST_Q) + warp * KW + 2 * g8 : nullptr;
+        auto qjl_step = [&](int ks) {
+          // bits c4 + 4i of word ks move to bit 2 + 4i (a0, a1: bits <= 15, so the
+          // left shift loses none), bits 16 + c4 + 4i likewise by a right shift (a2, a3)
+          const uint2 w2 = *reinterpret_cast<const uint2*>(qk + ks * RK);
+          const uint32_t a0 = pm1_bytes((w2.x << 2) >> c4), a1 = pm1_bytes((w2.y << 2) >> c4);
+          const uint32_t a2 = pm1_bytes(w2.x >> (14 + c4)), a3 = pm1_bytes(w2.y >> (14 + c4));
+          mma_s8_16832(accq[0], a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
+          if constexpr (!HL) mma_s8_16832(accq[HL ? 0 : 1], a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
+        };
   #pragma unroll
         for (int s = 0; s < NKS; ++s) {
+          if constexpr (QJL) {
+            if (s < QKS) qjl_step(s);
+          }
           // the code may straddle words wi and wi + 1; for the last word the
           // next row (the following block of the stage) supplies bits that the mask drops
           const int wi = static_cast<int>(cpos[s] >> 8), sh = static_cast<int>(cpos[s] & 31u);
@@ -1287,25 +1341,23 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
           if constexpr (!HL) v[i] += acc[NC - 1][i];
         }
         if constexpr (QJL) {
-          const uint32_t* qk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_Q) + warp * KW + 2 * g8;
-          float accq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   #pragma unroll
-          for (int ks = 0; ks < QKS; ++ks) {
-            // bits j0 and j0 + 16 of the word move to the sign bits 15 and 31
-            // (bit 1: +1, bit 0: -1); a2, a3 take bits j0 + 1, j0 + 17
-            const uint2 w2 = *reinterpret_cast<const uint2*>(qk + (ks >> 1) * RK);
-            const int shl = 15 - 8 * (ks & 1) - 2 * c4;
-            const uint32_t a0 = pm1_signs(w2.x << shl), a1 = pm1_signs(w2.y << shl);
-            const uint32_t a2 = pm1_signs(w2.x << (shl - 1)), a3 = pm1_signs(w2.y << (shl - 1));
-            mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
-            if constexpr (!HL) mma_bf16_16816(accq, a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
-          }
+          for (int ks = NKS; ks < QKS; ++ks) qjl_step(ks);  // sketch k-steps beyond the logit ones
           const float kq = 1.2533141373155003f / static_cast<float>(D);  // sqrt(pi/2)/m, m = d
           const uint2 nu = *reinterpret_cast<const uint2*>(
               reinterpret_cast<const uint32_t*>(st + Cfg::ST_N) + warp * KW + 2 * g8);
           const float fA = kq * __uint_as_float(nu.x), fB = kq * __uint_as_float(nu.y);
-          v[0] = fmaf(fA, accq[0], v[0]); v[1] = fmaf(fA, accq[1], v[1]);
-          v[2] = fmaf(fB, accq[2], v[2]); v[3] = fmaf(fB, accq[3], v[3]);
+          // the sum over the sketch: scale_r (256 hi-product + lo-product); in the
+          // HL layout lanes c4 < 2 hold the hi products and c4 >= 2 the lo ones,
+          // added by the column shuffle below
+          float sq[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if constexpr (HL) sq[i] = static_cast<float>(accq[0][i]) * (c4 < 2 ? 256.0f : 1.0f);
+            else sq[i] = fmaf(256.0f, static_cast<float>(accq[0][i]), static_cast<float>(accq[HL ? 0 : 1][i]));
+          }
+          v[0] = fmaf(fA * qscale0, sq[0], v[0]); v[1] = fmaf(fA * qscale1, sq[1], v[1]);
+          v[2] = fmaf(fB * qscale0, sq[2], v[2]); v[3] = fmaf(fB * qscale1, sq[3], v[3]);
         }
         if constexpr (HL) {
   #pragma unroll
