@@ -906,19 +906,14 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t& r0, uint32_t& r1, uint32
                : "r"(smem_u32(p)));
 }
 
-// D += A B for one m16n8k32 tile of signed 8-bit operands, 32-bit integer
-// accumulation (exact).
-__device__ __forceinline__ void mma_s8_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+// D += A B for one m16n8k32 tile, A unsigned and B signed 8-bit operands,
+// 32-bit integer accumulation (exact).
+__device__ __forceinline__ void mma_u8s8_16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-
-// Four signed bytes +1 / -1 for the bits at positions 2, 6, 10, 14 of x
-// being 1 / 0: a byte permute of (all -1, all +1) with those bits as the
-// selectors (0 picks -1, 4 picks +1).
-__device__ __forceinline__ uint32_t pm1_bytes(uint32_t x) { return __byte_perm(0xFFFFFFFFu, 0x01010101u, x & 0x4444u); }
 
 template <int D, int B, int G, bool QJL>
 __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
@@ -944,6 +939,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   __shared__ int s_last;
   __shared__ int s_abort;
   __shared__ float s_qscale[8];  // OCTOPUS-QJL: per query row scale of the integer sketch projections
+  __shared__ float s_qsum[8];    // ... and the sum of those integers
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool producer = warp == NWARP;
@@ -1130,31 +1126,39 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   }
   // Sketch B fragments: p_r = S q_rot_r as 16-bit integers v = round(p /
   // scale_r), scale_r = max_m |p_rm| / 32639, held as signed bytes hi = floor((v
-  // + 128) / 256) and lo = v - 256 hi (so v = 256 hi + lo, |hi| <= 127); the
-  // sketch contraction is exact integer arithmetic on them. Its k order is a
-  // relabelling of the coordinates chosen so that a lane's A fragment is a
-  // byte permute of its sketch word: in k-step ks (word ks), lane c4 takes
-  // bits c4 + 4i (k = 4c4 + i) and 16 + c4 + 4i (k = 4c4 + 16 + i), i < 4;
-  // over the four lanes: all 32 bits.
+  // + 128) / 256) and lo = v - 256 hi (so v = 256 hi + lo, |hi| <= 127). The A
+  // operand is the sketch bits themselves as 0/1 bytes, and
+  // sum_m v_m (2 b_m - 1) = 2 sum_m v_m b_m - sum_m v_m, the last a constant of
+  // the row: exact integer arithmetic throughout. The k order is a relabelling
+  // of the coordinates chosen so that a lane's A fragment is its sketch word
+  // shifted and masked: in k-step ks (word ks), lane c4 takes bits c4 + 8i
+  // (k = 4c4 + i) and c4 + 4 + 8i (k = 4c4 + 16 + i), i < 4; over the four
+  // lanes: all 32 bits.
   uint32_t bp[QJL ? QKS : 1][NB];
   float qscale0 = 0.0f, qscale1 = 0.0f;  // scales of this lane's query columns q0, q1 (below)
+  float qsum0 = 0.0f, qsum1 = 0.0f;      // their sum_m v_m
   if constexpr (QJL) {
     const float* pq = scratch + G * QROW;  // [G][D]
-    if (warp < G) {  // row warp: max |p| -> scale
+    if (warp < G) {  // row warp: max |p| -> scale, then sum_m v_m
       float mx = 0.0f;
       for (int m = lane; m < D; m += 32) mx = fmaxf(mx, fabsf(pq[warp * D + m]));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) s_qscale[warp] = mx / 32639.0f;
+      const float sc = mx / 32639.0f, inv = sc > 0.0f ? 1.0f / sc : 0.0f;
+      int vs = 0;
+      for (int m = lane; m < D; m += 32) vs += max(-32639, min(32639, __float2int_rn(pq[warp * D + m] * inv)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vs += __shfl_xor_sync(0xffffffffu, vs, o);
+      if (lane == 0) { s_qscale[warp] = sc; s_qsum[warp] = static_cast<float>(vs); }
     }
     __syncthreads();
-    auto qbytes = [&](int r, int m0, bool lo_bytes) -> uint32_t {  // 4 bytes of coordinates m0 + 4i
+    auto qbytes = [&](int r, int m0, bool lo_bytes) -> uint32_t {  // 4 bytes of coordinates m0 + 8i
       uint32_t w = 0;
       if (r < G) {
         const float sc = s_qscale[r], inv = sc > 0.0f ? 1.0f / sc : 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int v = max(-32639, min(32639, __float2int_rn(pq[r * D + m0 + 4 * i] * inv)));
+          const int v = max(-32639, min(32639, __float2int_rn(pq[r * D + m0 + 8 * i] * inv)));
           const int hi = (v + 128) >> 8, lo = v - 256 * hi;
           w |= (static_cast<uint32_t>(lo_bytes ? lo : hi) & 0xFFu) << (8 * i);
         }
@@ -1166,10 +1170,10 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
       const int m0 = 32 * ks + c4;
       if constexpr (HL) {
         bp[ks][0] = qbytes(brow, m0, blo);
-        bp[ks][1] = qbytes(brow, m0 + 16, blo);
+        bp[ks][1] = qbytes(brow, m0 + 4, blo);
       } else {
-        bp[ks][0] = qbytes(brow, m0, false); bp[ks][1] = qbytes(brow, m0 + 16, false);
-        bp[ks][NB - 2] = qbytes(brow, m0, true); bp[ks][NB - 1] = qbytes(brow, m0 + 16, true);
+        bp[ks][0] = qbytes(brow, m0, false); bp[ks][1] = qbytes(brow, m0 + 4, false);
+        bp[ks][NB - 2] = qbytes(brow, m0, true); bp[ks][NB - 1] = qbytes(brow, m0 + 4, true);
       }
     }
   }
@@ -1201,6 +1205,8 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   if constexpr (QJL) {
     qscale0 = q0 < G ? s_qscale[q0] : 0.0f;
     qscale1 = q1 < G ? s_qscale[q1] : 0.0f;
+    qsum0 = q0 < G ? s_qsum[q0] : 0.0f;
+    qsum1 = q1 < G ? s_qsum[q1] : 0.0f;
   }
   const bool owner = !HL || c4 < 2;  // writes this lane's columns (the HL mirror lanes do not)
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
@@ -1257,13 +1263,12 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         int accq[HL ? 1 : 2][4] = {};
         const uint32_t* qk = QJL ? reinterpret_cast<const uint32_t*>(st + Cfg::ST_Q) + warp * KW + 2 * g8 : nullptr;
         auto qjl_step = [&](int ks) {
-          // bits c4 + 4i of word ks move to bit 2 + 4i (a0, a1: bits <= 15, so the
-          // left shift loses none), bits 16 + c4 + 4i likewise by a right shift (a2, a3)
+          // bits c4 + 8i of word ks to byte i (a0, a1), bits c4 + 4 + 8i likewise (a2, a3)
           const uint2 w2 = *reinterpret_cast<const uint2*>(qk + ks * RK);
-          const uint32_t a0 = pm1_bytes((w2.x << 2) >> c4), a1 = pm1_bytes((w2.y << 2) >> c4);
-          const uint32_t a2 = pm1_bytes(w2.x >> (14 + c4)), a3 = pm1_bytes(w2.y >> (14 + c4));
-          mma_s8_16832(accq[0], a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
-          if constexpr (!HL) mma_s8_16832(accq[HL ? 0 : 1], a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
+          const uint32_t a0 = (w2.x >> c4) & 0x01010101u, a1 = (w2.y >> c4) & 0x01010101u;
+          const uint32_t a2 = (w2.x >> (c4 + 4)) & 0x01010101u, a3 = (w2.y >> (c4 + 4)) & 0x01010101u;
+          mma_u8s8_16832(accq[0], a0, a1, a2, a3, bp[ks][0], bp[ks][1]);
+          if constexpr (!HL) mma_u8s8_16832(accq[HL ? 0 : 1], a0, a1, a2, a3, bp[ks][NB - 2], bp[ks][NB - 1]);
         };
   #pragma unroll
         for (int s = 0; s < NKS; ++s) {
@@ -1347,14 +1352,18 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
           const uint2 nu = *reinterpret_cast<const uint2*>(
               reinterpret_cast<const uint32_t*>(st + Cfg::ST_N) + warp * KW + 2 * g8);
           const float fA = kq * __uint_as_float(nu.x), fB = kq * __uint_as_float(nu.y);
-          // the sum over the sketch: scale_r (256 hi-product + lo-product); in the
-          // HL layout lanes c4 < 2 hold the hi products and c4 >= 2 the lo ones,
-          // added by the column shuffle below
+          // sum_m v_m (2 b_m - 1) = 2 (256 hi-product + lo-product) - sum_m v_m,
+          // times scale_r; in the HL layout lanes c4 < 2 hold the hi products and
+          // c4 >= 2 the lo ones, added by the column shuffle below (the row
+          // constant goes with the hi lanes)
           float sq[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            if constexpr (HL) sq[i] = static_cast<float>(accq[0][i]) * (c4 < 2 ? 256.0f : 1.0f);
-            else sq[i] = fmaf(256.0f, static_cast<float>(accq[0][i]), static_cast<float>(accq[HL ? 0 : 1][i]));
+            const float qs = (i & 1) ? qsum1 : qsum0;
+            if constexpr (HL)
+              sq[i] = c4 < 2 ? fmaf(512.0f, static_cast<float>(accq[0][i]), -qs) : 2.0f * static_cast<float>(accq[0][i]);
+            else
+              sq[i] = fmaf(512.0f, static_cast<float>(accq[0][i]), fmaf(2.0f, static_cast<float>(accq[HL ? 0 : 1][i]), -qs));
           }
           v[0] = fmaf(fA * qscale0, sq[0], v[0]); v[1] = fmaf(fA * qscale1, sq[1], v[1]);
           v[2] = fmaf(fB * qscale0, sq[2], v[2]); v[3] = fmaf(fB * qscale1, sq[3], v[3]);
