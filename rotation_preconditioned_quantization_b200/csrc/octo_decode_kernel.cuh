@@ -746,8 +746,9 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // used. Either way the logits keep about 16 mantissa bits, well inside the
 // logit tolerance. P.V uses the same layouts with P split into hi + lo.
 //
-// Memory pipeline: the CTA's key range is cut into rounds of NWARP chunks of
-// 16 keys, one chunk per consumer warp. A producer warp stages whole rounds
+// Memory pipeline: the CTA's key range is cut into rounds of CPR chunks of
+// 16 keys, one chunk per consumer warp of a team (the consumer warps form
+// NWARP / CPR teams that take the rounds in turn). A producer warp stages whole rounds
 // into a ring of shared-memory stages with a few large tensor copies (TMA:
 // the round's V as two 128-byte-swizzled boxes, its gammas, one code box per
 // chunk), completion counted on the stage's full barrier; the consumer
@@ -760,24 +761,36 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 #ifndef OCTO_DECODE_SR_MIN_B
 #define OCTO_DECODE_SR_MIN_B 4  // bit budgets from which the norm is looked up apart from the direction
 #endif
-#ifndef OCTO_DECODE_TC_STAGES
-#define OCTO_DECODE_TC_STAGES 4  // rounds in flight at most (shared-memory stages; fewer when they do not fit)
+// Rounds in flight at most (shared-memory stages; fewer when they do not fit).
+#ifdef OCTO_DECODE_TC_STAGES
+constexpr int tc_stages(int, int) { return OCTO_DECODE_TC_STAGES; }
+#else
+constexpr int tc_stages(int d, int) { return d <= 64 ? 4 : 6; }
 #endif
 
-// Consumer warps per CTA (one 16-key chunk of every round each). A warp's
-// chunk is a long dependent sequence (code and table reads, MMAs, softmax,
-// P.V), so more warps hide more of it, as far as the stages still fit.
-// Measured best: 10 for d = 128 with b <= 3 (3 stages), 12 for d = 64, and 8
-// for b = 4, whose 64 KB table leaves room for fewer or smaller stages.
-// OCTO_DECODE_TC_WARPS overrides the choice for every configuration.
+// Consumer warps per CTA, and 16-key chunks per round. A warp's chunk is a
+// long dependent sequence (code and table reads, MMAs, softmax, P.V), so
+// more warps hide more of it; the round size sets the stage size, and with
+// it how many rounds fit in flight. When there are more warps than chunks,
+// the warps form teams that take the rounds in turn (team t: rounds t,
+// t + teams, ...), so warps can be added without growing the stages.
+// Measured best: for d = 128, 10 warps in two teams over 5-chunk rounds
+// (6 stages; against 8 warps over 8-chunk rounds, 4 stages: 2 % faster at
+// b = 4 and 3), for d = 64, 12 warps over 12-chunk rounds.
+// OCTO_DECODE_TC_WARPS / OCTO_DECODE_TC_CHUNKS override the choice.
 #ifdef OCTO_DECODE_TC_WARPS
 constexpr int tc_warps(int, int) { return OCTO_DECODE_TC_WARPS; }
 #else
-constexpr int tc_warps(int d, int b) { return b >= 4 ? 8 : (d <= 64 ? 12 : 10); }
+constexpr int tc_warps(int d, int) { return d <= 64 ? 12 : 10; }
+#endif
+#ifdef OCTO_DECODE_TC_CHUNKS
+constexpr int tc_chunks(int, int) { return OCTO_DECODE_TC_CHUNKS; }
+#else
+constexpr int tc_chunks(int d, int) { return d <= 64 ? 12 : 5; }
 #endif
 
 // Keys of one round (the tensor maps' boxes are built for this size).
-constexpr int tc_round_keys(int d, int b) { return 16 * tc_warps(d, b); }
+constexpr int tc_round_keys(int d, int b) { return 16 * tc_chunks(d, b); }
 
 // Tensor maps of one decode call (built on the host; token extents are
 // kv_len, so rows past the end arrive as zeros).
@@ -838,8 +851,11 @@ struct TcCfg {
   static constexpr int QW = D / 32;          // sketch words per key
   static constexpr int QKS = D / 32;         // sketch k-steps (32 coordinates each, 8-bit operands)
   static constexpr int NWARP = tc_warps(D, B);         // consumer warps
+  static constexpr int CPR = tc_chunks(D, B);          // chunks per round
+  static constexpr int NTEAM = NWARP / CPR;            // teams taking the rounds in turn
+  static_assert(NWARP % CPR == 0, "whole teams");
   static constexpr int THREADS = 32 * (NWARP + 1);     // + the producer warp
-  static constexpr int NS_MAX = OCTO_DECODE_TC_STAGES;
+  static constexpr int NS_MAX = tc_stages(D, B);
   static constexpr int RK = tc_round_keys(D, B);  // keys per round
   static constexpr int MT = D / 16, NCH = D / 64;
   // one stage: V (NCH swizzled boxes of RK rows x 128 bytes), per-warp code
@@ -848,7 +864,7 @@ struct TcCfg {
   static constexpr int CW = (4 * W * KW + 127) / 128 * 128;
   static constexpr int ST_V = 0;
   static constexpr int ST_C = ST_V + NCH * VHALF;
-  static constexpr int ST_G = ST_C + NWARP * CW;
+  static constexpr int ST_G = ST_C + CPR * CW;
   static constexpr int ST_Q = ST_G + (4 * RK + 127) / 128 * 128;
   static constexpr int ST_N = ST_Q + (QJL ? 4 * QW * RK : 0);
   static constexpr int ST_END = ST_N + (QJL ? (4 * RK + 127) / 128 * 128 : 0);
@@ -863,8 +879,8 @@ struct TcCfg {
   // shared memory without the stages (+ alignment slack)
   static constexpr size_t REST = NWARP * PBUF + TABLE + SCRATCH + 1024;
   // as many stages as fit, up to NS_MAX
-  static constexpr int NS = REST + size_t(NS_MAX) * STAGE <= BUDGET ? NS_MAX
-                            : REST + 3 * size_t(STAGE) <= BUDGET ? 3 : 2;
+  static constexpr int fit_stages(int n) { return n <= 2 || REST + size_t(n) * STAGE <= BUDGET ? n : fit_stages(n - 1); }
+  static constexpr int NS = fit_stages(NS_MAX);
   static constexpr size_t SREG = 0;                                  // [NS] stages
   static constexpr size_t PREG = SREG + size_t(NS) * STAGE;          // [NWARP] P
   static constexpr size_t TREG = PREG + NWARP * PBUF;                // table
@@ -874,7 +890,7 @@ struct TcCfg {
   static constexpr uint32_t TX_FIXED = (QJL ? 4u * QW * RK + 4u * RK : 0u) + 4u * RK;  // gammas (+ sketch, norms)
   static constexpr uint32_t TX_CHUNK = 4u * W * KW;                                     // one code box
   static_assert(G <= 8 && D <= 128 && NCH >= 1, "tensor-core logits shape");
-  static_assert(NWARP >= 4 && RK <= 256 && NS >= 2, "consumer warps, box rows, stages");
+  static_assert(CPR >= 4 && RK <= 256 && NS >= 2, "chunks per round, box rows, stages");
   static_assert(VHALF % 1024 == 0 && ST_C % 128 == 0 && ST_G % 128 == 0 && ST_Q % 128 == 0 && ST_N % 128 == 0,
                 "alignment of the stage parts");
   static_assert(size_t(NS) * STAGE >= sizeof(float) * NWARP * G * (D + 2), "the warp merge reuses the stages");
@@ -952,7 +968,8 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
 
   const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
   const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
-  // rounds of RK keys; consumer warp w takes keys [16 w, 16 w + 16) of each round
+  // rounds of RK keys; consumer warp w (team w / CPR, chunk cw = w % CPR)
+  // takes keys [16 cw, 16 cw + 16) of every NTEAM-th round
   const int n_rounds = k_end > k_begin ? static_cast<int>((k_end - k_begin + RK - 1) / RK) : 0;
   auto stage_base = [&](int s) { return base + Cfg::SREG + static_cast<size_t>(s) * Cfg::STAGE; };
   float* pw = reinterpret_cast<float*>(base + Cfg::PREG + (producer ? 0 : warp) * Cfg::PBUF);  // [G][PS]
@@ -1006,7 +1023,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NWARP);
+      mbar_init(&empty[s], Cfg::CPR);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int r = 0; r < NS && r < n_rounds; ++r) issue_round(r);
@@ -1234,14 +1251,15 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         if (!mbar_wait_bounded(&full[r % NS], (r / NS) & 1)) aborted = true;
     }
   } else {
-    for (int r = 0; r < n_rounds; ++r) {
+    const int cw = warp % Cfg::CPR;
+    for (int r = warp / Cfg::CPR; r < n_rounds; r += Cfg::NTEAM) {
       const int s = r % NS;
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (r / NS) & 1))) {
         aborted = true;  // warp-uniform
         break;
       }
       const unsigned char* st = stage_base(s);
-      const int64_t s0 = k_begin + static_cast<int64_t>(r) * RK + warp * KW;
+      const int64_t s0 = k_begin + static_cast<int64_t>(r) * RK + cw * KW;
       if (s0 < k_end) {  // warp-uniform: this warp's chunk of the round has keys
       // Logits of the chunk in C-fragment layout. Rows are permuted so that a
       // lane owns 2 consecutive keys: row g8 is key 2 g8, row g8 + 8 is key
@@ -1253,7 +1271,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         float acc[NC][4];
   #pragma unroll
         for (int c = 0; c < NC; ++c) acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.0f;
-        const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + warp * Cfg::CW) + 2 * g8 -
+        const uint32_t* bk = reinterpret_cast<const uint32_t*>(st + Cfg::ST_C + cw * Cfg::CW) + 2 * g8 -
                              (PRESHIFT ? KW : 0);
         // OCTOPUS-QJL: the sketch contraction runs interleaved with the logit
         // k-steps (independent work between dependent MMAs), in two
@@ -1261,7 +1279,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         // integer accumulators: the hi-byte and lo-byte products (the HL
         // layout keeps both in one, as separate columns)
         int accq[HL ? 1 : 2][4] = {};
-        const uint32_t* qk = QJL ? reinterpret_cast<const uint32_t*>(st + Cfg::ST_Q) + warp * KW + 2 * g8 : nullptr;
+        const uint32_t* qk = QJL ? reinterpret_cast<const uint32_t*>(st + Cfg::ST_Q) + cw * KW + 2 * g8 : nullptr;
         auto qjl_step = [&](int ks) {
           // bits c4 + 8i of word ks to byte i (a0, a1), bits c4 + 4 + 8i likewise (a2, a3)
           const uint2 w2 = *reinterpret_cast<const uint2*>(qk + ks * RK);
@@ -1350,7 +1368,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
           for (int ks = NKS; ks < QKS; ++ks) qjl_step(ks);  // sketch k-steps beyond the logit ones
           const float kq = 1.2533141373155003f / static_cast<float>(D);  // sqrt(pi/2)/m, m = d
           const uint2 nu = *reinterpret_cast<const uint2*>(
-              reinterpret_cast<const uint32_t*>(st + Cfg::ST_N) + warp * KW + 2 * g8);
+              reinterpret_cast<const uint32_t*>(st + Cfg::ST_N) + cw * KW + 2 * g8);
           const float fA = kq * __uint_as_float(nu.x), fB = kq * __uint_as_float(nu.y);
           // sum_m v_m (2 b_m - 1) = 2 (256 hi-product + lo-product) - sum_m v_m,
           // times scale_r; in the HL layout lanes c4 < 2 hold the hi products and
@@ -1373,7 +1391,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
           for (int i = 0; i < 4; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);  // hi column + lo column
         }
         const uint2 g2 = *reinterpret_cast<const uint2*>(
-            reinterpret_cast<const uint32_t*>(st + Cfg::ST_G) + warp * KW + 2 * g8);
+            reinterpret_cast<const uint32_t*>(st + Cfg::ST_G) + cw * KW + 2 * g8);
         const float gA = __uint_as_float(g2.x), gB = __uint_as_float(g2.y);
         lgv[0] = v[0] * gA; lgv[1] = v[1] * gA;
         lgv[2] = v[2] * gB; lgv[3] = v[3] * gB;
@@ -1458,7 +1476,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
         // row, which the swizzle keeps at unit ^ (key & 7) (this warp's rows
         // start at a multiple of 8); units 8.. are the second 64-dim box.
         const int vkey = (lane & 7) + ((lane >> 4) << 3);
-        const unsigned char* vrow = st + Cfg::ST_V + (warp * KW + vkey) * 128;
+        const unsigned char* vrow = st + Cfg::ST_V + (cw * KW + vkey) * 128;
   #pragma unroll
         for (int t = 0; t < MT; ++t) {
           const int unit = 2 * t + ((lane >> 3) & 1);
