@@ -675,12 +675,38 @@ DECODE_KERNEL_SOURCES = ("octo_common.cuh", "octo_decode_kernel.cuh", "octo_deco
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_tc_kernel_qjl_long_context_h32x8_d128_ctx131072_b4qjl.md")
 
 
+def _code_tokens(src: str) -> str:
+    """C/C++/CUDA source with its comments removed and whitespace runs collapsed
+    (string and character literals kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_sources_digest(names=DECODE_KERNEL_SOURCES) -> str:
-    """sha256 over the decode kernel's sources (detects a kernel changed since its ncu capture)."""
+    """sha256 over the decode kernel's sources without their comments (detects
+    a kernel changed since its ncu capture; a comment edit does not count)."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "rotation_preconditioned_quantization_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "rotation_preconditioned_quantization_b200", "csrc", n)) as f:
+            h.update(_code_tokens(f.read()).encode())
     return h.hexdigest()
 
 

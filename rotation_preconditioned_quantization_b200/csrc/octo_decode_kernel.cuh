@@ -729,14 +729,21 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
 // mma.sync m16n8k16 bf16 with keys as M, query rows as N and rotated
 // coordinates as K. Each 16-wide k-step holds 4 triplets: lane column c4
 // carries triplet 4s + c4 as (x, y | z, 0), so a lane decodes one triplet
-// code per key per k-step. The shared-memory table holds the decoded
-// triplets rho_hat * n_hat of the positive-level quadrant (codes with both
-// direction signs clear), already split into bf16 hi + lo halves in exactly
-// the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); a code's two
-// direction signs flip the sign bits of x and y in the fragment registers
-// (the codebook is odd-symmetric and the octahedral inverse map is odd in
-// each coordinate, so this is exact). The rotated queries are B fragments
-// held in registers for the whole CTA.
+// code per key per k-step. For b = 3 the shared-memory table holds the
+// decoded triplets rho_hat * n_hat of the positive-level quadrant (codes with
+// both direction signs clear), already split into bf16 hi + lo halves in
+// exactly the A-fragment register order ({xy_hi, z0_hi, xy_lo, z0_lo}); a
+// code's two direction signs flip the sign bits of x and y in the fragment
+// registers (the codebook is odd-symmetric and the octahedral inverse map is
+// odd in each coordinate, so this is exact). b = 2 indexes a table of every
+// signed code, and b = 4 looks up the direction and the signed norm apart
+// (TcCfg). The rotated queries are B fragments held in registers for the
+// whole CTA.
+//
+// OCTOPUS-QJL: the sketch sum <S q_rot, 2 bits - 1> runs on the 8-bit
+// integer tensor cores (mma.sync m16n8k32, unsigned 0/1 sketch bytes x
+// signed bytes of S q_rot rounded per query row to 16 bits), interleaved
+// with the logit k-steps; the integer sums are exact.
 //
 // Precision: with at most 4 query rows (HL layout) the 8 MMA columns hold the
 // rows' bf16 hi halves (columns 0-3) and lo halves (columns 4-7), so two
