@@ -51,6 +51,33 @@ static void choose_splits(int64_t heads, int64_t kv_len, int sms, int64_t unit_b
   n_splits = static_cast<int>(std::max<int64_t>(1, (kv_len + per - 1) / per));
 }
 
+// The slice plan of a call. When the CTAs span several waves and the last
+// one is partly empty, some heads take one slice more (so smaller slices)
+// until the CTAs fill whole waves: heads [0, heads_lo) keep n_lo slices of
+// per_lo keys, heads [heads_lo, heads) take n slices of per keys. Blocks are
+// dispatched in grid order as SMs free up, so the larger slices (lower
+// heads) start first and the smaller ones fill in behind them.
+struct SplitPlan {
+  int n;
+  int64_t per;
+  int heads_lo, n_lo;
+  int64_t per_lo;
+};
+
+static SplitPlan plan_splits(int64_t heads, int64_t kv_len, int sms, int64_t unit_bytes) {
+  int n;
+  int64_t per;
+  choose_splits(heads, kv_len, sms, unit_bytes, n, per);
+  SplitPlan p{n, per, 0, n, per};
+  const int64_t ctas = heads * n, rem = ctas % sms;
+  if (kv_len > 0 && ctas > sms && rem != 0 && sms - rem < heads) {
+    const int64_t per_hi = ((kv_len + n) / (n + 1) + 15) / 16 * 16;
+    if ((kv_len + per_hi - 1) / per_hi == n + 1)
+      p = SplitPlan{n + 1, per_hi, static_cast<int>(heads - (sms - rem)), n, per};
+  }
+  return p;
+}
+
 // Bytes one (token, KV head) costs decode: code words, gamma, V row (and
 // the sketch words and residual norm).
 static int64_t unit_bytes(const octo_layout* L) {
@@ -165,11 +192,9 @@ extern "C" size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq
   const int Gq = (Hq / Hkv) * Lq;
   if (Gq > 8) return 0;
   const int G = octo::rows_template(Gq);
-  int n_splits;
-  int64_t per;
-  octo::choose_splits(static_cast<int64_t>(B) * Hkv, std::max<int64_t>(kv_len, 1), octo::sm_count(), octo::unit_bytes(L),
-                      n_splits, per);
-  return ws_layout(static_cast<int64_t>(B) * Hkv, n_splits, G, L->d).total;
+  const octo::SplitPlan sp = octo::plan_splits(static_cast<int64_t>(B) * Hkv, std::max<int64_t>(kv_len, 1),
+                                               octo::sm_count(), octo::unit_bytes(L));
+  return ws_layout(static_cast<int64_t>(B) * Hkv, sp.n, G, L->d).total;
 }
 
 int octo::decode_validate(const octo_layout* L, const octo_tables* tab, const void* q, int q_dtype, int B, int Hq,
@@ -243,7 +268,12 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.table_heads = tab->n_heads;
   const int G = octo::rows_template(Gq);
 
-  octo::choose_splits(heads, kv_len, octo::sm_count(), octo::unit_bytes(L), a.n_splits, a.keys_per_split);
+  const octo::SplitPlan sp = octo::plan_splits(heads, kv_len, octo::sm_count(), octo::unit_bytes(L));
+  a.n_splits = sp.n;
+  a.keys_per_split = sp.per;
+  a.heads_lo = sp.heads_lo;
+  a.n_splits_lo = sp.n_lo;
+  a.keys_per_split_lo = sp.per_lo;
   const WsLayout w = ws_layout(heads, a.n_splits, G, D);
   if (ws_bytes < w.total) return OCTO_EWORKSPACE;
   char* base = static_cast<char*>(workspace);

@@ -76,8 +76,14 @@ struct DecodeArgs {
   const float* signs;
   const float* qjl_S;
   int64_t table_heads;
+  // Slices of the cache per head: heads [heads_lo, B * Hkv) have n_splits
+  // slices of keys_per_split keys, heads [0, heads_lo) n_splits_lo slices of
+  // keys_per_split_lo keys (n_splits_lo <= n_splits; the grid is n_splits
+  // wide, and the partials take n_splits slots per head).
   int n_splits;
   int64_t keys_per_split;
+  int heads_lo, n_splits_lo;
+  int64_t keys_per_split_lo;
   int* status;
   int* counters;
   float* part_m;
@@ -263,8 +269,12 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   const int64_t trow = bh % a.table_heads;
   const bool with_v = a.V != nullptr;
 
-  const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
-  const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
+  const bool lo_head = bh < a.heads_lo;
+  const int n_sl = lo_head ? a.n_splits_lo : a.n_splits;  // this head's slices
+  const int64_t kps = lo_head ? a.keys_per_split_lo : a.keys_per_split;
+  if (split >= n_sl) return;  // a grid slot this head does not use (nothing touched yet)
+  const int64_t k_begin = static_cast<int64_t>(split) * kps;
+  const int64_t k_end = min(a.kv_len, k_begin + kps);
   // chunks of KW keys, dealt to warps round-robin: warp w takes chunks w, w + NWARP, ...
   const int n_chunks = static_cast<int>((k_end - k_begin + KW - 1) / KW);
   const int my_chunks = warp < n_chunks ? (n_chunks - warp + NWARP - 1) / NWARP : 0;
@@ -653,10 +663,10 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   }
   __syncthreads();
 
-  const int S = a.n_splits;
-  float* pm = a.part_m + (static_cast<int64_t>(bh) * S + split) * G;
-  float* pl = a.part_l + (static_cast<int64_t>(bh) * S + split) * G;
-  float* po = a.part_o + (static_cast<int64_t>(bh) * S + split) * G * D;
+  const int S = n_sl, SW = a.n_splits;  // this head's slices; partial slots per head
+  float* pm = a.part_m + (static_cast<int64_t>(bh) * SW + split) * G;
+  float* pl = a.part_l + (static_cast<int64_t>(bh) * SW + split) * G;
+  float* po = a.part_o + (static_cast<int64_t>(bh) * SW + split) * G * D;
   for (int j = tid; j < G * D; j += Cfg::THREADS) {
     const int r = j / D, d = j - r * D;
     float M = -INFINITY;
@@ -695,9 +705,9 @@ __global__ void __launch_bounds__(DecCfg<D, B, G, QJL>::THREADS, 1) decode_kerne
   }
   __syncthreads();
   if (!s_last) return;
-  const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
-  const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
-  const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
+  const float* bm = a.part_m + static_cast<int64_t>(bh) * SW * G;
+  const float* bl = a.part_l + static_cast<int64_t>(bh) * SW * G;
+  const float* bo = a.part_o + static_cast<int64_t>(bh) * SW * G * D;
   // every thread loads its (row, column)'s S partials plus the row's (m, l)
   // in one round (independent, coalesced over d), then combines them
   for (int j = tid; j < a.Gq * D; j += Cfg::THREADS) {
@@ -973,8 +983,12 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   const int64_t trow = bh % a.table_heads;
   const bool with_v = a.V != nullptr;
 
-  const int64_t k_begin = static_cast<int64_t>(split) * a.keys_per_split;
-  const int64_t k_end = min(a.kv_len, k_begin + a.keys_per_split);
+  const bool lo_head = bh < a.heads_lo;
+  const int n_sl = lo_head ? a.n_splits_lo : a.n_splits;  // this head's slices
+  const int64_t kps = lo_head ? a.keys_per_split_lo : a.keys_per_split;
+  if (split >= n_sl) return;  // a grid slot this head does not use (nothing touched yet)
+  const int64_t k_begin = static_cast<int64_t>(split) * kps;
+  const int64_t k_end = min(a.kv_len, k_begin + kps);
   // rounds of RK keys; consumer warp w (team w / CPR, chunk cw = w % CPR)
   // takes keys [16 cw, 16 cw + 16) of every NTEAM-th round
   const int n_rounds = k_end > k_begin ? static_cast<int>((k_end - k_begin + RK - 1) / RK) : 0;
@@ -1535,10 +1549,10 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   }
   __syncthreads();
 
-  const int S = a.n_splits;
-  float* pm = a.part_m + (static_cast<int64_t>(bh) * S + split) * G;
-  float* pl = a.part_l + (static_cast<int64_t>(bh) * S + split) * G;
-  float* po = a.part_o + (static_cast<int64_t>(bh) * S + split) * G * D;
+  const int S = n_sl, SW = a.n_splits;  // this head's slices; partial slots per head
+  float* pm = a.part_m + (static_cast<int64_t>(bh) * SW + split) * G;
+  float* pl = a.part_l + (static_cast<int64_t>(bh) * SW + split) * G;
+  float* po = a.part_o + (static_cast<int64_t>(bh) * SW + split) * G * D;
   for (int j = tid; j < G * D; j += Cfg::THREADS) {
     const int r = j / D, d = j - r * D;
     float M = -INFINITY;
@@ -1575,9 +1589,9 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   }
   __syncthreads();
   if (!s_last) return;
-  const float* bm = a.part_m + static_cast<int64_t>(bh) * S * G;
-  const float* bl = a.part_l + static_cast<int64_t>(bh) * S * G;
-  const float* bo = a.part_o + static_cast<int64_t>(bh) * S * G * D;
+  const float* bm = a.part_m + static_cast<int64_t>(bh) * SW * G;
+  const float* bl = a.part_l + static_cast<int64_t>(bh) * SW * G;
+  const float* bo = a.part_o + static_cast<int64_t>(bh) * SW * G * D;
   if (S <= 32) {
     // Up to 32 splits (the usual case), one L2 round trip: every thread
     // issues the partial-O loads of its (at most) two outputs; meanwhile
