@@ -186,7 +186,10 @@ def test_status_strings():
 def _planned_workspace(heads, kv_len, d, words, qjl, G, sms=148):
     """Workspace bytes for the split count the planner documents: minimise
     waves(s) * (8 us + keys per slice * unit bytes / 30 GB/s per SM) over
-    s <= min(1024, ceil(kv/64)); slices are rounded up to 16 keys."""
+    s <= min(1024, ceil(kv/64)); slices are rounded up to 16 keys. Then, when
+    the CTAs span several waves and the last is partly empty, as many heads
+    as fill it take one slice more (if that adds a slice), and the partials
+    take that larger count of slots per head."""
     unit = 4 * words + 4 + 2 * d + (4 * (d // 32) + 4 if qjl else 0)
     kv = max(kv_len, 1)
     best, best_s = None, 1
@@ -198,6 +201,11 @@ def _planned_workspace(heads, kv_len, d, words, qjl, G, sms=148):
     per = -(-kv // best_s)
     per = -(-per // 16) * 16
     n_splits = max(1, -(-kv // per))
+    ctas, rem = heads * n_splits, heads * n_splits % sms
+    if kv_len > 0 and ctas > sms and rem and sms - rem < heads:
+        per_hi = -(-(-(-kv // (n_splits + 1))) // 16) * 16
+        if -(-kv // per_hi) == n_splits + 1:
+            n_splits += 1
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
     total = 256 + up(4 * heads) + 2 * up(4 * heads * n_splits * G) + up(4 * heads * n_splits * G * d)
     return n_splits, total
@@ -219,6 +227,9 @@ def test_split_planner_workspace(B, Hq, Hkv, Lq, d, b, qjl, kv, G):
     assert _lib.lib().octo_decode_attn_workspace(L.ref, B, Hq, Hkv, Lq, kv) == total
     if (B, kv) == (1, 32768):
         assert n_splits == 18  # 8 heads x 18 slices: 144 CTAs, one wave on 148 SMs
+    if (B, kv, b) == (8, 131072, 4):
+        # 64 heads x 9 slices = 576 CTAs leave the fourth wave 16 short: 16 heads take 10 slices (592 = 4 x 148)
+        assert n_splits == 10
 
 
 @pytest.mark.parametrize("b,delta", [(3, -1), (3, 0), (3, 1), (3, 2), (4, -1), (4, 0), (4, 1), (2, 0), (2, 1)])
