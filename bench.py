@@ -574,7 +574,8 @@ def run_gpu(args):
     total_ms = t_start.elapsed_time(t_end)
     enc_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    launches = 2 * args.steps
+    # per step: encode, decode (+ the decode's query preparation for the sketch, d <= 128)
+    launches = (3 if w.QJL and w.D <= 128 else 2) * args.steps
 
     total_ms_max = _max_over_ranks(total_ms, ws)
     dec_sum_max = _max_over_ranks(float(np.sum(dec_ms)), ws)

@@ -93,10 +93,17 @@ namespace {
 // Workspace: a status word (own 256-byte line), the per-head arrival
 // counters, then the per-split (m, l) and O partials.
 struct WsLayout {
-  size_t status, counters, m, l, o, total;
+  size_t status, counters, m, l, o, prep, total;
 };
 
-WsLayout ws_layout(int64_t heads, int n_splits, int G, int D) {
+// Floats per head of the OCTOPUS-QJL query preparation (the tensor-core
+// kernel's query scratch image: G rotated rows of tc_qrow(d) floats, then
+// p = S q_rot, G rows of d floats); none otherwise.
+int64_t prep_floats(bool qjl, int G, int D) {
+  return qjl && D <= 128 ? static_cast<int64_t>(G) * (octo::tc_qrow(D) + D) : 0;
+}
+
+WsLayout ws_layout(int64_t heads, int n_splits, int G, int D, bool qjl) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   WsLayout w{};
   w.status = 0;
@@ -104,7 +111,8 @@ WsLayout ws_layout(int64_t heads, int n_splits, int G, int D) {
   w.m = w.counters + up(sizeof(int) * heads);
   w.l = w.m + up(sizeof(float) * heads * n_splits * G);
   w.o = w.l + up(sizeof(float) * heads * n_splits * G);
-  w.total = w.o + up(sizeof(float) * heads * n_splits * G * D);
+  w.prep = w.o + up(sizeof(float) * heads * n_splits * G * D);
+  w.total = w.prep + up(sizeof(float) * heads * prep_floats(qjl, G, D));
   return w;
 }
 
@@ -194,7 +202,7 @@ extern "C" size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq
   const int G = octo::rows_template(Gq);
   const octo::SplitPlan sp = octo::plan_splits(static_cast<int64_t>(B) * Hkv, std::max<int64_t>(kv_len, 1),
                                                octo::sm_count(), octo::unit_bytes(L));
-  return ws_layout(static_cast<int64_t>(B) * Hkv, sp.n, G, L->d).total;
+  return ws_layout(static_cast<int64_t>(B) * Hkv, sp.n, G, L->d, L->qjl != 0).total;
 }
 
 int octo::decode_validate(const octo_layout* L, const octo_tables* tab, const void* q, int q_dtype, int B, int Hq,
@@ -274,7 +282,7 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.heads_lo = sp.heads_lo;
   a.n_splits_lo = sp.n_lo;
   a.keys_per_split_lo = sp.per_lo;
-  const WsLayout w = ws_layout(heads, a.n_splits, G, D);
+  const WsLayout w = ws_layout(heads, a.n_splits, G, D, L->qjl != 0);
   if (ws_bytes < w.total) return OCTO_EWORKSPACE;
   char* base = static_cast<char*>(workspace);
   a.status = reinterpret_cast<int*>(base + w.status);
@@ -282,6 +290,8 @@ extern "C" int octo_decode_attn(const octo_layout* L, const octo_tables* tab, co
   a.part_m = reinterpret_cast<float*>(base + w.m);
   a.part_l = reinterpret_cast<float*>(base + w.l);
   a.part_o = reinterpret_cast<float*>(base + w.o);
+  a.prep = reinterpret_cast<float*>(base + w.prep);
+  a.prep_stride = prep_floats(L->qjl != 0, G, D);
   const dim3 grid(static_cast<unsigned>(a.n_splits), static_cast<unsigned>(heads));
   // tensor maps for the tensor-core kernel (d <= 128)
   octo::TmaDesc tm;

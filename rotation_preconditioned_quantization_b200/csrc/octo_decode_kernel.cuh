@@ -86,6 +86,11 @@ struct DecodeArgs {
   int64_t keys_per_split_lo;
   int* status;
   int* counters;
+  // OCTOPUS-QJL, tensor-core kernel: per KV head, the rotated query rows and
+  // p = S q_rot as the kernel's query scratch image ([G][QROW] then [G][D]
+  // floats, prep_stride floats a head), written by decode_prep_kernel
+  float* prep;
+  int64_t prep_stride;
   float* part_m;
   float* part_l;
   float* part_o;
@@ -806,6 +811,10 @@ constexpr int tc_chunks(int, int) { return OCTO_DECODE_TC_CHUNKS; }
 constexpr int tc_chunks(int d, int) { return d <= 64 ? 12 : 5; }
 #endif
 
+// Floats per rotated query row in the tensor-core kernel's scratch: whole
+// k-steps of 4 triplets (12 floats), at least d + 4.
+constexpr int tc_qrow(int d) { return 12 * (((d + 2) / 3 + 3) / 4) > d + 4 ? 12 * (((d + 2) / 3 + 3) / 4) : d + 4; }
+
 // Keys of one round (the tensor maps' boxes are built for this size).
 constexpr int tc_round_keys(int d, int b) { return 16 * tc_chunks(d, b); }
 
@@ -888,8 +897,12 @@ struct TcCfg {
   static constexpr int STAGE = (ST_END + 1023) / 1024 * 1024;
   static constexpr int PS = KW + 8;          // P row stride (floats)
   static constexpr size_t TABLE = sizeof(uint4) * NE * REP + sizeof(float2) * NSR * REP_SR;
-  static constexpr size_t QROW = (12 * NKS > D + 4 ? 12 * NKS : D + 4);  // padded rotated query row
+  static constexpr size_t QROW = tc_qrow(D);  // padded rotated query row
   static constexpr size_t SCRATCH = (sizeof(float) * G * (QROW + (QJL ? D : 0)) + 15) / 16 * 16;
+  // OCTOPUS-QJL: the query scratch arrives from decode_prep_kernel's output
+  // with the first round (one bulk copy of the whole image)
+  static constexpr uint32_t PREP_BYTES = QJL ? static_cast<uint32_t>(sizeof(float) * G * (QROW + D)) : 0u;
+  static_assert(PREP_BYTES % 16 == 0, "bulk copy size");
   static constexpr size_t PBUF = (sizeof(float) * G * PS + 15) / 16 * 16;  // per consumer warp
   // offsets from a 1024-byte aligned base
   static constexpr size_t BUDGET = 227 * 1024 - 2048;
@@ -1006,8 +1019,10 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
     unsigned char* st = stage_base(s);
     uint64_t* bar = &full[s];
     const int x = static_cast<int>(r0);
+    const bool prep = QJL && r == 0;  // the first round also brings the query scratch image
     mbar_expect_tx(bar, Cfg::TX_FIXED + static_cast<uint32_t>(nch) * Cfg::TX_CHUNK +
-                            (with_v ? static_cast<uint32_t>(NCH * Cfg::VHALF) : 0u));
+                            (with_v ? static_cast<uint32_t>(NCH * Cfg::VHALF) : 0u) + (prep ? Cfg::PREP_BYTES : 0u));
+    if (prep) bulk_g2s(scratch, a.prep + bh * a.prep_stride, Cfg::PREP_BYTES, bar);
     if (with_v) {
 #pragma unroll
       for (int hh = 0; hh < NCH; ++hh) tma_load_3d(st + Cfg::ST_V + hh * Cfg::VHALF, &tm.v, 64 * hh, x, bh, bar);
@@ -1026,7 +1041,7 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   float qraw[E];
   const float dir_v = tid < NDIR ? __ldg(a.dir_c + tid) : 0.0f;
   const float rho_v = tid < Cfg::NRHO ? __ldg(a.rho_c + tid) : 0.0f;
-  if (warp < G && warp < a.Gq) {
+  if (!QJL && warp < G && warp < a.Gq) {
     const int gi = warp / a.Lq, lq = warp - gi * a.Lq;
     const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
     const float* sg = a.signs + trow * D + lane * E;
@@ -1090,53 +1105,23 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
       srt[e] = make_float2((idx & 1) ? -r : r, (idx & 2) ? -r : r);
     }
   }
-  // rotate the query rows: warp r handles row r
-  if (warp < G) {
-    fwht_warp<E>(qraw, lane);
-    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
-    float* qrow = scratch + warp * QROW;
+  if constexpr (QJL) {
+    // the query scratch image (rotated rows, p = S q_rot) lands with the
+    // first round; on a timeout the main loop times out on the same round
+    const bool ok = n_rounds == 0 || mbar_wait_bounded(&full[0], 0);
+    if (!ok && lane == 0) atomicOr(a.status, OCTO_DEVICE_TIMEOUT);
+  } else {
+    // rotate the query rows: warp r handles row r
+    if (warp < G) {
+      fwht_warp<E>(qraw, lane);
+      const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+      float* qrow = scratch + warp * QROW;
 #pragma unroll
-    for (int e = 0; e < E; ++e) qrow[lane * E + e] = qraw[e] * inv_sqrt_d;
-    for (int c = D + lane; c < QROW; c += 32) qrow[c] = 0.0f;  // zero pad to whole k-steps
+      for (int e = 0; e < E; ++e) qrow[lane * E + e] = qraw[e] * inv_sqrt_d;
+      for (int c = D + lane; c < QROW; c += 32) qrow[c] = 0.0f;  // zero pad to whole k-steps
+    }
   }
   __syncthreads();
-  if constexpr (QJL) {
-    // p_r = S q_rot_r. Four lanes share a row m of S, each taking a quarter
-    // of it with 16-byte loads (a warp reads 8 rows, 2 KB contiguous), and
-    // their partial dot products for every query row meet by two shuffles.
-    float* p = scratch + G * QROW;  // [G][D]
-    const float* S = a.qjl_S + trow * D * D;
-    constexpr int NWT = Cfg::THREADS / 32, TPL = D / 4;
-    const int part = lane & 3;
-    for (int m0 = warp * 8; m0 < D; m0 += NWT * 8) {
-      const int m = m0 + (lane >> 2);
-      const float4* srow = reinterpret_cast<const float4*>(S + static_cast<int64_t>(m) * D + part * TPL);
-      float4 sv[TPL / 4];
-#pragma unroll
-      for (int i = 0; i < TPL / 4; ++i) sv[i] = __ldg(srow + i);
-      float acc[G];
-#pragma unroll
-      for (int r = 0; r < G; ++r) {
-        const float4* qv = reinterpret_cast<const float4*>(scratch + r * QROW + part * TPL);
-        float s0 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < TPL / 4; ++i) {
-          const float4 q4 = qv[i];
-          s0 = fmaf(sv[i].x, q4.x, s0);
-          s0 = fmaf(sv[i].y, q4.y, s0);
-          s0 = fmaf(sv[i].z, q4.z, s0);
-          s0 = fmaf(sv[i].w, q4.w, s0);
-        }
-        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-        acc[r] = s0 + __shfl_xor_sync(0xffffffffu, s0, 2);
-      }
-      if (part == 0) {
-#pragma unroll
-        for (int r = 0; r < G; ++r) p[r * D + m] = acc[r];
-      }
-    }
-    __syncthreads();
-  }
 
   // B fragments of the rotated queries: triplet 4s + c4 as (x, y | z, 0) of
   // MMA column g8, i.e. query row g8 & 3, lo half for g8 >= 4 (HL), or row
@@ -1676,6 +1661,66 @@ __global__ void __launch_bounds__(TcCfg<D, B, G, QJL>::THREADS, 1)
   if (tid == 0) atomicExch(a.counters + bh, 0);  // ready for the next call
 }
 
+// OCTOPUS-QJL query preparation for the tensor-core kernel, one block per
+// KV head: the rotated query rows q_rot_r = (1/sqrt(d)) H (s_h * q_r) (zero
+// rows past the group, zero pad to QROW) and p_r = S q_rot_r, written as the
+// decode CTAs' query scratch image. Every CTA of the head then copies the
+// image with its first round instead of reading the head's d x d sketch
+// matrix itself.
+template <int D, int G>
+__global__ void __launch_bounds__(256) decode_prep_kernel(DecodeArgs a) {
+  using Cfg = TcCfg<D, 2, G, true>;  // the scratch layout does not depend on b
+  constexpr int QROW = static_cast<int>(Cfg::QROW), E = D / 32;
+  static_assert(G <= 8, "one warp per query row");
+  __shared__ __align__(16) float q[G][QROW];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x;
+  const int bidx = bh / a.Hkv, hkv = bh - bidx * a.Hkv;
+  const int64_t trow = bh % a.table_heads;
+  float* out = a.prep + bh * a.prep_stride;
+  if (warp < G) {
+    float v[E];
+    if (warp < a.Gq) {
+      const int gi = warp / a.Lq, lq = warp - gi * a.Lq;
+      const int64_t qoff = ((static_cast<int64_t>(bidx) * a.Hq + hkv * a.g + gi) * a.Lq + lq) * D + lane * E;
+      const float* sg = a.signs + trow * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float x = a.q_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q)[qoff + e])
+                                 : static_cast<const float*>(a.q)[qoff + e];
+        v[e] = x * __ldg(sg + e);
+      }
+      fwht_warp<E>(v, lane);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = 0.0f;
+    }
+    const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
+#pragma unroll
+    for (int e = 0; e < E; ++e) q[warp][lane * E + e] = v[e] * inv_sqrt_d;
+    for (int c = D + lane; c < QROW; c += 32) q[warp][c] = 0.0f;
+  }
+  __syncthreads();
+  for (int j = tid; j < G * QROW; j += blockDim.x) out[j] = q[j / QROW][j % QROW];
+  // p: warp w takes rows m = w, w + 8, ... of S; a lane sums D/32 terms, the
+  // warp reduces
+  const float* S = a.qjl_S + trow * D * D;
+  float* p = out + G * QROW;
+  for (int m = warp; m < D; m += blockDim.x / 32) {
+    float sv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) sv[e] = __ldg(S + static_cast<int64_t>(m) * D + lane + 32 * e);
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc = fmaf(sv[e], q[r][lane + 32 * e], acc);
+      acc = warp_sum(acc);
+      if (lane == 0) p[r * D + m] = acc;
+    }
+  }
+}
+
 // Launch one decode instantiation for head dimension D (defined in the
 // per-D translation units so that the templates compile in parallel).
 cudaError_t launch_decode_d64(const DecodeArgs& a, const TmaDesc& tm, int b, int G, bool qjl, dim3 grid, cudaStream_t st);
@@ -1703,6 +1748,7 @@ cudaError_t launch_decode_one(const DecodeArgs& a, const TmaDesc& tm, dim3 grid,
     int resident = 0;
     const cudaError_t e = launch_setup(k, cache, Cfg::THREADS, Cfg::SMEM, resident);
     if (e != cudaSuccess) return e;
+    if constexpr (QJL) decode_prep_kernel<D, G><<<grid.y, 256, 0, st>>>(a);  // one block per head
     k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a, tm);  // grid: (splits, heads)
   } else {
     using Cfg = DecCfg<D, B, G, QJL>;

@@ -208,6 +208,12 @@ def _planned_workspace(heads, kv_len, d, words, qjl, G, sms=148):
             n_splits += 1
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
     total = 256 + up(4 * heads) + 2 * up(4 * heads * n_splits * G) + up(4 * heads * n_splits * G * d)
+    if qjl and d <= 128:
+        # the sketch's query preparation: per head G rotated rows of whole 12-float k-steps (at least d + 4
+        # floats), then G rows of p = S q_rot
+        t = (d + 2) // 3
+        qrow = max(12 * ((t + 3) // 4), d + 4)
+        total += up(4 * heads * G * (qrow + d))
     return n_splits, total
 
 
