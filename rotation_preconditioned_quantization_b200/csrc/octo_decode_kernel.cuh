@@ -1678,6 +1678,15 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(DecodeArgs a) {
   const int bidx = bh / a.Hkv, hkv = bh - bidx * a.Hkv;
   const int64_t trow = bh % a.table_heads;
   float* out = a.prep + bh * a.prep_stride;
+  // warp w takes rows m = w + 8 i of S; all of its loads are issued first
+  // (S does not depend on the query), so they overlap the rotation below
+  constexpr int RPW = D / 8;
+  const float* S = a.qjl_S + trow * D * D;
+  float sv[RPW][E];
+#pragma unroll
+  for (int i = 0; i < RPW; ++i)
+#pragma unroll
+    for (int e = 0; e < E; ++e) sv[i][e] = __ldg(S + static_cast<int64_t>(warp + 8 * i) * D + lane + 32 * e);
   if (warp < G) {
     float v[E];
     if (warp < a.Gq) {
@@ -1702,21 +1711,17 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(DecodeArgs a) {
   }
   __syncthreads();
   for (int j = tid; j < G * QROW; j += blockDim.x) out[j] = q[j / QROW][j % QROW];
-  // p: warp w takes rows m = w, w + 8, ... of S; a lane sums D/32 terms, the
-  // warp reduces
-  const float* S = a.qjl_S + trow * D * D;
+  // p: a lane sums D/32 terms of each row, the warp reduces
   float* p = out + G * QROW;
-  for (int m = warp; m < D; m += blockDim.x / 32) {
-    float sv[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) sv[e] = __ldg(S + static_cast<int64_t>(m) * D + lane + 32 * e);
+  for (int i = 0; i < RPW; ++i) {
 #pragma unroll
     for (int r = 0; r < G; ++r) {
       float acc = 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc = fmaf(sv[e], q[r][lane + 32 * e], acc);
+      for (int e = 0; e < E; ++e) acc = fmaf(sv[i][e], q[r][lane + 32 * e], acc);
       acc = warp_sum(acc);
-      if (lane == 0) p[r * D + m] = acc;
+      if (lane == 0) p[r * D + warp + 8 * i] = acc;
     }
   }
 }
@@ -1748,7 +1753,7 @@ cudaError_t launch_decode_one(const DecodeArgs& a, const TmaDesc& tm, dim3 grid,
     int resident = 0;
     const cudaError_t e = launch_setup(k, cache, Cfg::THREADS, Cfg::SMEM, resident);
     if (e != cudaSuccess) return e;
-    if constexpr (QJL) decode_prep_kernel<D, G><<<grid.y, 256, 0, st>>>(a);  // one block per head
+    if constexpr (QJL) decode_prep_kernel<D, G><<<grid.y, 256, 0, st>>>(a);  // one block (8 warps) per head
     k<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(a, tm);  // grid: (splits, heads)
   } else {
     using Cfg = DecCfg<D, B, G, QJL>;
