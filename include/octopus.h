@@ -206,8 +206,14 @@ OCTO_API size_t octo_decode_attn_workspace(const octo_layout* L, int B, int Hq, 
  *            (the outputs of that call are then invalid). Bytes [256, 256 +
  *            4*B*Hkv) are arrival counters. Status and counters must be zero
  *            before the first call (zero the whole workspace once); every
- *            completed call leaves the counters zero again. Calls that share
- *            a workspace must not overlap on the GPU.
+ *            completed call leaves the counters zero again. The rest is
+ *            the call's scratch (per-slice partial results; with
+ *            layout.qjl and d <= 128 also the rotated queries and S q_rot of
+ *            every KV head). Calls that share a workspace must not overlap
+ *            on the GPU.
+ * The call launches one kernel on `stream`, two with layout.qjl and
+ * d <= 128 (a per-KV-head query preparation into the workspace, then the
+ * decode, which reads it).
  * kv_len == 0 gives out = 0. Errors: OCTO_EINVAL (NULL required pointer,
  * bad sizes, kv_len > cache_cap, both V and logits NULL, misalignment),
  * OCTO_EUNSUPPORTED (g*Lq > 8 or B*Hkv > 65535), OCTO_EWORKSPACE. */
