@@ -13,11 +13,13 @@
 // Because R is orthogonal, q . k_hat = gamma q_rot . u_rot_hat, so the keys
 // are never inverse-rotated.
 //
-// The file holds two kernels. decode_tc_kernel (further below) serves every
-// head dimension up to 128: logits and P.V on tensor cores, whole rounds of
-// keys staged by TMA tensor copies from a producer warp, 8 to 12 consumer
-// warps. decode_kernel, described here, serves d = 256 (where the
-// tensor-core layout does not fit in shared memory):
+// The file holds three kernels. decode_tc_kernel (further below) serves
+// every head dimension up to 128: logits and P.V on tensor cores, whole
+// rounds of keys staged by TMA tensor copies from a producer warp, 10 to 12
+// consumer warps. With OCTOPUS-QJL it is preceded by decode_prep_kernel,
+// which rotates the query rows and forms p = S q_rot once per KV head.
+// decode_kernel, described here, serves d = 256 (where the tensor-core
+// layout does not fit in shared memory):
 //
 // Structure of decode_kernel (one CTA = one KV head x one contiguous slice
 // of the cache, 8 warps, every warp a consumer, thread 0 also the producer):
