@@ -149,6 +149,13 @@ def test_decode_attention_cases(cuda_ok, case):
     _run_case(**case)
 
 
+def test_decode_many_heads_mixed_slice_counts(cuda_ok):
+    """160 KV heads of 300 keys, OCTOPUS-QJL at d=128, b=4. On 148 SMs one slice per head would leave the second
+    wave 136 CTAs short, so the planner gives 136 heads two slices and keeps one for the other 24 (296 CTAs, two
+    whole waves): both kinds of head, and the query preparation of every head, against the oracle."""
+    _run_case(B=2, Hq=320, Hkv=80, Lq=1, d=128, b=4, N=300, qjl=True)
+
+
 def test_decode_rescale_when_the_maximum_jumps(cuda_ok):
     """Keys along the query direction: the first 400 give scaled logits near 0, the rest near 9 (base 2),
     so the running maximum jumps past the slack once; the earlier keys keep a share of about
