@@ -588,39 +588,56 @@ def run_gpu(args):
 
     # end to end through the public API from pinned host buffers: per step the
     # keys, V and queries go host -> device, then encode + decode, then the
-    # output comes back
+    # output comes back. The copies run on their own stream into one of two
+    # device input sets, so that step i + 1's inputs cross PCIe while step i
+    # computes (the way a serving loop overlaps them); every step's copy is
+    # inside the timed region.
     e2e_cache = caches[0]
     hk = s["keys"].cpu().pin_memory()
     hV = s["V"].cpu().pin_memory()
     hq = s["q"].cpu().pin_memory()
     hout = torch.empty_like(s["out"], device="cpu").pin_memory()
-    dk, dV, dq = s["keys"], s["V"], s["q"]
+    sets = [(s["keys"], s["V"], s["q"]),
+            (torch.empty_like(s["keys"]), torch.empty_like(s["V"]), torch.empty_like(s["q"]))]
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event() for _ in sets]
+    freed = [torch.cuda.Event() for _ in sets]
+    for ev in freed:
+        ev.record(stream)
 
-    def e2e_step():
-        dk.copy_(hk, non_blocking=True)
-        dV.copy_(hV, non_blocking=True)
-        dq.copy_(hq, non_blocking=True)
+    def e2e_step(i):
+        dk, dV, dq = sets[i % 2]
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(freed[i % 2])  # the step that last read this set has finished
+            dk.copy_(hk, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            copied[i % 2].record(copy_stream)
+        stream.wait_event(copied[i % 2])
         api.encode(lay, tabs, dk, e2e_cache, 0)
         api.decode_attn(lay, tabs, dq, e2e_cache, dV, w.HKV, kv_len=w.N, out=s["out"], workspace=s["wsp"])
+        freed[i % 2].record(stream)
         hout.copy_(s["out"], non_blocking=True)
 
     e2e_steps = max(1, min(args.steps, 10))
-    for _ in range(max(1, min(args.warmup, 3))):
-        e2e_step()
+    for i in range(max(1, min(args.warmup, 3))):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     _barrier(ws)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    for ev in freed:  # no copy of the timed steps starts before e0
+        ev.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), ws)
     h2d = hk.numel() * 2 + hV.numel() * 2 + hq.numel() * 2
     d2h = hout.numel() * 4
     e2e_val = ws * dbytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
-    del hk, hV
+    del hk, hV, sets
 
     peak, peak_kind = _peaks()
     dec_avg_s = float(np.mean(dec_ms)) * 1e-3
@@ -654,7 +671,9 @@ def run_gpu(args):
                             "hbm_peak": peak, "unit": "GB/s",
                             "hbm_frac": ebytes / (float(np.mean(enc_ms)) * 1e-3) / 1e9 / peak},
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps},
+                "ms_per_step": e2e_ms / e2e_steps, "steps": e2e_steps,
+                "method": "public API from pinned host memory; step i+1's host-to-device copy on a second stream "
+                          "overlaps step i's encode + decode (two device input sets)"},
         "gpu_launches": launches,
         "other_workloads": extra,
         "dequant": dq,
