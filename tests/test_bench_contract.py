@@ -23,3 +23,20 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert "workload" in d["config"]
+
+
+def test_kernel_source_digest_ignores_comments_only():
+    """The digest that ties the committed ncu traffic to the decode sources: a comment or whitespace edit keeps it, a
+    code edit (also inside a string literal, such as an inline-PTX instruction) changes it."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = 'int f(int x) { // the count\n  /* a block\n comment */ asm("add.s32 %0, %1, 1; // not a comment");\n  return x + 1;\n}\n'
+    same = 'int f(int x) {   // another remark\n  asm("add.s32 %0, %1, 1; // not a comment");\n\n  return x + 1;   }\n'
+    code_changed = src.replace("x + 1", "x + 2")
+    string_changed = src.replace("add.s32", "sub.s32")
+    t = bench._code_tokens
+    assert t(src) == t(same)
+    assert t(src) != t(code_changed) and t(src) != t(string_changed)
+    assert "// not a comment" in t(src) and "the count" not in t(src)
+    assert len(bench.kernel_sources_digest()) == 64
